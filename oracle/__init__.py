@@ -1,0 +1,242 @@
+"""CPU oracle for the SageAttention-style 8-bit attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference legs of ``bench.py`` may import this package.  The
+product library never loads it, and this package never imports the product.
+
+The arithmetic lives in ``sage_oracle.c`` (plain C, fp64 / exact integers,
+``-ffp-contract=off``); this module only marshals numpy arrays through ctypes.
+Every function cites the passage it follows on the page "SageAttention:
+Accurate 8-Bit Attention for Plug-and-play Inference Acceleration"
+(research.elamur.ai summary), sections Summary, Key points and Interesting
+ideas.
+
+Parity status (which functions are pinned by checks other than themselves):
+  smooth_k ........ pinned (exact fp64 mean for power-of-two N; shift of K by a
+                    constant; numpy mean within 1 ulp)
+  quant ........... pinned (integer grid identity, round-trip bound, +-127 at the
+                    absmax, all-zero group, numpy-free brute force on tiny cases)
+  qk_int .......... pinned (brute-force Python loops; int64 numpy matmul)
+  attn ............ pinned (identity-quantizer special case vs exact fp64
+                    attention within the fp16 error bound; causal row 0 equals
+                    V[0]; causal rows ignore later keys; rows of P sum to 1)
+  attn_fp64 ....... pinned (softmax shift invariance; hand-derived closed forms
+                    in tests/golden)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sage_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libsage_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GROUP_PER_TOKEN = (1, 1)
+GROUP_PER_BLOCK = (128, 64)  # (Q tokens, K tokens) per quantization group
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no FMA contraction, OpenMP)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64, i32, f64, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+            lib.oracle_smooth_k.argtypes = [vp, i64, i64, i64, vp]
+            lib.oracle_quant.argtypes = [vp, vp, i64, i64, i64, i64, vp, vp]
+            lib.oracle_qk_int.argtypes = [vp, vp, i64, i64, i64, vp]
+            lib.oracle_attn.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f64, i64, i64, vp, vp]
+            lib.oracle_attn_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp,
+                                             i64, vp, vp]
+            lib.oracle_attn_probs.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp]
+            lib.oracle_attn_fp64.argtypes = [vp, vp, vp, i64, i64, i64, i32, f64, vp]
+            lib.oracle_round_fp16.argtypes = [vp, i64, vp]
+            lib.oracle_round_fp16.restype = None
+            for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_attn",
+                         "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
+                getattr(lib, name).restype = i32
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _as_fp16_bits(x) -> np.ndarray:
+    """Accept a numpy float16 array or a torch fp16 tensor; return uint16 bits."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().contiguous().numpy()
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float16:
+        return x.view(np.uint16)
+    if x.dtype == np.uint16:
+        return x
+    raise TypeError(f"expected fp16 data, got {x.dtype}")
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"{name} failed with status {rc}")
+
+
+def _bhnd(x: np.ndarray):
+    if x.ndim == 4:
+        B, H, N, d = x.shape
+        return B * H, N, d
+    if x.ndim == 3:
+        return x.shape
+    raise ValueError("expected [B,H,N,d] or [BH,N,d]")
+
+
+def smooth_k(k) -> np.ndarray:
+    """Per-(b,h) channel mean of K over tokens (Summary bullet 1; idea I1).
+
+    Returns fp32 [*lead, d] where lead = k.shape[:-2]."""
+    kb = _as_fp16_bits(k)
+    BH, N, d = _bhnd(kb)
+    km = np.empty(kb.shape[:-2] + (d,), np.float32)
+    _check(_load().oracle_smooth_k(_ptr(kb), BH, N, d, _ptr(km)), "oracle_smooth_k")
+    return km
+
+
+def scale_count(N: int, g: int) -> int:
+    return (N + g - 1) // g
+
+
+def quant(x, g: int, mu=None):
+    """Symmetric absmax INT8 quantization over groups of g tokens (Summary
+    bullet 1; Key points on per-token granularity).  mu: optional fp32 channel
+    mean subtracted first (K smoothing).  Returns (int8 codes, fp32 scales)."""
+    xb = _as_fp16_bits(x)
+    BH, N, d = _bhnd(xb)
+    q = np.empty(xb.shape, np.int8)
+    s = np.empty(xb.shape[:-2] + (scale_count(N, g),), np.float32)
+    mu_arr = None
+    if mu is not None:
+        mu_arr = np.ascontiguousarray(mu, dtype=np.float32)
+        if mu_arr.size != BH * d:
+            raise ValueError("mu must hold one value per (head, channel)")
+    _check(_load().oracle_quant(_ptr(xb), _ptr(mu_arr) if mu_arr is not None else None, BH, N, d, g,
+                                _ptr(q), _ptr(s)), "oracle_quant")
+    return q, s
+
+
+def qk_int(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:
+    """Exact integer q8 . k8^T per head (int64 [*lead, N, N])."""
+    q8 = np.ascontiguousarray(q8, np.int8)
+    k8 = np.ascontiguousarray(k8, np.int8)
+    BH, N, d = _bhnd(q8)
+    S = np.empty(q8.shape[:-1] + (N,), np.int64)
+    _check(_load().oracle_qk_int(_ptr(q8), _ptr(k8), BH, N, d, _ptr(S)), "oracle_qk_int")
+    return S
+
+
+def attn(q8, k8, sq, sk, v, causal: bool, sm_scale: float, groups=GROUP_PER_TOKEN):
+    """Quantized attention: dequantized scores, fp64 softmax, P rounded to fp16,
+    fp64 P.V (Summary bullets 1-2).  Returns (O fp64, O fp16)."""
+    q8 = np.ascontiguousarray(q8, np.int8)
+    k8 = np.ascontiguousarray(k8, np.int8)
+    sq = np.ascontiguousarray(sq, np.float32)
+    sk = np.ascontiguousarray(sk, np.float32)
+    vb = _as_fp16_bits(v)
+    BH, N, d = _bhnd(vb)
+    o64 = np.empty(vb.shape, np.float64)
+    o16 = np.empty(vb.shape, np.uint16)
+    gq, gk = groups
+    _check(_load().oracle_attn(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(vb), BH, N, d,
+                               int(bool(causal)), float(sm_scale), gq, gk, _ptr(o64), _ptr(o16)),
+           "oracle_attn")
+    return o64, o16.view(np.float16)
+
+
+def attn_rows(q8h, k8h, sqh, skh, vh, rows, causal: bool, sm_scale: float, groups=GROUP_PER_TOKEN):
+    """Like attn() for one head [N,d] but only for the listed query rows."""
+    q8h = np.ascontiguousarray(q8h, np.int8)
+    k8h = np.ascontiguousarray(k8h, np.int8)
+    sqh = np.ascontiguousarray(sqh, np.float32)
+    skh = np.ascontiguousarray(skh, np.float32)
+    vb = _as_fp16_bits(vh)
+    N, d = vb.shape
+    rows = np.ascontiguousarray(rows, np.int64)
+    o64 = np.empty((rows.size, d), np.float64)
+    o16 = np.empty((rows.size, d), np.uint16)
+    gq, gk = groups
+    _check(_load().oracle_attn_rows(_ptr(q8h), _ptr(k8h), _ptr(sqh), _ptr(skh), _ptr(vb), N, d,
+                                    int(bool(causal)), float(sm_scale), gq, gk, _ptr(rows),
+                                    rows.size, _ptr(o64), _ptr(o16)), "oracle_attn_rows")
+    return o64, o16.view(np.float16)
+
+
+def attn_probs(q8h, k8h, sqh, skh, vh, causal: bool, sm_scale: float, groups=GROUP_PER_TOKEN):
+    """Normalized softmax probabilities of one head (N x N fp64)."""
+    q8h = np.ascontiguousarray(q8h, np.int8)
+    k8h = np.ascontiguousarray(k8h, np.int8)
+    sqh = np.ascontiguousarray(sqh, np.float32)
+    skh = np.ascontiguousarray(skh, np.float32)
+    vb = _as_fp16_bits(vh)
+    N, d = vb.shape
+    P = np.empty((N, N), np.float64)
+    gq, gk = groups
+    _check(_load().oracle_attn_probs(_ptr(q8h), _ptr(k8h), _ptr(sqh), _ptr(skh), _ptr(vb), N, d,
+                                     int(bool(causal)), float(sm_scale), gq, gk, _ptr(P)),
+           "oracle_attn_probs")
+    return P
+
+
+def attn_fp64(q, k, v, causal: bool, sm_scale: float) -> np.ndarray:
+    """Exact (unquantized) attention in fp64 (idea I5's tensor-level reference)."""
+    qb, kb, vb = _as_fp16_bits(q), _as_fp16_bits(k), _as_fp16_bits(v)
+    BH, N, d = _bhnd(qb)
+    o = np.empty(qb.shape, np.float64)
+    _check(_load().oracle_attn_fp64(_ptr(qb), _ptr(kb), _ptr(vb), BH, N, d, int(bool(causal)),
+                                    float(sm_scale), _ptr(o)), "oracle_attn_fp64")
+    return o
+
+
+def round_fp16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    _load().oracle_round_fp16(_ptr(x), x.size, _ptr(out))
+    return out.view(np.float16)
+
+
+def sage_attn(q, k, v, causal: bool, sm_scale: float, per_block: bool, smooth: bool = True):
+    """The whole method in the page's order: smooth K, quantize Q and K, then
+    attention (Summary bullets 1-2).  Returns a dict with every intermediate."""
+    gq, gk = GROUP_PER_BLOCK if per_block else GROUP_PER_TOKEN
+    km = smooth_k(k) if smooth else None
+    q8, sq = quant(q, gq)
+    k8, sk = quant(k, gk, km)
+    o64, o16 = attn(q8, k8, sq, sk, v, causal, sm_scale, (gq, gk))
+    return dict(km=km, q8=q8, sq=sq, k8=k8, sk=sk, o64=o64, o16=o16)
+
+
+def metrics(a: np.ndarray, b: np.ndarray) -> dict:
+    """Tensor-level accuracy metrics named by idea I5: cosine similarity,
+    relative L1 (sum|a-b| / sum|b|) and RMSE, with b the reference."""
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
+    cos = float(np.dot(a, b) / (np.linalg.norm(a) * np.linalg.norm(b)))
+    rel_l1 = float(np.abs(a - b).sum() / np.abs(b).sum())
+    rmse = float(np.sqrt(np.mean((a - b) ** 2)))
+    return dict(cos=cos, rel_l1=rel_l1, rmse=rmse)
