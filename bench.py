@@ -1,0 +1,335 @@
+"""Benchmark of the SageAttention-style 8-bit attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = the whole method on one batch of synthetic input resident in HBM:
+smooth K -> quantize Q and K -> fused INT8 Q.K^T / online softmax / FP16 P.V
+attention (``sage_attn_fwd``, the call a user makes).  Default workload: B=1,
+H=64, N=16384, d=128, non-causal, per-block INT8 (the N=16k, d=128 point of the
+B*H*N = 2^20-token sweep), Gaussian Q/V and K with +-20 bias on 4 channels.
+
+Metric: TOPS = 4 N^2 d B H / t (halved when causal).  Rank 0 prints one JSON
+line.  Under torchrun every rank runs its own independent batch (heads are
+independent problems: no collective on the data path), so ``value`` is the
+total work of all ranks over the slowest rank's time ("scaling": "weak").
+
+``--impl reference`` times the CPU oracle (the plain C implementation under
+oracle/) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "SageAttn fwd TOPS (4N²d·BH/time) at N=16k,d=128; % of INT8+FP16 roofline"
+UNIT = "TOPS"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def mixed_peak_tops(p_f16: float) -> float:
+    """Effective TOPS of the mixed roofline: half the attention ops (Q.K^T) at the INT8
+    tensor peak, half (P.V) at the FP16 one; INT8 = 2x FP16 (dense datasheet ratio)."""
+    p_i8 = 2.0 * p_f16
+    return 4.0 / (2.0 / p_i8 + 2.0 / p_f16)
+
+
+# ------------------------------------------------------------------ clocks sampler
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([c.strip() for c in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(w: W.Workload, budget_s: float = 12.0):
+    """Time the CPU oracle (smooth K, quantize, attention) on a bounded sample of the
+    workload: one head, R query rows; the rate is scaled to TOPS by the rows' share of
+    the attention work.  Returns (tops, cores, description)."""
+    import numpy as np
+
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    q, k, v = W.make_qkv(W.Workload(w.name + "_head", 1, 1, w.N, w.d, w.causal, w.per_block, w.q_std,
+                                    w.bias_std, w.n_out, w.out_mag))
+    gq, gk = oracle.GROUP_PER_BLOCK if w.per_block else oracle.GROUP_PER_TOKEN
+    t0 = time.perf_counter()
+    km = oracle.smooth_k(k)
+    q8, sq = oracle.quant(q, gq)
+    k8, sk = oracle.quant(k, gk, km)
+    t_prep = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(w.N, size=min(w.N, max(cores, 8)), replace=False)).astype(np.int64)
+    t1 = time.perf_counter()
+    oracle.attn_rows(q8[0, 0], k8[0, 0], sq[0, 0], sk[0, 0], v[0, 0], rows, w.causal, w.sm_scale, (gq, gk))
+    t_probe = time.perf_counter() - t1
+    n = int(min(w.N, max(rows.size, rows.size * max(1.0, (budget_s - t_prep) / max(t_probe, 1e-3)))))
+    rows = np.sort(rng.choice(w.N, size=n, replace=False)).astype(np.int64)
+    t2 = time.perf_counter()
+    oracle.attn_rows(q8[0, 0], k8[0, 0], sq[0, 0], sk[0, 0], v[0, 0], rows, w.causal, w.sm_scale, (gq, gk))
+    t_rows = time.perf_counter() - t2
+    # attention ops of the sampled rows (causal rows see i+1 keys)
+    keys = (rows + 1).sum() if w.causal else rows.size * w.N
+    ops = 4.0 * keys * w.d
+    # prep cost charged pro rata to the sampled share of one head's work
+    head_ops = 4.0 * w.N * w.N * w.d / (2 if w.causal else 1)
+    t = t_rows + t_prep * (ops / head_ops)
+    desc = (f"oracle (plain C, OpenMP) on 1 head of {w.name}: smooth+quantize the head, then attention for "
+            f"{rows.size} of {w.N} query rows; {t:.1f} s")
+    return ops / t / 1e12, cores, desc
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, w: W.Workload):
+    import torch.distributed as dist
+
+    import quantized_attention_02_b200 as sa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    gran = sa.SAGE_PER_BLOCK if w.per_block else sa.SAGE_PER_TOKEN
+    # every rank draws its own batch (seed = rank): independent problems
+    qh, kh, vh = W.make_qkv(w, seed=rank)
+    q, k, v = qh.to(dev), kh.to(dev), vh.to(dev)
+    o = torch.empty_like(q)
+    km, q8, k8, sq, sk = sa.empty_quantized(q, gran)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def step():
+        sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if sa.sage_last_device_error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out during warm-up")
+
+    # ---- headline: K whole steps, inputs resident (each input 2*B*H*N*d bytes > L2)
+    clocks = ClockSampler(dev.index if world == 1 else local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # ---- the fused kernel alone (already-quantized inputs), same stream, for the roofline
+    sa.sage_smooth_k(k, km, stream)
+    sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream)
+    for _ in range(3):
+        sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
+    torch.cuda.synchronize(dev)
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(args.steps):
+        sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
+    k1.record(stream)
+    torch.cuda.synchronize(dev)
+    kernel_ms = k0.elapsed_time(k1) / args.steps
+
+    # ---- end to end through the C ABI with host buffers: H2D inputs, D2H output per step
+    qp, kp, vp = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
+    op = torch.empty_like(qp).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+        op.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = x0.elapsed_time(x1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if sa.sage_last_device_error(stream) != 0:
+        raise RuntimeError("a kernel wait timed out during timing")
+
+    result = None
+    if rank == 0:
+        peaks, src = load_peaks()
+        ops = w.ops()
+        value = world * ops / (ms_max * 1e-3) / 1e12
+        p_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        p_burst = float(peaks["bf16_tflops"])
+        peak = mixed_peak_tops(p_sus)
+        achieved = ops / (kernel_ms * 1e-3) / 1e12
+        traffic = _traffic_from_profiles(w)
+        cpu_tops, cores, desc = oracle_sample(w)
+        elem_bytes = w.BH * w.N * w.d * 2
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8+f16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                       "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
+                       "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default)",
+                       "parallelism": f"independent batch per rank x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "sage_attn_kernel", "achieved": round(achieved, 2),
+                         "peak": round(peak, 2), "unit": "TOPS", "frac": round(achieved / peak, 4),
+                         "traffic": traffic,
+                         "peak_note": (f"mixed INT8+FP16 roofline from the {src} sustained bf16 peak "
+                                       f"{p_sus} TFLOP/s (INT8 = 2x): {peak:.1f} TOPS; with the burst peak "
+                                       f"{p_burst}: {mixed_peak_tops(p_burst):.1f} TOPS "
+                                       f"(frac {achieved / mixed_peak_tops(p_burst):.4f})"),
+                         "kernel_ms": round(kernel_ms, 4)},
+            "cpu_baseline": {"value": cpu_tops, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def _traffic_from_profiles(w):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, if it was
+    taken on this workload with the current kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get(w.name)
+    except (OSError, ValueError):
+        return None
+
+
+def run_reference(args, w: W.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    samples = []
+    for i in range(args.warmup + args.steps):
+        tops, cores, desc = oracle_sample(w, budget_s=4.0)
+        if i >= args.warmup:
+            samples.append(tops)
+    value = statistics.median(samples)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64+f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = W.ALL[args.workload]
+    res = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,110 @@
+/*
+ * sage_attn.h -- C ABI of the B200 (sm_100a) SageAttention-style 8-bit attention library.
+ *
+ * The operation follows "SageAttention: Accurate 8-Bit Attention for Plug-and-play
+ * Inference Acceleration" (research.elamur.ai summary page):
+ *   O = softmax(Q K^T * sm_scale) V, where
+ *   - K is first smoothed by subtracting its per-channel mean over tokens
+ *     (Summary, first bullet; Interesting idea I1: a component shared by all tokens of K
+ *     can be removed without changing the softmax);
+ *   - Q and K are quantized to INT8 with absmax scales (Summary, first bullet;
+ *     Key points: per-token granularity), here per token or per block of tokens;
+ *   - Q K^T runs as an INT8 matrix product with INT32 accumulation and is dequantized by
+ *     scale_q * scale_k * sm_scale;
+ *   - softmax runs online over key/value tiles, FlashAttention-style (Summary: the kernels
+ *     follow FlashAttention-style tiling);
+ *   - P V runs on 16-bit floating-point operands (Summary, second bullet), P rounded to fp16.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are device memory owned by the caller, dense and contiguous in the order
+ *     [B][H][N][d] ("BHND").  Q, K, V and O are IEEE fp16.  q8/k8 are int8 with the same
+ *     layout.  km is fp32 [B][H][d].  Scales are fp32 [B][H][G] with
+ *     G = sage_scale_count(N, granularity, is_q).
+ *   - granularity SAGE_PER_TOKEN: one scale per token (G = N);
+ *     SAGE_PER_BLOCK: one scale per 128 consecutive Q tokens / 64 consecutive K tokens.
+ *   - d must be 64 or 128; N must be a positive multiple of 128; B, H >= 1;
+ *     B*H*N*d must stay below 2^31.  sm_scale must be finite and > 0.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls only enqueue work:
+ *     they never synchronize the host.  Arguments are validated before anything is
+ *     enqueued; an invalid call returns an error and launches nothing.
+ *   - Return value: SAGE_OK (0) or a negative sage_status.  A kernel whose bounded
+ *     internal wait gave up leaves a code readable with sage_last_device_error().
+ *   - Inputs must not alias outputs.  Non-finite inputs give unspecified (but bounded,
+ *     non-faulting) results.
+ */
+#ifndef SAGE_ATTN_H
+#define SAGE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID = -1,     /* null pointer, bad size, bad sm_scale, bad granularity */
+  SAGE_ERR_UNSUPPORTED = -2, /* valid request outside what the kernels implement (d, N) */
+  SAGE_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  SAGE_ERR_TIMEOUT = -4,     /* a kernel's bounded wait gave up (sage_last_device_error) */
+  SAGE_ERR_NOMEM = -5        /* workspace allocation failed */
+} sage_status;
+
+enum { SAGE_PER_TOKEN = 0, SAGE_PER_BLOCK = 1 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sage_status_string(int status);
+
+/* Number of scales per (b,h): N for per-token; ceil(N/128) for Q and ceil(N/64) for K
+ * per-block.  Returns 0 for an unknown granularity or N <= 0. */
+size_t sage_scale_count(int N, int granularity, int is_q);
+
+/* K smoothing (Summary, first bullet; idea I1).
+ * km[b,h,c] = mean over the N tokens of K[b,h,:,c], computed from the exact sum
+ * (fixed point, order independent) as fl32(fl32(sum) / N).
+ * k: fp16 [B,H,N,d] (in); km: fp32 [B,H,d] (out). */
+int sage_smooth_k(const void* k, float* km, int B, int H, int N, int d, void* stream);
+
+/* INT8 quantization of Q and K (Summary, first bullet; Key points: per-token).
+ * For every group (one token, or 128 Q / 64 K consecutive tokens, all d channels):
+ *   x = Q, or x = fl32(K - km) when km != NULL (no smoothing when km == NULL);
+ *   a = max|x|; scale = fl32(a/127); code = clamp(round_half_even(fl32(x * fl32(127/a))), +-127)
+ *   (a == 0: scale 0, codes 0).
+ * q, k: fp16 [B,H,N,d] (in); km: fp32 [B,H,d] or NULL (in);
+ * q8, k8: int8 [B,H,N,d] (out); sq: fp32 [B,H,Gq], sk: fp32 [B,H,Gk] (out). */
+int sage_quant_qk(const void* q, const void* k, const float* km, int8_t* q8, int8_t* k8, float* sq,
+                  float* sk, int B, int H, int N, int d, int granularity, void* stream);
+
+/* The whole forward pass as a user calls it: smooth K, quantize Q and K, fused attention.
+ * q, k, v: fp16 [B,H,N,d] (in); o: fp16 [B,H,N,d] (out).  causal: keys j > i masked
+ * (top-left aligned).  Workspace (int8 Q/K, scales, km: 2*B*H*N*d bytes plus scales) is
+ * allocated and freed stream-ordered (cudaMallocAsync / cudaFreeAsync) inside the call. */
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                  int causal, float sm_scale, int granularity, void* stream);
+
+/* The fused attention kernel alone, on already-quantized inputs (Summary bullets 1-2):
+ * S = (q8 k8^T) * sq * sk * sm_scale with INT32 accumulation on the tensor cores, online
+ * softmax in fp32 with exp2, P rounded to fp16, O = P V with fp16 operands and fp32
+ * accumulation, O stored as fp16.  q8, k8: int8 [B,H,N,d]; sq, sk: fp32 scales of the
+ * given granularity; v: fp16 [B,H,N,d] (in); o: fp16 [B,H,N,d] (out). */
+int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
+                            const void* v, void* o, int B, int H, int N, int d, int causal,
+                            float sm_scale, int granularity, void* stream);
+
+/* Debug: the full integer product s[b,h,i,j] = sum_c q8[b,h,i,c] * k8[b,h,j,c] as int32
+ * (exact: |s| <= 128*127*127 < 2^31), computed with the same tensor-core path as the fused
+ * kernel.  s: int32 [B,H,N,N] (out); needs B*H*N*N < 2^31. */
+int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, int H, int N, int d,
+                        void* stream);
+
+/* Waits for all work on stream, then returns and clears the device status word written by
+ * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out).  Returns
+ * SAGE_ERR_CUDA (negative) if the synchronization itself failed. */
+int sage_last_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_ATTN_H */

@@ -64,6 +64,7 @@ def _load():
             lib.oracle_smooth_k.argtypes = [vp, i64, i64, i64, vp]
             lib.oracle_quant.argtypes = [vp, vp, i64, i64, i64, i64, vp, vp]
             lib.oracle_qk_int.argtypes = [vp, vp, i64, i64, i64, vp]
+            lib.oracle_qk_int_rows.argtypes = [vp, vp, i64, i64, vp, i64, vp]
             lib.oracle_attn.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f64, i64, i64, vp, vp]
             lib.oracle_attn_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp,
                                              i64, vp, vp]
@@ -71,7 +72,7 @@ def _load():
             lib.oracle_attn_fp64.argtypes = [vp, vp, vp, i64, i64, i64, i32, f64, vp]
             lib.oracle_round_fp16.argtypes = [vp, i64, vp]
             lib.oracle_round_fp16.restype = None
-            for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_attn",
+            for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_qk_int_rows", "oracle_attn",
                          "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
                 getattr(lib, name).restype = i32
             _lib = lib
@@ -148,6 +149,19 @@ def qk_int(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:
     BH, N, d = _bhnd(q8)
     S = np.empty(q8.shape[:-1] + (N,), np.int64)
     _check(_load().oracle_qk_int(_ptr(q8), _ptr(k8), BH, N, d, _ptr(S)), "oracle_qk_int")
+    return S
+
+
+def qk_int_rows(q8h: np.ndarray, k8h: np.ndarray, rows) -> np.ndarray:
+    """Exact integer products of the listed query rows of one head [N,d] with
+    all N keys (int64 [len(rows), N])."""
+    q8h = np.ascontiguousarray(q8h, np.int8)
+    k8h = np.ascontiguousarray(k8h, np.int8)
+    N, d = q8h.shape
+    rows = np.ascontiguousarray(rows, np.int64)
+    S = np.empty((rows.size, N), np.int64)
+    _check(_load().oracle_qk_int_rows(_ptr(q8h), _ptr(k8h), N, d, _ptr(rows), rows.size, _ptr(S)),
+           "oracle_qk_int_rows")
     return S
 
 

@@ -151,6 +151,26 @@ int oracle_qk_int(const int8_t* q8, const int8_t* k8, int64_t BH, int64_t N, int
     return ORACLE_OK;
 }
 
+/* The same products for selected query rows of one head only (rows[r] in [0,N)):
+ * S[r][j] = sum_c q8h[rows[r]][c] * k8h[j][c] for all N keys. */
+int oracle_qk_int_rows(const int8_t* q8h, const int8_t* k8h, int64_t N, int64_t d, const int64_t* rows,
+                       int64_t nrows, int64_t* S) {
+    if (!q8h || !k8h || !rows || !S || N <= 0 || d <= 0) return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return ORACLE_ERR_ARG;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < nrows; ++r) {
+        for (int64_t j = 0; j < N; ++j) {
+            const int8_t* qi = q8h + rows[r] * d;
+            const int8_t* kj = k8h + j * d;
+            int64_t acc = 0;
+            for (int64_t c = 0; c < d; ++c) acc += (int64_t)qi[c] * (int64_t)kj[c];
+            S[r * N + j] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* ---------------------------------------------------------------------------
  * Steps 4-6 for one query row: dequantized scores, softmax, P.V.
  *   s_j  = S_int[i][j] * sq(i) * sk(j) * sm_scale           (fp64)

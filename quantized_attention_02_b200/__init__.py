@@ -1,0 +1,161 @@
+"""Python binding of the B200 SageAttention-style 8-bit attention library.
+
+Argument marshalling only: every step of the method runs in the CUDA kernels of
+``libsage_attn.so`` (built in-tree by ``python -m quantized_attention_02_b200.build``).
+The functions mirror the C ABI of ``include/sage_attn.h`` one to one and take
+torch CUDA tensors, passing their device pointers and the current CUDA stream.
+There is no CPU fallback: a missing library raises at import time, and a call
+on tensors that are not on a CUDA device raises before anything is launched.
+
+The method follows "SageAttention: Accurate 8-Bit Attention for Plug-and-play
+Inference Acceleration" (research.elamur.ai summary page, Summary and idea I1).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage_attn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sage_attn.h")
+
+SAGE_OK = 0
+SAGE_ERR_INVALID = -1
+SAGE_ERR_UNSUPPORTED = -2
+SAGE_ERR_CUDA = -3
+SAGE_ERR_TIMEOUT = -4
+SAGE_ERR_NOMEM = -5
+SAGE_PER_TOKEN = 0
+SAGE_PER_BLOCK = 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m quantized_attention_02_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+_i, _f, _p, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+lib.sage_status_string.argtypes = [_i]
+lib.sage_status_string.restype = ctypes.c_char_p
+lib.sage_scale_count.argtypes = [_i, _i, _i]
+lib.sage_scale_count.restype = _sz
+lib.sage_smooth_k.argtypes = [_p, _p, _i, _i, _i, _i, _p]
+lib.sage_quant_qk.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+lib.sage_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+lib.sage_attn_fwd_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+lib.sage_debug_qk_int32.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p]
+lib.sage_last_device_error.argtypes = [_p]
+for _n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
+           "sage_debug_qk_int32", "sage_last_device_error"):
+    getattr(lib, _n).restype = _i
+
+
+class SageError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {sage_status_string(status)} ({status})")
+        self.status = status
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/sage_attn.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def sage_status_string(status: int) -> str:
+    return lib.sage_status_string(int(status)).decode()
+
+
+def sage_scale_count(N: int, granularity: int, is_q: bool) -> int:
+    return int(lib.sage_scale_count(int(N), int(granularity), int(bool(is_q))))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _shape(x: torch.Tensor):
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(s) for s in x.shape)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != SAGE_OK:
+        raise SageError(rc, where)
+
+
+def sage_smooth_k(k: torch.Tensor, km: torch.Tensor, stream=None) -> None:
+    B, H, N, d = _shape(k)
+    _check(lib.sage_smooth_k(_ptr(k), _ptr(km), B, H, N, d, _stream(stream)), "sage_smooth_k")
+
+
+def sage_quant_qk(q, k, km, q8, k8, sq, sk, granularity: int, stream=None) -> None:
+    B, H, N, d = _shape(q)
+    _check(lib.sage_quant_qk(_ptr(q), _ptr(k), _ptr(km), _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk),
+                             B, H, N, d, int(granularity), _stream(stream)), "sage_quant_qk")
+
+
+def sage_attn_fwd(q, k, v, o, causal: bool, sm_scale: float, granularity: int, stream=None) -> None:
+    B, H, N, d = _shape(q)
+    _check(lib.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+                             float(sm_scale), int(granularity), _stream(stream)), "sage_attn_fwd")
+
+
+def sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float, granularity: int,
+                            stream=None) -> None:
+    B, H, N, d = _shape(v)
+    _check(lib.sage_attn_fwd_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v), _ptr(o), B, H, N,
+                                       d, int(bool(causal)), float(sm_scale), int(granularity),
+                                       _stream(stream)), "sage_attn_fwd_quantized")
+
+
+def sage_debug_qk_int32(q8, k8, s, stream=None) -> None:
+    B, H, N, d = _shape(q8)
+    _check(lib.sage_debug_qk_int32(_ptr(q8), _ptr(k8), _ptr(s), B, H, N, d, _stream(stream)),
+           "sage_debug_qk_int32")
+
+
+def sage_last_device_error(stream=None) -> int:
+    return int(lib.sage_last_device_error(_stream(stream)))
+
+
+# ------------------------------------------------------------------ conveniences
+def empty_quantized(q: torch.Tensor, granularity: int):
+    """Allocate (km, q8, k8, sq, sk) for inputs shaped like q."""
+    B, H, N, d = _shape(q)
+    dev = q.device
+    km = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    q8 = torch.empty((B, H, N, d), dtype=torch.int8, device=dev)
+    k8 = torch.empty((B, H, N, d), dtype=torch.int8, device=dev)
+    sq = torch.empty((B, H, sage_scale_count(N, granularity, True)), dtype=torch.float32, device=dev)
+    sk = torch.empty((B, H, sage_scale_count(N, granularity, False)), dtype=torch.float32, device=dev)
+    return km, q8, k8, sq, sk
+
+
+def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             sm_scale: float | None = None, granularity: int = SAGE_PER_BLOCK, stream=None) -> torch.Tensor:
+    """O = softmax(Q K^T sm_scale) V with smoothed INT8 Q K^T and FP16 P V.
+    sm_scale defaults to d^-1/2."""
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(q.shape[-1])
+    o = torch.empty_like(q)
+    sage_attn_fwd(q, k, v, o, causal, sm_scale, granularity, stream)
+    return o

@@ -1,0 +1,541 @@
+// attn_kernels.cu -- the fused 8-bit attention forward kernel for sm_100a, and the debug
+// kernel that exposes its INT32 Q.K^T.
+//
+// Method (SageAttention summary page, Summary bullets 1-2 and "FlashAttention-style tiling"):
+//   S   = q8 . k8^T                       INT8 x INT8 -> INT32 on the tensor cores (tcgen05 kind::i8)
+//   s   = S * sq(i) * sk(j) * sm_scale    dequantized in fp32, kept in log2 units (x log2 e)
+//   online softmax over key tiles: running row max m, row sum l, exp2
+//   P~  = fp16(exp2(s - m))               written back to tensor memory
+//   O  += P~ . V                          FP16 x FP16 -> FP32 on the tensor cores (kind::f16,
+//                                         A operand read straight from tensor memory)
+//   O   = O / l                           stored as fp16
+//
+// CTA organisation (one CTA per SM: 512 TMEM columns and > 114 KB of shared memory):
+//   work unit = (head, pair of 128-row query tiles); 12 warps:
+//     warp 0      TMA producer: Q tiles once, then K / V tiles through a STAGES-deep ring
+//     warp 1      TMEM allocator and single-thread MMA issuer
+//     warps 4-7   softmax for query tile 0 (thread = one query row = one TMEM lane)
+//     warps 8-11  softmax for query tile 1
+//   TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D); P~_t (fp16,
+//   64 columns) overwrites the first half of S_t once S_t has been read.
+//   The MMA issue order per key tile j is  PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that while
+//   one softmax warpgroup works the tensor core serves the other tile (ping-pong).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "attn_kernels.cuh"
+#include "sm100_ptx.cuh"
+
+namespace sage {
+
+template <int D>
+struct AttnLayout {
+  static constexpr int BM = 128;          // query rows per tile
+  static constexpr int BN = 128;          // keys per tile
+  static constexpr int NQT = 2;           // query tiles per CTA
+  static constexpr int STAGES = D == 128 ? 3 : 4;
+  static constexpr int Q_BYTES = BM * D;  // int8 tile
+  static constexpr int K_BYTES = BN * D;  // int8 tile
+  static constexpr int V_BOX = BN * 128;  // one 64-column fp16 box (128-byte rows)
+  static constexpr int V_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
+  static constexpr int OFF_SK = OFF_V + STAGES * V_BYTES;           // per-token key scales
+  static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 3 * NQT + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int USED = OFF_MISC + 16;
+  // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
+  static constexpr int SMEM = (USED + 1024 > 116 * 1024 ? USED + 1024 : 116 * 1024);
+  __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
+  __host__ __device__ static constexpr uint32_t o_col(int t) { return 256u + D * t; }
+  static constexpr int THREADS = 384;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Bounded wait used on exit paths: ignores the abort flag, records a timeout.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicExch(&g_device_error, kDevTimeoutBarrier);
+      return;
+    }
+  }
+}
+
+template <int D, bool CAUSAL, bool PER_TOKEN>
+__global__ void __launch_bounds__(384, 1)
+    sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ sq,
+                     const float* __restrict__ sk, __half* __restrict__ o, int BH, int N,
+                     float sm_scale_log2) {
+  using L = AttnLayout<D>;
+  constexpr int STAGES = L::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  float* sSK = reinterpret_cast<float*>(smem + L::OFF_SK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_k_full = bars + 1;
+  uint64_t* bar_v_full = bars + 1 + STAGES;
+  uint64_t* bar_kv_empty = bars + 1 + 2 * STAGES;
+  uint64_t* bar_s_full = bars + 1 + 3 * STAGES;
+  uint64_t* bar_p_full = bar_s_full + 2;
+  uint64_t* bar_o_done = bar_s_full + 4;
+  uint64_t* bar_drain = bar_s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heavy query-tile pairs first (causal work grows with the row index)
+  const int n_qtiles = N / L::BM;
+  const int n_pairs = (n_qtiles + 1) / 2;
+  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int tile0 = 2 * pair;
+  const int n_tiles = min(2, n_qtiles - tile0);
+  const int n_kv_total = N / L::BN;
+  int n_iter[2];
+  n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
+  n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
+  const int n_kv = max(n_iter[0], n_iter[1]);
+  const int row_base = bh * N;  // first row of this head in the [BH*N, D] views
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_v_full + s, 1);
+      mbar_init(bar_kv_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + t, 1);
+      mbar_init(bar_p_full + t, 128);
+      mbar_init(bar_o_done + t, 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      int issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      mbar_arrive_expect_tx(bar_q, n_tiles * L::Q_BYTES);
+      for (int t = 0; t < n_tiles; ++t)
+        tma_load_2d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, row_base + (tile0 + t) * L::BM);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % STAGES;
+        const int it = j / STAGES;
+        if (j >= STAGES && !mbar_wait(bar_kv_empty + s, (it - 1) & 1, abort_flag)) break;
+        const int key_row = row_base + j * L::BN;
+        mbar_arrive_expect_tx(bar_k_full + s, L::K_BYTES + (PER_TOKEN ? L::BN * 4 : 0));
+        tma_load_2d(sK + s * L::K_BYTES, &tm_k, bar_k_full + s, 0, key_row);
+        if constexpr (PER_TOKEN) bulk_load(sSK + s * L::BN, sk + key_row, L::BN * 4, bar_k_full + s);
+        mbar_arrive_expect_tx(bar_v_full + s, L::V_BYTES);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_2d(sV + s * L::V_BYTES + b * L::V_BOX, &tm_v, bar_v_full + s, 64 * b, key_row);
+        issued[s] = it + 1;
+      }
+      if (*abort_flag) {  // let copies in flight land before the CTA exits
+        mbar_drain(bar_q, 0);
+        for (int s = 0; s < STAGES; ++s) {
+          if (issued[s] > 0) {
+            mbar_drain(bar_k_full + s, (issued[s] - 1) & 1);
+            mbar_drain(bar_v_full + s, (issued[s] - 1) & 1);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
+      constexpr uint32_t IDESC_PV = make_idesc(1 /*f32*/, 0 /*f16*/, 0 /*f16*/, 0, 1 /*V is MN-major*/, 128, D);
+      constexpr SwizzleMode QK_SWZ = D == 128 ? kSwizzle128B : kSwizzle64B;
+      constexpr uint32_t QK_SBO = D == 128 ? 1024 : 512;  // 8 rows of D bytes
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+
+      auto issue_qk = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = make_smem_desc(q_base + t * L::Q_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
+          const uint64_t b = make_smem_desc(k_base + s * L::K_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
+          mma_i8_ss(tmem + L::s_col(t), a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s_full + t);
+      };
+      auto issue_pv = [&](int t, int s, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < L::BN / 16; ++kk) {
+          // 16 keys per MMA = 16 rows of 128 B in the V box; LBO jumps to the next 64 columns
+          const uint64_t b = make_smem_desc(v_base + s * L::V_BYTES + kk * 16 * 128, L::V_BOX, 1024, kSwizzle128B);
+          mma_f16_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(bar_o_done + t);
+      };
+
+      bool ok = mbar_wait(bar_q, 0, abort_flag) && mbar_wait(bar_k_full, 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < n_tiles; ++t) issue_qk(t, 0);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j % STAGES;
+        if (!mbar_wait(bar_v_full + s, (j / STAGES) & 1, abort_flag)) break;
+        for (int t = 0; t < n_tiles && ok; ++t) {
+          if (j >= n_iter[t]) continue;
+          if (!mbar_wait(bar_p_full + t, j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, s, j == 0);
+          if (j + 1 < n_iter[t]) {
+            const int s1 = (j + 1) % STAGES;
+            // next S_t overwrites P~_t: wait until this PV has consumed it
+            if (!mbar_wait(bar_k_full + s1, ((j + 1) / STAGES) & 1, abort_flag) ||
+                !mbar_wait(bar_o_done + t, j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk(t, s1);
+          }
+        }
+        mma_commit(bar_kv_empty + s);
+      }
+      // all MMAs issued by this thread must finish before TMEM is released
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0);
+    }
+  } else if (warp >= 4) {
+    // ================================================================ softmax warpgroups
+    const int t = (warp - 4) >> 2;
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;
+    if (t < n_tiles) {
+      const int q_tile = tile0 + t;
+      const int q_row = q_tile * L::BM + r;
+      const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+      const uint32_t tS = tmem + lane_addr + L::s_col(t);
+      const uint32_t tO = tmem + lane_addr + L::o_col(t);
+      const float sq_r = PER_TOKEN ? __ldg(sq + row_base + q_row) : __ldg(sq + bh * n_qtiles + q_tile);
+      const float a_r = sq_r * sm_scale_log2;  // log2-unit scale of one integer step, before sk
+      float m_use = -INFINITY;  // offset used in the exponents so far (log2 units)
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_iter[t]; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t x[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
+        tmem_wait_ld();
+
+        const bool diag = CAUSAL && (j == q_tile);
+        const int s = j % STAGES;
+        float c_blk0 = 0.f, c_blk1 = 0.f;
+        if constexpr (PER_TOKEN) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
+        } else {
+          c_blk0 = a_r * __ldg(sk + bh * (N / 64) + 2 * j);
+          c_blk1 = a_r * __ldg(sk + bh * (N / 64) + 2 * j + 1);
+        }
+        const float* skj = sSK + s * L::BN;
+
+        // ---- row maximum of the dequantized scores (log2 units)
+        float mx = -INFINITY;
+        if constexpr (PER_TOKEN) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[c]);
+            if (!(diag && c > r)) mx = fmaxf(mx, v);
+          }
+        } else {
+          int im0 = INT_MIN, im1 = INT_MIN;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!(diag && c > r)) im0 = max(im0, static_cast<int>(x[c]));
+#pragma unroll
+          for (int c = 64; c < 128; ++c)
+            if (!(diag && c > r)) im1 = max(im1, static_cast<int>(x[c]));
+          if (im0 != INT_MIN) mx = fmaxf(mx, c_blk0 * static_cast<float>(im0));
+          if (im1 != INT_MIN) mx = fmaxf(mx, c_blk1 * static_cast<float>(im1));
+        }
+
+        // ---- rescale only when the maximum grew by more than 2^8 (bounds P~ by 256)
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_use = mx;
+        } else if (mx > m_use + 8.f) {
+          alpha = fast_exp2(m_use - mx);
+          m_use = mx;
+          rescale = true;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+          l *= alpha;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int cb = 0; cb < D; cb += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + cb, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(tO + cb, ov);
+          }
+        }
+
+        // ---- P~ = exp2(s - m_use) in fp16, row sum in fp32 from the unrounded values
+        float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cb = 0; cb < 128; cb += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float p2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int c = cb + i + u;
+              const float cs = PER_TOKEN ? a_r * skj[c] : (c < 64 ? c_blk0 : c_blk1);
+              float p = fast_exp2(fmaf(static_cast<float>(static_cast<int>(x[c])), cs, -m_use));
+              if (diag && c > r) p = 0.f;
+              p2[u] = p;
+            }
+            lsum[(i >> 1) & 3] += p2[0] + p2[1];
+            pk[i >> 1] = pack_half2(p2[0], p2[1]);
+          }
+          tmem_st16(tS + (cb >> 1), pk);
+        }
+        l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full + t);
+      }
+
+      // ---- epilogue: O / l -> fp16 -> global
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (n_iter[t] - 1) & 1, abort_flag))) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        __half* orow = o + (static_cast<size_t>(row_base) + q_row) * D;
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + cb, ov);
+          tmem_wait_ld();
+          uint32_t hv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            hv[i] = pack_half2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- debug: INT32 S = q8 k8^T
+// One CTA per (128-row query tile, head).  Thread 0 issues the TMA loads and the same
+// kind::i8 MMA as the fused kernel; warps 4-7 copy S from TMEM to global memory.
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    sage_qk_debug_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         int32_t* __restrict__ s_out, int N) {
+  constexpr int BM = 128, BN = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + BM * D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BM * D + BN * D);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_k = bars + 1;
+  uint64_t* bar_s = bars + 2;
+  uint64_t* bar_free = bars + 3;
+  uint64_t* bar_drain = bars + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q_tile = blockIdx.x, bh = blockIdx.y;
+  const int row_base = bh * N;
+  const int n_kv = N / BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_free, 128);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = make_idesc(2, 1, 1, 0, 0, 128, BN);
+      constexpr SwizzleMode SWZ = D == 128 ? kSwizzle128B : kSwizzle64B;
+      constexpr uint32_t SBO = D == 128 ? 1024 : 512;
+      mbar_arrive_expect_tx(bar_q, BM * D);
+      tma_load_2d(sQ, &tm_q, bar_q, 0, row_base + q_tile * BM);
+      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      int k_loads = 0;
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j > 0 && !mbar_wait(bar_free, (j - 1) & 1, abort_flag)) break;  // S and K buffer free
+        mbar_arrive_expect_tx(bar_k, BN * D);
+        tma_load_2d(sK, &tm_k, bar_k, 0, row_base + j * BN);
+        ++k_loads;
+        if (!mbar_wait(bar_k, j & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = make_smem_desc(smem_u32(sQ) + kk * 32, 16, SBO, SWZ);
+          const uint64_t b = make_smem_desc(smem_u32(sK) + kk * 32, 16, SBO, SWZ);
+          mma_i8_ss(tmem, a, b, IDESC, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0);
+      if (k_loads > 0) mbar_drain(bar_k, (k_loads - 1) & 1);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    int32_t* srow = s_out + (static_cast<size_t>(row_base) + q_tile * BM + r) * N;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < BN; cb += 32) {
+        uint32_t v[32];
+        tmem_ld32(tS + cb, v);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(srow + j * BN + cb);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_free);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ---------------------------------------------------------------- launchers
+template <int D, bool CAUSAL, bool PER_TOKEN>
+static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
+  using L = AttnLayout<D>;
+  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN>;
+  static bool configured = false;  // attribute set once per instantiation (idempotent)
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int n_qtiles = a.N / L::BM;
+  const int n_pairs = (n_qtiles + 1) / 2;
+  dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
+  kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sq, a.sk, a.o, a.BH, a.N, a.sm_scale_log2);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
+  if (a.causal) return a.per_token ? launch_attn_t<D, true, true>(a, st) : launch_attn_t<D, true, false>(a, st);
+  return a.per_token ? launch_attn_t<D, false, true>(a, st) : launch_attn_t<D, false, false>(a, st);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  return a.D == 128 ? launch_attn_d<128>(a, st) : launch_attn_d<64>(a, st);
+}
+
+template <int D>
+static cudaError_t launch_qk_debug_d(const CUtensorMap& tq, const CUtensorMap& tk, int32_t* s, int BH, int N,
+                                     cudaStream_t st) {
+  // 4 CTAs per SM at most (4 x 128 TMEM columns): ask for 56 KB of shared memory each
+  constexpr int SMEM = 56 * 1024;
+  auto kern = sage_qk_debug_kernel<D>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid(N / 128, BH);
+  kern<<<grid, 256, SMEM, st>>>(tq, tk, s, N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qk_debug(const CUtensorMap& tq, const CUtensorMap& tk, int32_t* s, int BH, int N, int D,
+                            cudaStream_t st) {
+  return D == 128 ? launch_qk_debug_d<128>(tq, tk, s, BH, N, st) : launch_qk_debug_d<64>(tq, tk, s, BH, N, st);
+}
+
+int read_and_clear_device_error(cudaStream_t st, cudaError_t* err) {
+  *err = cudaStreamSynchronize(st);
+  if (*err != cudaSuccess) return -1;
+  int h = 0;
+  *err = cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int));
+  if (*err != cudaSuccess) return -1;
+  const int zero = 0;
+  *err = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (*err != cudaSuccess) return -1;
+  return h;
+}
+
+}  // namespace sage

@@ -1,0 +1,28 @@
+// attn_kernels.cuh -- launchers for the fused attention kernel and the INT32 Q.K^T debug kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace sage {
+
+struct AttnArgs {
+  const CUtensorMap* tm_q;  // int8 [BH*N, D], box {D, 128}, 128 B (D=128) / 64 B (D=64) swizzle
+  const CUtensorMap* tm_k;  // int8 [BH*N, D], same boxes
+  const CUtensorMap* tm_v;  // fp16 [BH*N, D], box {64, 128}, 128 B swizzle
+  const float* sq;          // [BH, N] per token or [BH, N/128] per block
+  const float* sk;          // [BH, N] per token or [BH, N/64] per block
+  __half* o;                // fp16 [BH, N, D]
+  int BH, N, D;
+  bool causal, per_token;
+  float sm_scale_log2;      // sm_scale * log2(e)
+};
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_qk_debug(const CUtensorMap& tq, const CUtensorMap& tk, int32_t* s, int BH, int N, int D,
+                            cudaStream_t st);
+// Synchronizes st, returns the device status word (and clears it); -1 if a CUDA call failed.
+int read_and_clear_device_error(cudaStream_t st, cudaError_t* err);
+
+}  // namespace sage

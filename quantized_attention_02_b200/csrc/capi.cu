@@ -1,0 +1,221 @@
+// capi.cu -- the C ABI declared in include/sage_attn.h: argument validation, TMA tensor
+// maps, stream-ordered workspace and the launches of the three steps of the method
+// (smooth K -> quantize Q and K -> fused INT8/FP16 attention).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn_kernels.cuh"
+#include "prep_kernels.cuh"
+#include "sage_attn.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled comes from the driver through the runtime's entry-point query, so
+// the library links no libcuda and loads on machines without a GPU driver.
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major view [rows, D] with a box of {box_cols, 128} rows.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes, long long rows, int D,
+              int box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_qk_map(CUtensorMap* map, const int8_t* base, long long rows, int D) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, D, D,
+                  D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+bool make_v_map(CUtensorMap* map, const void* base, long long rows, int D) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, D, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every entry point.
+int check_shape(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SAGE_ERR_INVALID;
+  if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return SAGE_ERR_UNSUPPORTED;
+  const long long elems = static_cast<long long>(B) * H * N * d;
+  if (elems >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+int check_scale(float sm_scale) {
+  return (std::isfinite(sm_scale) && sm_scale > 0.f) ? SAGE_OK : SAGE_ERR_INVALID;
+}
+
+int check_gran(int g) { return (g == SAGE_PER_TOKEN || g == SAGE_PER_BLOCK) ? SAGE_OK : SAGE_ERR_INVALID; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
+
+int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v, void* o,
+                        int B, int H, int N, int d, int causal, float sm_scale, int granularity,
+                        cudaStream_t st) {
+  const int BH = B * H;
+  const long long rows = static_cast<long long>(BH) * N;
+  CUtensorMap tq, tk, tv;
+  if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d) || !make_v_map(&tv, v, rows, d))
+    return SAGE_ERR_CUDA;
+  sage::AttnArgs a{};
+  a.tm_q = &tq;
+  a.tm_k = &tk;
+  a.tm_v = &tv;
+  a.sq = sq;
+  a.sk = sk;
+  a.o = static_cast<__half*>(o);
+  a.BH = BH;
+  a.N = N;
+  a.D = d;
+  a.causal = causal != 0;
+  a.per_token = granularity == SAGE_PER_TOKEN;
+  a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  return cuda_status(sage::launch_attn(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sage_status_string(int status) {
+  switch (status) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128, N a multiple of 128)";
+    case SAGE_ERR_CUDA: return "CUDA runtime error";
+    case SAGE_ERR_TIMEOUT: return "a kernel wait timed out";
+    case SAGE_ERR_NOMEM: return "workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+size_t sage_scale_count(int N, int granularity, int is_q) {
+  if (N <= 0) return 0;
+  if (granularity == SAGE_PER_TOKEN) return static_cast<size_t>(N);
+  if (granularity == SAGE_PER_BLOCK) {
+    const int g = is_q ? 128 : 64;
+    return static_cast<size_t>((N + g - 1) / g);
+  }
+  return 0;
+}
+
+int sage_smooth_k(const void* k, float* km, int B, int H, int N, int d, void* stream) {
+  if (!k || !km) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (!aligned16(k)) return SAGE_ERR_INVALID;
+  return cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, B * H, N, d,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int sage_quant_qk(const void* q, const void* k, const float* km, int8_t* q8, int8_t* k8, float* sq, float* sk,
+                  int B, int H, int N, int d, int granularity, void* stream) {
+  if (!q || !k || !q8 || !k8 || !sq || !sk) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_gran(granularity))) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pt = granularity == SAGE_PER_TOKEN;
+  const int BH = B * H;
+  cudaError_t e = sage::launch_quant(static_cast<const __half*>(q), nullptr, q8, sq, BH, N, d, pt ? 1 : 128, st);
+  if (e != cudaSuccess) return SAGE_ERR_CUDA;
+  e = sage::launch_quant(static_cast<const __half*>(k), km, k8, sk, BH, N, d, pt ? 1 : 64, st);
+  return cuda_status(e);
+}
+
+int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v,
+                            void* o, int B, int H, int N, int d, int causal, float sm_scale, int granularity,
+                            void* stream) {
+  if (!q8 || !k8 || !sq || !sk || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(sk)) return SAGE_ERR_INVALID;
+  return attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                  float sm_scale, int granularity, void* stream) {
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const size_t elems = static_cast<size_t>(BH) * N * d;
+  const size_t nsq = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 1);
+  const size_t nsk = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 0);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t off_k8 = up(elems);
+  const size_t off_sq = off_k8 + up(elems);
+  const size_t off_sk = off_sq + up(nsq * 4);
+  const size_t off_km = off_sk + up(nsk * 4);
+  const size_t total = off_km + up(static_cast<size_t>(BH) * d * 4);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, total, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int8_t* q8 = reinterpret_cast<int8_t*>(w);
+  int8_t* k8 = reinterpret_cast<int8_t*>(w + off_k8);
+  float* sq = reinterpret_cast<float*>(w + off_sq);
+  float* sk = reinterpret_cast<float*>(w + off_sk);
+  float* km = reinterpret_cast<float*>(w + off_km);
+  rc = cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, BH, N, d, st));
+  if (!rc) rc = sage_quant_qk(q, k, km, q8, k8, sq, sk, B, H, N, d, granularity, stream);
+  if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity, st);
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
+}
+
+int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, int H, int N, int d, void* stream) {
+  if (!q8 || !k8 || !s) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (static_cast<long long>(B) * H * N * N >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(s)) return SAGE_ERR_INVALID;
+  const long long rows = static_cast<long long>(B) * H * N;
+  CUtensorMap tq, tk;
+  if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d)) return SAGE_ERR_CUDA;
+  return cuda_status(sage::launch_qk_debug(tq, tk, s, B * H, N, d, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_last_device_error(void* stream) {
+  cudaError_t e;
+  const int code = sage::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);
+  return code < 0 ? SAGE_ERR_CUDA : code;
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every
+function include/sage_attn.h declares, and rejects invalid calls before launching
+anything (argument validation happens ahead of any CUDA call)."""
+import ctypes
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sa():
+    from quantized_attention_02_b200 import build
+    build.build()
+    import quantized_attention_02_b200 as sa
+    return sa
+
+
+def test_library_exports_every_header_function(sa):
+    names = sa.header_functions()
+    assert set(names) >= {"sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
+                          "sage_debug_qk_int32", "sage_status_string", "sage_scale_count",
+                          "sage_last_device_error"}
+    lib = ctypes.CDLL(sa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_has_no_driver_link_dependency(sa):
+    # the driver is reached through the runtime's entry-point query only
+    import subprocess
+    out = subprocess.run(["ldd", sa.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_status_strings_and_scale_counts(sa):
+    for s in (0, -1, -2, -3, -4, -5, 42):
+        assert isinstance(sa.sage_status_string(s), str) and sa.sage_status_string(s)
+    assert sa.sage_scale_count(1024, sa.SAGE_PER_TOKEN, True) == 1024
+    assert sa.sage_scale_count(1024, sa.SAGE_PER_BLOCK, True) == 8
+    assert sa.sage_scale_count(1024, sa.SAGE_PER_BLOCK, False) == 16
+    assert sa.sage_scale_count(300, sa.SAGE_PER_BLOCK, False) == 5
+    assert sa.sage_scale_count(0, sa.SAGE_PER_BLOCK, False) == 0
+    assert sa.sage_scale_count(128, 7, False) == 0
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (B, H, N, d)
+    ((1, 1, 128, 96), -2),   # d not 64/128
+    ((1, 1, 100, 64), -2),   # N not a multiple of 128
+    ((0, 1, 128, 64), -1),   # empty batch
+    ((1, 1, 0, 64), -1),     # empty sequence
+    ((1, -1, 128, 64), -1),
+    ((4096, 4096, 1024, 128), -2),  # too many elements for 32-bit indexing
+])
+def test_shape_validation(sa, args, expect):
+    B, H, N, d = args
+    L = sa.lib
+    s = ctypes.c_void_p(0)
+    assert L.sage_smooth_k(FAKE, FAKE, B, H, N, d, s) == expect
+    assert L.sage_quant_qk(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, B, H, N, d, 1, s) == expect
+    assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, B, H, N, d, 0, 0.1, 1, s) == expect
+    assert L.sage_attn_fwd_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, H, N, d, 0, 0.1, 1, s) == expect
+    assert L.sage_debug_qk_int32(FAKE, FAKE, FAKE, B, H, N, d, s) == expect
+
+
+def test_null_pointers_and_bad_scalars(sa):
+    L = sa.lib
+    s = ctypes.c_void_p(0)
+    assert L.sage_smooth_k(None, FAKE, 1, 1, 128, 64, s) == -1
+    assert L.sage_quant_qk(FAKE, FAKE, None, FAKE, None, FAKE, FAKE, 1, 1, 128, 64, 1, s) == -1
+    assert L.sage_attn_fwd(FAKE, FAKE, FAKE, None, 1, 1, 128, 64, 0, 0.1, 1, s) == -1
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, bad, 1, s) == -1
+        assert L.sage_attn_fwd_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, bad, 1, s) == -1
+    for g in (-1, 2, 17):
+        assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, 0.1, g, s) == -1
+        assert L.sage_quant_qk(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, g, s) == -1
+    misaligned = ctypes.c_void_p(0x1008)
+    assert L.sage_smooth_k(misaligned, FAKE, 1, 1, 128, 64, s) == -1
+    assert L.sage_debug_qk_int32(FAKE, FAKE, None, 1, 1, 128, 64, s) == -1
+
+
+def test_binding_rejects_cpu_tensors(sa):
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        sa.sageattn(q, q, q)

@@ -186,6 +186,13 @@ def test_qk_int_matches_brute_force_and_int64_matmul():
     np.testing.assert_array_equal(oracle.qk_int(q8b, k8b)[0], ref)
 
 
+def test_qk_int_rows_matches_full_product():
+    q8 = RNG.integers(-127, 128, (1, 40, 16), dtype=np.int8)
+    k8 = RNG.integers(-127, 128, (1, 40, 16), dtype=np.int8)
+    rows = np.array([0, 7, 39])
+    np.testing.assert_array_equal(oracle.qk_int_rows(q8[0], k8[0], rows), oracle.qk_int(q8, k8)[0, rows])
+
+
 def test_qk_int_extreme_values_fit():
     q8 = np.full((1, 4, 128), 127, np.int8)
     k8 = np.full((1, 4, 128), -127, np.int8)
