@@ -253,7 +253,7 @@ def run_ours(args, w: W.Workload):
         peak = mixed_peak_tops(p_sus)
         achieved = ops / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
-        cpu_tops, cores, desc = oracle_sample(w)
+        cpu_tops, cores, desc = (None, None, "skipped") if args.no_cpu_baseline else oracle_sample(w)
         elem_bytes = w.BH * w.N * w.d * 2
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -321,6 +321,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (profiler runs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

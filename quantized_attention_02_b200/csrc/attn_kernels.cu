@@ -66,6 +66,42 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Magic-number integer -> float: for |S| < 2^22 the bits of S + 0x4B400000 are the float
+// 1.5 * 2^23 + S exactly.
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr float kMagicF = 12582912.0f;
+
+// Scale c with its 3 lowest mantissa bits cleared (21 significant bits): kMagicF * c is then
+// exact in fp32 (relative change of c at most 2^-20).
+__device__ __forceinline__ float trim_scale(float c) { return __uint_as_float(__float_as_uint(c) & ~7u); }
+
+// 4 ulps of x (a power of two), or the smallest normal for tiny / zero x.
+__device__ __forceinline__ float offset_quantum(float x) {
+  const int e = static_cast<int>((__float_as_uint(x) >> 23) & 0xFFu);
+  return e > 22 ? __uint_as_float(static_cast<uint32_t>(e - 21) << 23) : 0x1p-126f;
+}
+
+// Smallest multiple of the power of two q that is >= x (exact).  Floats of magnitude at
+// least 2^23 q are multiples of q already (and x / q might overflow).
+__device__ __forceinline__ float round_up_to(float x, float q) {
+  return fabsf(x) < q * 8388608.0f ? ceilf(x / q) * q : x;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Bounded wait used on exit paths: ignores the abort flag, records a timeout.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -106,11 +142,12 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: heavy query-tile pairs first (causal work grows with the row index)
+  // ---- work unit: consecutive CTAs share a head (its K/V stay in L2); within a head the
+  // query-tile pairs with the most key tiles (causal) come first
   const int n_qtiles = N / L::BM;
   const int n_pairs = (n_qtiles + 1) / 2;
-  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int bh = static_cast<int>(blockIdx.x) / n_pairs;
+  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
   const int tile0 = 2 * pair;
   const int n_tiles = min(2, n_qtiles - tile0);
   const int n_kv_total = N / L::BN;
@@ -148,7 +185,12 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  // Registers: the block is launched with 168 per thread (384 x 168); the control
+  // warpgroup hands most of its share to the two softmax warpgroups: 128 x 56 + 256 x 224.
+  // Each setmaxnreg is executed by a whole warpgroup and dominates that group's code.
+  if (warp < 4) {
+    reg_dealloc<56>();
+    if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
       int issued[STAGES];
@@ -222,10 +264,10 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           issue_pv(t, s, j == 0);
           if (j + 1 < n_iter[t]) {
+            // S_t(j+1) overwrites P~_t(j): tcgen05 MMAs issued by one thread execute in
+            // issue order, so the P.V above has read P~_t before this product writes S_t.
             const int s1 = (j + 1) % STAGES;
-            // next S_t overwrites P~_t: wait until this PV has consumed it
-            if (!mbar_wait(bar_k_full + s1, ((j + 1) / STAGES) & 1, abort_flag) ||
-                !mbar_wait(bar_o_done + t, j & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bar_k_full + s1, ((j + 1) / STAGES) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             issue_qk(t, s1);
           }
@@ -236,7 +278,9 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(bar_drain);
       mbar_drain(bar_drain, 0);
     }
-  } else if (warp >= 4) {
+    }
+  } else {
+    reg_alloc<224>();
     // ================================================================ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
@@ -248,9 +292,25 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t tS = tmem + lane_addr + L::s_col(t);
       const uint32_t tO = tmem + lane_addr + L::o_col(t);
       const float sq_r = PER_TOKEN ? __ldg(sq + row_base + q_row) : __ldg(sq + bh * n_qtiles + q_tile);
-      const float a_r = sq_r * sm_scale_log2;  // log2-unit scale of one integer step, before sk
-      float m_use = -INFINITY;  // offset used in the exponents so far (log2 units)
-      float l = 0.f;
+      const float a_r = sq_r * sm_scale_log2;  // log2-unit value of one integer step, before sk
+      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : N / 64);
+
+      // Offset quantum: the exponent offset m_use is kept a multiple of qm, a power of two at
+      // least 4 ulps of kMagic * c for every key scale c of this row.  Then kMagic * c' + m_use
+      // is exact in fp32 and fma(f, c', -(kMagic * c' + m_use)) = fl(S * c' - m_use): the
+      // integer-to-float conversion by the magic-number add costs no extra rounding.
+      float qm = 0x1p-126f;
+      if constexpr (!PER_TOKEN) {
+        // largest key scale of the head: the warp's lanes split the N/64 scales, then reduce
+        float skmax = 0.f;
+        for (int i = lane; i < N / 64; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) skmax = fmaxf(skmax, __shfl_xor_sync(0xffffffffu, skmax, off));
+        qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
+      }
+
+      float m_use = 0.f;  // exponent offset (log2 units) applied to this row so far
+      float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       bool ok = true;
       for (int j = 0; j < n_iter[t]; ++j) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { ok = false; break; }
@@ -264,47 +324,52 @@ __global__ void __launch_bounds__(384, 1)
 
         const bool diag = CAUSAL && (j == q_tile);
         const int s = j % STAGES;
-        float c_blk0 = 0.f, c_blk1 = 0.f;
+        // f = kMagic + S exactly (|S| < 2^22), as float bits
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] += kMagicBits;
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > r) x[c] = 0xFF800000u;  // -inf: masked key
+        }
+
+        float mx;            // row maximum of the dequantized scores (log2 units)
+        float cb0 = 0.f, cb1 = 0.f, nb0 = 0.f, nb1 = 0.f;
+        const float* skj = sSK + s * L::BN;
         if constexpr (PER_TOKEN) {
           if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
+          mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            mx = fmaxf(mx, (__uint_as_float(x[c]) - kMagicF) * (a_r * skj[c]));
         } else {
-          c_blk0 = a_r * __ldg(sk + bh * (N / 64) + 2 * j);
-          c_blk1 = a_r * __ldg(sk + bh * (N / 64) + 2 * j + 1);
-        }
-        const float* skj = sSK + s * L::BN;
-
-        // ---- row maximum of the dequantized scores (log2 units)
-        float mx = -INFINITY;
-        if constexpr (PER_TOKEN) {
+          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
+          cb1 = trim_scale(a_r * __ldg(sk_head + 2 * j + 1));
+          float f0 = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
+          float f1 = max3f(__uint_as_float(x[64]), __uint_as_float(x[65]), __uint_as_float(x[66]));
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[c]);
-            if (!(diag && c > r)) mx = fmaxf(mx, v);
-          }
-        } else {
-          int im0 = INT_MIN, im1 = INT_MIN;
+          for (int c = 3; c < 63; c += 2) f0 = max3f(f0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+          f0 = fmaxf(f0, __uint_as_float(x[63]));
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!(diag && c > r)) im0 = max(im0, static_cast<int>(x[c]));
-#pragma unroll
-          for (int c = 64; c < 128; ++c)
-            if (!(diag && c > r)) im1 = max(im1, static_cast<int>(x[c]));
-          if (im0 != INT_MIN) mx = fmaxf(mx, c_blk0 * static_cast<float>(im0));
-          if (im1 != INT_MIN) mx = fmaxf(mx, c_blk1 * static_cast<float>(im1));
+          for (int c = 67; c < 127; c += 2) f1 = max3f(f1, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+          f1 = fmaxf(f1, __uint_as_float(x[127]));
+          mx = fmaxf(cb0 * (f0 - kMagicF), cb1 * (f1 - kMagicF));  // -inf halves stay -inf
         }
 
         // ---- rescale only when the maximum grew by more than 2^8 (bounds P~ by 256)
         float alpha = 1.f;
         bool rescale = false;
         if (j == 0) {
-          m_use = mx;
+          m_use = round_up_to(mx, qm);
         } else if (mx > m_use + 8.f) {
-          alpha = fast_exp2(m_use - mx);
-          m_use = mx;
+          const float m_new = round_up_to(mx, qm);
+          alpha = fast_exp2(m_use - m_new);
+          m_use = m_new;
           rescale = true;
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          l *= alpha;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
           if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -317,29 +382,38 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(tO + cb, ov);
           }
         }
+        if constexpr (!PER_TOKEN) {
+          nb0 = -fmaf(kMagicF, cb0, m_use);  // exact: see offset_quantum above
+          nb1 = -fmaf(kMagicF, cb1, m_use);
+        }
 
-        // ---- P~ = exp2(s - m_use) in fp16, row sum in fp32 from the unrounded values
-        float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- P~ = exp2(s - m_use) in fp16; the row sum takes the unrounded values
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            float p2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = cb + i + u;
-              const float cs = PER_TOKEN ? a_r * skj[c] : (c < 64 ? c_blk0 : c_blk1);
-              float p = fast_exp2(fmaf(static_cast<float>(static_cast<int>(x[c])), cs, -m_use));
-              if (diag && c > r) p = 0.f;
-              p2[u] = p;
+            const int c = cb + i;
+            float2 tt;
+            if constexpr (PER_TOKEN) {
+              tt.x = fmaf(__uint_as_float(x[c]) - kMagicF, a_r * skj[c], -m_use);
+              tt.y = fmaf(__uint_as_float(x[c + 1]) - kMagicF, a_r * skj[c + 1], -m_use);
+            } else {
+              const float cs = c < 64 ? cb0 : cb1;
+              const float nb = c < 64 ? nb0 : nb1;
+              tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), make_float2(cs, cs),
+                              make_float2(nb, nb));
             }
-            lsum[(i >> 1) & 3] += p2[0] + p2[1];
-            pk[i >> 1] = pack_half2(p2[0], p2[1]);
+            float2 p = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
+            if (diag) {
+              if (c > r) p.x = 0.f;
+              if (c + 1 > r) p.y = 0.f;
+            }
+            lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
+            pk[i >> 1] = pack_half2(p.x, p.y);
           }
           tmem_st16(tS + (cb >> 1), pk);
         }
-        l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p_full + t);
@@ -348,7 +422,8 @@ __global__ void __launch_bounds__(384, 1)
       // ---- epilogue: O / l -> fp16 -> global
       if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (n_iter[t] - 1) & 1, abort_flag))) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float2 l2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+        const float inv_l = 1.f / (l2.x + l2.y);
         __half* orow = o + (static_cast<size_t>(row_base) + q_row) * D;
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {

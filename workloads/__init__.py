@@ -80,8 +80,10 @@ def sweep(N: int, d: int, causal: bool) -> Workload:
 SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768)
 SWEEP_D = (64, 128)
 HEADLINE = sweep(16384, 128, False)
+# a quarter of the headline problem (inputs still larger than L2) for profiler captures
+PROFILE = Workload("profile_b1h16_n16384_d128", 1, 16, 16384, 128, False, True, n_out=4, out_mag=20.0)
 
-ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT)}
+ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
