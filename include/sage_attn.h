@@ -48,7 +48,8 @@ typedef enum {
   SAGE_ERR_UNSUPPORTED = -2, /* valid request outside what the kernels implement (d, N) */
   SAGE_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
   SAGE_ERR_TIMEOUT = -4,     /* a kernel's bounded wait gave up (sage_last_device_error) */
-  SAGE_ERR_NOMEM = -5        /* workspace allocation failed */
+  SAGE_ERR_NOMEM = -5,       /* workspace allocation failed */
+  SAGE_ERR_TOO_LARGE = -6    /* problem needs more than the fixed no-alloc scratch */
 } sage_status;
 
 enum { SAGE_PER_TOKEN = 0, SAGE_PER_BLOCK = 1 };
@@ -102,6 +103,35 @@ int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, i
  * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out).  Returns
  * SAGE_ERR_CUDA (negative) if the synchronization itself failed. */
 int sage_last_device_error(void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Allocation-free variant of sage_attn_fwd.  The SageAttention page has no counterpart of
+ * this entry point: it exists for callers that cannot allocate device memory while they
+ * run -- e.g. code being captured into a CUDA graph that must not contain allocations, or
+ * hosts whose device-memory budget is fixed at start-up -- and so cannot use the
+ * stream-ordered workspace of sage_attn_fwd.
+ *
+ * Same arguments, results and validation as sage_attn_fwd (bit-identical output), but the
+ * workspace (INT8 Q/K, scales, K mean) lives in a scratch array compiled into the library:
+ * SAGE_NOALLOC_SCRATCH_BYTES of device memory that every GPU which loads the library holds
+ * until the process exits.  The call allocates nothing (no cudaMalloc / cudaFree, no
+ * library allocator).  Problems whose workspace, sage_noalloc_scratch_bytes(), exceeds the
+ * scratch size return SAGE_ERR_TOO_LARGE without launching anything.
+ *
+ * The first call on each device looks up the scratch array's device address with
+ * cudaGetSymbolAddress (with that device current) and caches it; make that first call
+ * before any stream capture.  All calls share the one scratch array and nothing in it needs
+ * clearing (every value is rewritten before it is read), but two calls whose work overlaps
+ * on the GPU (different streams, or different host threads on one device) race on it:
+ * serialize them on one stream. */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* Scratch bytes a problem needs: 2*B*H*N*d (INT8 Q, K) plus the scales and the K mean,
+ * each rounded up to 256 bytes.  0 for invalid sizes or granularity. */
+size_t sage_noalloc_scratch_bytes(int B, int H, int N, int d, int granularity);
+
+int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                          int causal, float sm_scale, int granularity, void* stream);
 
 #ifdef __cplusplus
 }

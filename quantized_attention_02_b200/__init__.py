@@ -29,27 +29,39 @@ SAGE_ERR_UNSUPPORTED = -2
 SAGE_ERR_CUDA = -3
 SAGE_ERR_TIMEOUT = -4
 SAGE_ERR_NOMEM = -5
+SAGE_ERR_TOO_LARGE = -6
 SAGE_PER_TOKEN = 0
 SAGE_PER_BLOCK = 1
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m quantized_attention_02_b200.build`")
+_lib = None
 
-lib = ctypes.CDLL(LIB_PATH)
-_i, _f, _p, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
-lib.sage_status_string.argtypes = [_i]
-lib.sage_status_string.restype = ctypes.c_char_p
-lib.sage_scale_count.argtypes = [_i, _i, _i]
-lib.sage_scale_count.restype = _sz
-lib.sage_smooth_k.argtypes = [_p, _p, _i, _i, _i, _i, _p]
-lib.sage_quant_qk.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
-lib.sage_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
-lib.sage_attn_fwd_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
-lib.sage_debug_qk_int32.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p]
-lib.sage_last_device_error.argtypes = [_p]
-for _n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
-           "sage_debug_qk_int32", "sage_last_device_error"):
-    getattr(lib, _n).restype = _i
+
+def get_lib() -> ctypes.CDLL:
+    """The loaded libsage_attn.so (loaded on first use; raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m quantized_attention_02_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        _i, _f, _p, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+        lib.sage_status_string.argtypes = [_i]
+        lib.sage_status_string.restype = ctypes.c_char_p
+        lib.sage_scale_count.argtypes = [_i, _i, _i]
+        lib.sage_scale_count.restype = _sz
+        lib.sage_smooth_k.argtypes = [_p, _p, _i, _i, _i, _i, _p]
+        lib.sage_quant_qk.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+        lib.sage_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_attn_fwd_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_debug_qk_int32.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_last_device_error.argtypes = [_p]
+        lib.sage_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_noalloc_scratch_bytes.argtypes = [_i, _i, _i, _i, _i]
+        lib.sage_noalloc_scratch_bytes.restype = _sz
+        for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
+                  "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc"):
+            getattr(lib, n).restype = _i
+        _lib = lib
+    return _lib
 
 
 class SageError(RuntimeError):
@@ -66,11 +78,11 @@ def header_functions() -> list[str]:
 
 
 def sage_status_string(status: int) -> str:
-    return lib.sage_status_string(int(status)).decode()
+    return get_lib().sage_status_string(int(status)).decode()
 
 
 def sage_scale_count(N: int, granularity: int, is_q: bool) -> int:
-    return int(lib.sage_scale_count(int(N), int(granularity), int(bool(is_q))))
+    return int(get_lib().sage_scale_count(int(N), int(granularity), int(bool(is_q))))
 
 
 def _ptr(t):
@@ -104,37 +116,51 @@ def _check(rc: int, where: str) -> None:
 
 def sage_smooth_k(k: torch.Tensor, km: torch.Tensor, stream=None) -> None:
     B, H, N, d = _shape(k)
-    _check(lib.sage_smooth_k(_ptr(k), _ptr(km), B, H, N, d, _stream(stream)), "sage_smooth_k")
+    _check(get_lib().sage_smooth_k(_ptr(k), _ptr(km), B, H, N, d, _stream(stream)), "sage_smooth_k")
 
 
 def sage_quant_qk(q, k, km, q8, k8, sq, sk, granularity: int, stream=None) -> None:
     B, H, N, d = _shape(q)
-    _check(lib.sage_quant_qk(_ptr(q), _ptr(k), _ptr(km), _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk),
+    _check(get_lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(km), _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk),
                              B, H, N, d, int(granularity), _stream(stream)), "sage_quant_qk")
 
 
 def sage_attn_fwd(q, k, v, o, causal: bool, sm_scale: float, granularity: int, stream=None) -> None:
     B, H, N, d = _shape(q)
-    _check(lib.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+    _check(get_lib().sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
                              float(sm_scale), int(granularity), _stream(stream)), "sage_attn_fwd")
 
 
 def sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float, granularity: int,
                             stream=None) -> None:
     B, H, N, d = _shape(v)
-    _check(lib.sage_attn_fwd_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v), _ptr(o), B, H, N,
+    _check(get_lib().sage_attn_fwd_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v), _ptr(o), B, H, N,
                                        d, int(bool(causal)), float(sm_scale), int(granularity),
                                        _stream(stream)), "sage_attn_fwd_quantized")
 
 
 def sage_debug_qk_int32(q8, k8, s, stream=None) -> None:
     B, H, N, d = _shape(q8)
-    _check(lib.sage_debug_qk_int32(_ptr(q8), _ptr(k8), _ptr(s), B, H, N, d, _stream(stream)),
+    _check(get_lib().sage_debug_qk_int32(_ptr(q8), _ptr(k8), _ptr(s), B, H, N, d, _stream(stream)),
            "sage_debug_qk_int32")
 
 
+def sage_attn_fwd_noalloc(q, k, v, o, causal: bool, sm_scale: float, granularity: int, stream=None) -> None:
+    """sage_attn_fwd for callers that cannot allocate device memory during the call: the
+    workspace is the library's fixed scratch array (SAGE_NOALLOC_SCRATCH_BYTES per GPU).
+    Calls that overlap on the GPU race on that array."""
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+                                     float(sm_scale), int(granularity), _stream(stream)),
+           "sage_attn_fwd_noalloc")
+
+
+def sage_noalloc_scratch_bytes(B: int, H: int, N: int, d: int, granularity: int) -> int:
+    return int(get_lib().sage_noalloc_scratch_bytes(B, H, N, d, granularity))
+
+
 def sage_last_device_error(stream=None) -> int:
-    return int(lib.sage_last_device_error(_stream(stream)))
+    return int(get_lib().sage_last_device_error(_stream(stream)))
 
 
 # ------------------------------------------------------------------ conveniences

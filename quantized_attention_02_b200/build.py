@@ -28,6 +28,7 @@ SOURCES = {
     "capi.cu": [],
     "prep_kernels.cu": ["--fmad=false"],
     "attn_kernels.cu": [],
+    "noalloc.cu": [],
 }
 HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "prep_kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

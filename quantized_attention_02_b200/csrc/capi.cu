@@ -112,6 +112,7 @@ const char* sage_status_string(int status) {
     case SAGE_ERR_CUDA: return "CUDA runtime error";
     case SAGE_ERR_TIMEOUT: return "a kernel wait timed out";
     case SAGE_ERR_NOMEM: return "workspace allocation failed";
+    case SAGE_ERR_TOO_LARGE: return "problem needs more than the no-alloc scratch (SAGE_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

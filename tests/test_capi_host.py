@@ -59,7 +59,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
 ])
 def test_shape_validation(sa, args, expect):
     B, H, N, d = args
-    L = sa.lib
+    L = sa.get_lib()
     s = ctypes.c_void_p(0)
     assert L.sage_smooth_k(FAKE, FAKE, B, H, N, d, s) == expect
     assert L.sage_quant_qk(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, B, H, N, d, 1, s) == expect
@@ -69,7 +69,7 @@ def test_shape_validation(sa, args, expect):
 
 
 def test_null_pointers_and_bad_scalars(sa):
-    L = sa.lib
+    L = sa.get_lib()
     s = ctypes.c_void_p(0)
     assert L.sage_smooth_k(None, FAKE, 1, 1, 128, 64, s) == -1
     assert L.sage_quant_qk(FAKE, FAKE, None, FAKE, None, FAKE, FAKE, 1, 1, 128, 64, 1, s) == -1
