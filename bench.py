@@ -59,31 +59,43 @@ def mixed_peak_tops(p_f16: float) -> float:
 
 # ------------------------------------------------------------------ clocks sampler
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons polled through NVML (read-only queries) every
+    50 ms from a thread of this process while the timed region runs."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.rows = []
+        self.samples = []
         self._stop = threading.Event()
         self._t = None
+        self._nvml = None
 
     def _run(self):
+        nv = self._nvml
+        h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         while not self._stop.is_set():
             try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=5).stdout.strip()
-                if out:
-                    self.rows.append([c.strip() for c in out.split(",")])
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, mx, pw, bits))
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(0.05)
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._nvml = None
         return self
 
     def __exit__(self, *exc):
@@ -92,18 +104,14 @@ class ClockSampler:
             self._t.join(timeout=10)
 
     def summary(self):
-        if not self.rows:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for r in self.rows:
-            for i, n in enumerate(names):
-                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(self.rows)}
+        nv = self._nvml
+        reasons = sorted({name for (_, _, _, bits) in self.samples for name, attr in self.REASONS
+                          if bits & getattr(nv, attr)})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.samples[0][1],
+                "power_w_max": round(max(s[2] for s in self.samples), 1), "reasons": reasons,
+                "samples": len(self.samples), "source": "NVML, 50 ms"}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -214,6 +222,25 @@ def run_ours(args, w: W.Workload):
     torch.cuda.synchronize(dev)
     kernel_ms = k0.elapsed_time(k1) / args.steps
 
+    # ---- per-step breakdown (each entry point alone, same stream, events)
+    def timed(fn, n):
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        b0.record(stream)
+        for _ in range(n):
+            fn()
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        return b0.elapsed_time(b1) / n
+
+    nb = max(3, min(args.steps, 10))
+    breakdown = {
+        "smooth_k_ms": timed(lambda: sa.sage_smooth_k(k, km, stream), nb),
+        "quant_qk_ms": timed(lambda: sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream), nb),
+        "attn_kernel_ms": kernel_ms,
+        "step_ms": ms,
+    }
+
     # ---- end to end through the C ABI with host buffers: H2D inputs, D2H output per step
     qp, kp, vp = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
     op = torch.empty_like(qp).pin_memory()
@@ -242,6 +269,17 @@ def run_ours(args, w: W.Workload):
         e2e_ms = float(t.item())
     if sa.sage_last_device_error(stream) != 0:
         raise RuntimeError("a kernel wait timed out during timing")
+
+    # ---- tensor-core rate probe (the MMA shapes of the fused kernel), for the roofline notes
+    probe = {}
+    try:
+        for mode, n, chains in ((0, 128, 1), (0, 128, 2), (0, 256, 1), (0, 64, 4), (1, 128, 1), (1, 128, 2),
+                                (1, 64, 4), (2, 128, 1), (2, 128, 2), (2, 256, 1)):
+            r = sa.mma_rate(mode, n, chains)
+            probe[f"{r['kind']} N{n} x{chains}"] = {"macs_per_clk_per_sm": round(r["macs_per_clk_per_sm"], 1),
+                                                    "tops": round(r["tops"], 1)}
+    except Exception as exc:  # the probe is informational only
+        probe = {"error": str(exc)}
 
     result = None
     if rank == 0:
@@ -275,6 +313,8 @@ def run_ours(args, w: W.Workload):
             "e2e": {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "ms_per_step": round(e2e_ms, 4)},
+            "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
+            "mma_probe": probe,
             "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
         }
@@ -317,7 +357,7 @@ def run_reference(args, w: W.Workload):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))

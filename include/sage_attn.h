@@ -99,6 +99,31 @@ int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq,
 int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, int H, int N, int d,
                         void* stream);
 
+/* Debug / tracing: sage_attn_fwd_quantized (per-block granularity only) built with SM clock
+ * stamps (clock64) of its pipeline events, for the first trace_ctas CTAs.  Output equals the
+ * untraced kernel's.  trace: int64 [trace_ctas][2 + 10*T] with T = N/128 key tiles, zeroed by
+ * the caller; per CTA: [0] start, [1] end, then for key tile j:
+ *   [2 + (3t+e)*T + j]   softmax warpgroup of query tile t (0/1), event e: 0 = S ready,
+ *                        1 = row max and offset done, 2 = P~ written and signalled;
+ *   [2 + (6+2t+e)*T + j] MMA thread, tile t, event e: 0 = P.V issued, 1 = next Q.K^T issued.
+ * Slots of events that do not happen (causal tiles, a missing second query tile) stay 0.
+ * CTA c works on head c / ceil(N/256) and query tiles 2p, 2p+1 with p = ceil(N/256)-1 - c % ceil(N/256). */
+int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
+                          const void* v, void* o, int B, int H, int N, int d, int causal,
+                          float sm_scale, int granularity, long long* trace, int trace_ctas,
+                          void* stream);
+
+/* Debug: tensor-core throughput probe for the MMA shapes of the fused kernel.  Launches
+ * `ctas` CTAs (use the SM count; one per SM); in each, one thread issues `iters` (<= 2^24)
+ * back-to-back MMAs rotating over `chains` independent accumulators, on zero-filled operands,
+ * and writes the CTA's SM-clock cycles to cycles[cta] (int64 [ctas], device memory).  status
+ * (device int, caller-zeroed) is set to 1 if the final wait gave up.  Modes: 0 = kind::i8 M128
+ * K32 (both operands in shared memory), 1 = kind::f16 M128 K16 (A in tensor memory, B MN-major
+ * in shared memory, n <= 128), 2 = kind::f16 M128 K16 (both in shared memory); n in {64, 128,
+ * 256}, chains in 1..4 with chains*n <= 256.  Multiply-accumulates per MMA: 128*n*K. */
+int sage_debug_mma_rate(int mode, int n, int chains, int iters, int ctas, long long* cycles, int* status,
+                        void* stream);
+
 /* Waits for all work on stream, then returns and clears the device status word written by
  * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out).  Returns
  * SAGE_ERR_CUDA (negative) if the synchronization itself failed. */

@@ -29,6 +29,7 @@ SOURCES = {
     "prep_kernels.cu": ["--fmad=false"],
     "attn_kernels.cu": [],
     "noalloc.cu": [],
+    "mma_rate.cu": [],
 }
 HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "prep_kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

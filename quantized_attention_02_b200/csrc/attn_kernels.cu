@@ -45,7 +45,7 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_SK = OFF_V + STAGES * V_BYTES;           // per-token key scales
   static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 3 * NQT + 1;
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 4 * NQT + 1 + NQT;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int USED = OFF_MISC + 16;
   // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
@@ -93,6 +93,20 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
+// Maximum of 64 signed integers held as bits: four independent chains of one 2-input and
+// seven 3-input maxima (4 * (2 + 7 * 2) = 64 elements, x[0..63] exactly).
+__device__ __forceinline__ int imax64(const uint32_t* x) {
+  int a[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = max(static_cast<int>(x[k]), static_cast<int>(x[4 + k]));
+#pragma unroll
+  for (int i = 8; i < 64; i += 8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = __vimax3_s32(a[k], static_cast<int>(x[i + k]), static_cast<int>(x[i + 4 + k]));
+  }
+  return max(max(a[0], a[1]), max(a[2], a[3]));
+}
+
 template <uint32_t N>
 __device__ __forceinline__ void reg_alloc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -113,12 +127,14 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D, bool CAUSAL, bool PER_TOKEN>
+// TRACE builds record SM clock stamps of the pipeline events of the first trace_ctas CTAs
+// (layout documented at sage_debug_attn_trace in include/sage_attn.h).
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE>
 __global__ void __launch_bounds__(384, 1)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ sq,
                      const float* __restrict__ sk, __half* __restrict__ o, int BH, int N,
-                     float sm_scale_log2) {
+                     float sm_scale_log2, long long* __restrict__ trace, int trace_ctas) {
   using L = AttnLayout<D>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -133,9 +149,11 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_v_full = bars + 1 + STAGES;
   uint64_t* bar_kv_empty = bars + 1 + 2 * STAGES;
   uint64_t* bar_s_full = bars + 1 + 3 * STAGES;
-  uint64_t* bar_p_full = bar_s_full + 2;
+  uint64_t* bar_p_full = bar_s_full + 2;  // P~ of keys 64..127 (the whole tile) written
   uint64_t* bar_o_done = bar_s_full + 4;
   uint64_t* bar_drain = bar_s_full + 6;
+  uint64_t* bar_seq = bar_s_full + 7;     // softmax group t finished the exp2 phase of a key tile
+  uint64_t* bar_p_lo = bar_s_full + 9;    // P~ of keys 0..63 written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -156,6 +174,21 @@ __global__ void __launch_bounds__(384, 1)
   n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
   const int n_kv = max(n_iter[0], n_iter[1]);
   const int row_base = bh * N;  // first row of this head in the [BH*N, D] views
+  long long* trace_row = nullptr;
+  if constexpr (TRACE) {
+    if (static_cast<int>(blockIdx.x) < trace_ctas) {
+      trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * (N / L::BN));
+      if (threadIdx.x == 0) trace_row[0] = clock64();
+    }
+  }
+  // trace slots: [0] start, [1] end, then per key tile j: softmax group t events e (0 S ready,
+  // 1 max done, 2 P~ signalled) at 2 + (3t+e) n_kv_total + j; MMA thread events e (0 P.V issued,
+  // 1 next Q.K^T issued) for tile t at 2 + (6 + 2t + e) n_kv_total + j
+  auto stamp = [&](int slot) {
+    if constexpr (TRACE) {
+      if (trace_row) trace_row[2 + slot] = clock64();
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -170,6 +203,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar_o_done + t, 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_seq, 128);
+    mbar_init(bar_seq + 1, 128);
+    mbar_init(bar_p_lo, 128);
+    mbar_init(bar_p_lo + 1, 128);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
@@ -186,10 +223,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   // Registers: the block is launched with 168 per thread (384 x 168); the control
-  // warpgroup hands most of its share to the two softmax warpgroups: 128 x 56 + 256 x 224.
+  // warpgroup hands most of its share to the two softmax warpgroups: 128 x 72 + 256 x 216.
   // Each setmaxnreg is executed by a whole warpgroup and dominates that group's code.
   if (warp < 4) {
-    reg_dealloc<56>();
+    reg_dealloc<72>();
     if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
@@ -224,63 +261,77 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (uniform control flow and descriptors); elect.sync lets
+    // one lane issue each tcgen05 instruction.
+    {
       constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
       constexpr uint32_t IDESC_PV = make_idesc(1 /*f32*/, 0 /*f16*/, 0 /*f16*/, 0, 1 /*V is MN-major*/, 128, D);
       constexpr SwizzleMode QK_SWZ = D == 128 ? kSwizzle128B : kSwizzle64B;
       constexpr uint32_t QK_SBO = D == 128 ? 1024 : 512;  // 8 rows of D bytes
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
 
       auto issue_qk = [&](int t, int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t a = make_smem_desc(q_base + t * L::Q_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
           const uint64_t b = make_smem_desc(k_base + s * L::K_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
-          mma_i8_ss(tmem + L::s_col(t), a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_i8_ss_warp(tmem + L::s_col(t), a, b, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s_full + t);
+        mma_commit_warp(bar_s_full + t);
       };
-      auto issue_pv = [&](int t, int s, bool first) {
+      // P.V for keys [16*k0, 16*k1) of the tile: 16 keys per MMA = 16 rows of 128 B in the V box
+      // (LBO jumps to the next 64 columns); P~ columns hold two fp16 keys each
+      auto issue_pv = [&](int t, int s, bool first, int k0, int k1) {
 #pragma unroll
-        for (int kk = 0; kk < L::BN / 16; ++kk) {
-          // 16 keys per MMA = 16 rows of 128 B in the V box; LBO jumps to the next 64 columns
+        for (int kk = k0; kk < k1; ++kk) {
           const uint64_t b = make_smem_desc(v_base + s * L::V_BYTES + kk * 16 * 128, L::V_BOX, 1024, kSwizzle128B);
-          mma_f16_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          mma_f16_ts_warp(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
         }
-        mma_commit(bar_o_done + t);
       };
 
-      bool ok = mbar_wait(bar_q, 0, abort_flag) && mbar_wait(bar_k_full, 0, abort_flag);
+      bool ok = wait(bar_q, 0) && wait(bar_k_full, 0);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < n_tiles; ++t) issue_qk(t, 0);
       }
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait(bar_v_full + s, (j / STAGES) & 1, abort_flag)) break;
+        if (!wait(bar_v_full + s, (j / STAGES) & 1)) break;
         for (int t = 0; t < n_tiles && ok; ++t) {
           if (j >= n_iter[t]) continue;
-          if (!mbar_wait(bar_p_full + t, j & 1, abort_flag)) { ok = false; break; }
+          // the first half of P~ is signalled separately, so that its P.V overlaps the
+          // exp2 work on the second half
+          if (!wait(bar_p_lo + t, j & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(t, s, j == 0);
+          if (j == 0) issue_pv(t, s, true, 0, L::BN / 32);
+          else issue_pv(t, s, false, 0, L::BN / 32);
+          if (!wait(bar_p_full + t, j & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, s, false, L::BN / 32, L::BN / 16);
+          mma_commit_warp(bar_o_done + t);
+          if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
           if (j + 1 < n_iter[t]) {
             // S_t(j+1) overwrites P~_t(j): tcgen05 MMAs issued by one thread execute in
             // issue order, so the P.V above has read P~_t before this product writes S_t.
             const int s1 = (j + 1) % STAGES;
-            if (!mbar_wait(bar_k_full + s1, ((j + 1) / STAGES) & 1, abort_flag)) { ok = false; break; }
+            if (!wait(bar_k_full + s1, ((j + 1) / STAGES) & 1)) { ok = false; break; }
             tc_fence_after();
             issue_qk(t, s1);
+            if (lane == 0) stamp((7 + 2 * t) * n_kv_total + j);
           }
         }
-        mma_commit(bar_kv_empty + s);
+        mma_commit_warp(bar_kv_empty + s);
       }
-      // all MMAs issued by this thread must finish before TMEM is released
-      mma_commit(bar_drain);
+      // all MMAs issued by this warp must finish before TMEM is released
+      mma_commit_warp(bar_drain);
       mbar_drain(bar_drain, 0);
     }
     }
   } else {
-    reg_alloc<224>();
+    reg_alloc<216>();
     // ================================================================ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
@@ -315,45 +366,44 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < n_iter[t]; ++j) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
+        if (r == 0) stamp((3 * t) * n_kv_total + j);
         uint32_t x[128];
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(x + 0));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(x + 64));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(x + 96));
-        tmem_wait_ld();
+        tmem_ld64_sync(tS + 0, *reinterpret_cast<uint32_t(*)[64]>(x + 0));
+        tmem_ld64_sync(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(x + 64));
 
         const bool diag = CAUSAL && (j == q_tile);
         const int s = j % STAGES;
-        // f = kMagic + S exactly (|S| < 2^22), as float bits
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] += kMagicBits;
-        if (diag) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > r) x[c] = 0xFF800000u;  // -inf: masked key
-        }
-
         float mx;            // row maximum of the dequantized scores (log2 units)
         float cb0 = 0.f, cb1 = 0.f, nb0 = 0.f, nb1 = 0.f;
         const float* skj = sSK + s * L::BN;
         if constexpr (PER_TOKEN) {
+          // f = kMagic + S exactly (|S| < 2^22), as float bits; masked keys -inf
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = (diag && c > r) ? 0xFF800000u : x[c] + kMagicBits;
           if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
           mx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             mx = fmaxf(mx, (__uint_as_float(x[c]) - kMagicF) * (a_r * skj[c]));
         } else {
+          // integer maxima of the two 64-key halves (one key scale each); masked keys INT_MIN
           cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
           cb1 = trim_scale(a_r * __ldg(sk_head + 2 * j + 1));
-          float f0 = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
-          float f1 = max3f(__uint_as_float(x[64]), __uint_as_float(x[65]), __uint_as_float(x[66]));
+          if (diag) {
 #pragma unroll
-          for (int c = 3; c < 63; c += 2) f0 = max3f(f0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-          f0 = fmaxf(f0, __uint_as_float(x[63]));
+            for (int c = 0; c < 64; ++c)
+              if (c > r) x[c] = 0x80000000u;
+          }
+          const int im0 = imax64(x);
+          if (diag) {
 #pragma unroll
-          for (int c = 67; c < 127; c += 2) f1 = max3f(f1, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-          f1 = fmaxf(f1, __uint_as_float(x[127]));
-          mx = fmaxf(cb0 * (f0 - kMagicF), cb1 * (f1 - kMagicF));  // -inf halves stay -inf
+            for (int c = 64; c < 128; ++c)
+              if (c > r) x[c] = 0x80000000u;
+          }
+          const int im1 = imax64(x + 64);
+          const float m0 = im0 == INT_MIN ? -INFINITY : cb0 * static_cast<float>(im0);
+          const float m1 = im1 == INT_MIN ? -INFINITY : cb1 * static_cast<float>(im1);
+          mx = fmaxf(m0, m1);
         }
 
         // ---- rescale only when the maximum grew by more than 2^8 (bounds P~ by 256)
@@ -375,8 +425,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int cb = 0; cb < D; cb += 32) {
             uint32_t ov[32];
-            tmem_ld32(tO + cb, ov);
-            tmem_wait_ld();
+            tmem_ld32_sync(tO + cb, ov);
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
             tmem_st32(tO + cb, ov);
@@ -385,6 +434,16 @@ __global__ void __launch_bounds__(384, 1)
         if constexpr (!PER_TOKEN) {
           nb0 = -fmaf(kMagicF, cb0, m_use);  // exact: see offset_quantum above
           nb1 = -fmaf(kMagicF, cb1, m_use);
+        }
+        if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
+
+        // ---- the two softmax groups take turns on the exp2 unit: group 0 runs key tile j
+        // after group 1 finished tile j-1, group 1 after group 0 finished tile j
+        if (n_tiles > 1) {
+          bool go = true;
+          if (t == 0 && j > 0) go = mbar_wait(bar_seq + 1, (j - 1) & 1, abort_flag);
+          if (t == 1 && j < n_iter[0]) go = mbar_wait(bar_seq, j & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, go)) { ok = false; break; }
         }
 
         // ---- P~ = exp2(s - m_use) in fp16; the row sum takes the unrounded values
@@ -401,8 +460,9 @@ __global__ void __launch_bounds__(384, 1)
             } else {
               const float cs = c < 64 ? cb0 : cb1;
               const float nb = c < 64 ? nb0 : nb1;
-              tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), make_float2(cs, cs),
-                              make_float2(nb, nb));
+              // kMagic + S as float (exact), then one rounding: fl(S * c' - m_use)
+              tt = __ffma2_rn(make_float2(__uint_as_float(x[c] + kMagicBits), __uint_as_float(x[c + 1] + kMagicBits)),
+                              make_float2(cs, cs), make_float2(nb, nb));
             }
             float2 p = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
             if (diag) {
@@ -413,10 +473,17 @@ __global__ void __launch_bounds__(384, 1)
             pk[i >> 1] = pack_half2(p.x, p.y);
           }
           tmem_st16(tS + (cb >> 1), pk);
+          if (cb == 32) {  // keys 0..63 done: let their P.V start
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_p_lo + t);
+          }
         }
+        if (n_tiles > 1) mbar_arrive(bar_seq + t);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p_full + t);
+        if (r == 0) stamp((3 * t + 2) * n_kv_total + j);
       }
 
       // ---- epilogue: O / l -> fp16 -> global
@@ -428,8 +495,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t ov[32];
-          tmem_ld32(tO + cb, ov);
-          tmem_wait_ld();
+          tmem_ld32_sync(tO + cb, ov);
           uint32_t hv[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -444,6 +510,9 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (TRACE) {
+    if (trace_row && threadIdx.x == 0) trace_row[1] = clock64();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -533,8 +602,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int cb = 0; cb < BN; cb += 32) {
         uint32_t v[32];
-        tmem_ld32(tS + cb, v);
-        tmem_wait_ld();
+        tmem_ld32_sync(tS + cb, v);
         uint4* dst = reinterpret_cast<uint4*>(srow + j * BN + cb);
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -552,10 +620,10 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // ---------------------------------------------------------------- launchers
-template <int D, bool CAUSAL, bool PER_TOKEN>
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE = false>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<D>;
-  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN>;
+  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN, TRACE>;
   static bool configured = false;  // attribute set once per instantiation (idempotent)
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
@@ -565,7 +633,8 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   const int n_qtiles = a.N / L::BM;
   const int n_pairs = (n_qtiles + 1) / 2;
   dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
-  kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sq, a.sk, a.o, a.BH, a.N, a.sm_scale_log2);
+  kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sq, a.sk, a.o, a.BH, a.N, a.sm_scale_log2,
+                                          a.trace, a.trace_ctas);
   return cudaGetLastError();
 }
 
@@ -576,6 +645,11 @@ static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  if (a.trace) {  // traced builds exist for per-block granularity only
+    if (a.per_token) return cudaErrorNotSupported;
+    if (a.D == 128) return a.causal ? launch_attn_t<128, true, false, true>(a, st) : launch_attn_t<128, false, false, true>(a, st);
+    return a.causal ? launch_attn_t<64, true, false, true>(a, st) : launch_attn_t<64, false, false, true>(a, st);
+  }
   return a.D == 128 ? launch_attn_d<128>(a, st) : launch_attn_d<64>(a, st);
 }
 

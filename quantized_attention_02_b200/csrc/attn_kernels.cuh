@@ -17,6 +17,8 @@ struct AttnArgs {
   int BH, N, D;
   bool causal, per_token;
   float sm_scale_log2;      // sm_scale * log2(e)
+  long long* trace = nullptr;  // non-null: traced build, stamps of the first trace_ctas CTAs
+  int trace_ctas = 0;
 };
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);

@@ -78,7 +78,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CU
 
 int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v, void* o,
                         int B, int H, int N, int d, int causal, float sm_scale, int granularity,
-                        cudaStream_t st) {
+                        cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0) {
   const int BH = B * H;
   const long long rows = static_cast<long long>(BH) * N;
   CUtensorMap tq, tk, tv;
@@ -97,7 +97,10 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
   a.causal = causal != 0;
   a.per_token = granularity == SAGE_PER_TOKEN;
   a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
-  return cuda_status(sage::launch_attn(a, st));
+  a.trace = trace;
+  a.trace_ctas = trace_ctas;
+  const cudaError_t e = sage::launch_attn(a, st);
+  return e == cudaErrorNotSupported ? SAGE_ERR_UNSUPPORTED : cuda_status(e);
 }
 
 }  // namespace
@@ -211,6 +214,20 @@ int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, i
   CUtensorMap tq, tk;
   if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d)) return SAGE_ERR_CUDA;
   return cuda_status(sage::launch_qk_debug(tq, tk, s, B * H, N, d, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v,
+                          void* o, int B, int H, int N, int d, int causal, float sm_scale, int granularity,
+                          long long* trace, int trace_ctas, void* stream) {
+  if (!trace || trace_ctas <= 0) return SAGE_ERR_INVALID;
+  if (granularity != SAGE_PER_BLOCK) return SAGE_ERR_UNSUPPORTED;
+  if (!q8 || !k8 || !sq || !sk || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_scale(sm_scale))) return rc;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
+  return attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity,
+                             static_cast<cudaStream_t>(stream), trace, trace_ctas);
 }
 
 int sage_last_device_error(void* stream) {

@@ -25,12 +25,14 @@ __device__ __forceinline__ long long half_bits_to_fixed(uint32_t h) {
   return (h & 0x8000u) ? -mag : mag;
 }
 
-// One CTA per (32-channel chunk, head).  256 threads: thread = (token phase 0..63, 16-byte
-// piece 0..3 of the 64-byte chunk row).  Loads are 16-byte vectors, 64 tokens per pass, so a
-// warp reads 8 tokens x 64 contiguous bytes.
+// One CTA of 1024 threads per (32-channel chunk, head): thread = (token phase 0..255, 16-byte
+// piece 0..3 of the 64-byte chunk row).  Each thread keeps four 16-byte loads in flight
+// (tokens t, t+256, t+512, t+768) so that the whole GPU has enough bytes in flight to run
+// at HBM speed even with few heads.
 template <int D>
-__global__ void __launch_bounds__(256) smooth_k_kernel(const __half* __restrict__ k, float* __restrict__ km,
-                                                       int N) {
+__global__ void __launch_bounds__(1024) smooth_k_kernel(const __half* __restrict__ k, float* __restrict__ km,
+                                                        int N) {
+  constexpr int PHASES = 256;
   const int chunk = blockIdx.x;  // 32 channels
   const int bh = blockIdx.y;
   const int piece = threadIdx.x & 3;
@@ -41,13 +43,20 @@ __global__ void __launch_bounds__(256) smooth_k_kernel(const __half* __restrict_
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0;
 
-  for (int t = tok0; t < N; t += 64) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t) * D));
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  for (int t = tok0; t < N; t += 4 * PHASES) {
+    uint4 w[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] += half_bits_to_fixed(words[i] & 0xFFFFu);
-      acc[2 * i + 1] += half_bits_to_fixed(words[i] >> 16);
+    for (int u = 0; u < 4; ++u)
+      w[u] = (t + u * PHASES < N) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * PHASES) * D))
+                                  : make_uint4(0u, 0u, 0u, 0u);  // +0.0 contributes nothing
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += half_bits_to_fixed(words[i] & 0xFFFFu);
+        acc[2 * i + 1] += half_bits_to_fixed(words[i] >> 16);
+      }
     }
   }
   // lanes sharing `piece` differ in lane bits 2..4
@@ -56,7 +65,7 @@ __global__ void __launch_bounds__(256) smooth_k_kernel(const __half* __restrict_
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
   }
-  __shared__ long long part[8][4][8];
+  __shared__ long long part[32][4][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane < 4) {
 #pragma unroll
@@ -67,7 +76,7 @@ __global__ void __launch_bounds__(256) smooth_k_kernel(const __half* __restrict_
     const int p = threadIdx.x >> 3, i = threadIdx.x & 7;  // channel = chunk*32 + p*8 + i
     long long s = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][p][i];
+    for (int w = 0; w < 32; ++w) s += part[w][p][i];
     const float s32 = __ll2float_rn(s);
     const float mean = __fdiv_rn(s32, static_cast<float>(N));
     km[static_cast<size_t>(bh) * D + chunk * 32 + p * 8 + i] = __fmul_rn(mean, 5.9604644775390625e-08f);
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
 template <int D>
 static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cudaStream_t st) {
   dim3 grid(D / 32, BH);
-  smooth_k_kernel<D><<<grid, 256, 0, st>>>(k, km, N);
+  smooth_k_kernel<D><<<grid, 1024, 0, st>>>(k, km, N);
   return cudaGetLastError();
 }
 

@@ -122,10 +122,14 @@ def test_small_full_parity(sa, w):
 
 
 def test_causal_first_row_equals_first_value_row(sa):
+    # Row 0 sees key 0 only: O[0] = fp16(fp16(p) * V[0] / p) for the single weight p.  The
+    # kernel's exponent offset may sit up to one offset quantum above the row maximum, so p
+    # can be just below 1 and each fp16 rounding adds at most 2^-11 relative error.
     w = W.Workload("c0", 1, 2, 256, 128, True, True, n_out=4, out_mag=20.0)
     q, k, v = W.make_qkv(w)
     o = sa.sageattn(q.cuda(), k.cuda(), v.cuda(), True, w.sm_scale, 1).cpu()
-    assert torch.equal(o[:, :, 0], v[:, :, 0])
+    v0 = v[:, :, 0].double()
+    assert torch.all((o[:, :, 0].double() - v0).abs() <= 2.0**-10 * v0.abs() + 1e-7)
 
 
 def test_zero_queries_give_prefix_means(sa):
@@ -234,3 +238,31 @@ def _exact_rows(qh, kh, vh, rows, w):
     s -= s.max(axis=1, keepdims=True)
     e = np.exp(s)
     return (e / e.sum(axis=1, keepdims=True)) @ vf
+
+
+def test_traced_kernel_matches_untraced_and_stamps_are_ordered(sa):
+    w = W.Workload("trace_b1h2_n1024_d128", 1, 2, 1024, 128, False, True, n_out=4, out_mag=20.0)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    km, q8, k8, sq, sk = sa.empty_quantized(q, 1)
+    sa.sage_smooth_k(k, km)
+    sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, 1)
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o1, w.causal, w.sm_scale, 1)
+    T = w.N // 128
+    tr = torch.zeros((3, 2 + 10 * T), dtype=torch.int64, device="cuda")
+    sa.sage_debug_attn_trace(q8, k8, sq, sk, v, o2, w.causal, w.sm_scale, 1, tr, 3)
+    torch.cuda.synchronize()
+    assert sa.sage_last_device_error() == 0
+    assert torch.equal(o1, o2)
+    tr = tr.cpu().numpy()
+    assert np.all(tr[:, 1] > tr[:, 0])
+    for t in range(2):
+        s_ready = tr[:, 2 + 3 * t * T: 2 + (3 * t + 1) * T]
+        p_sig = tr[:, 2 + (3 * t + 2) * T: 2 + (3 * t + 3) * T]
+        assert np.all(p_sig > s_ready) and np.all(np.diff(s_ready, axis=1) > 0)
+
+
+def test_mma_rate_probe_runs(sa):
+    for mode, n, chains in ((0, 128, 1), (0, 256, 1), (1, 128, 2), (2, 64, 4)):
+        r = sa.mma_rate(mode, n, chains, iters=2000)
+        assert 100 < r["macs_per_clk_per_sm"] < 100000 and r["tops"] > 1
