@@ -114,15 +114,16 @@ int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, c
                           void* stream);
 
 /* Debug: tensor-core throughput probe for the MMA shapes of the fused kernel.  Launches
- * `ctas` CTAs (use the SM count; one per SM); in each, one thread issues `iters` (<= 2^24)
- * back-to-back MMAs rotating over `chains` independent accumulators, on zero-filled operands,
- * and writes the CTA's SM-clock cycles to cycles[cta] (int64 [ctas], device memory).  status
- * (device int, caller-zeroed) is set to 1 if the final wait gave up.  Modes: 0 = kind::i8 M128
- * K32 (both operands in shared memory), 1 = kind::f16 M128 K16 (A in tensor memory, B MN-major
- * in shared memory, n <= 128), 2 = kind::f16 M128 K16 (both in shared memory); n in {64, 128,
- * 256}, chains in 1..4 with chains*n <= 256.  Multiply-accumulates per MMA: 128*n*K. */
-int sage_debug_mma_rate(int mode, int n, int chains, int iters, int ctas, long long* cycles, int* status,
-                        void* stream);
+ * `ctas` CTAs (use the SM count; one per SM); in each, `issuers` warps (1 or 2) issue back-to-back
+ * MMAs, iters/issuers each (iters a multiple of 4*issuers, <= 2^24), each warp rotating over its
+ * own `chains` accumulators, on zero-filled operands; issuer 0 writes the CTA's SM-clock cycles
+ * to cycles[cta] (int64 [ctas], device memory).  status (device int, caller-zeroed) is set to 1
+ * if a final wait gave up.  Modes: 0 = kind::i8 M128 K32 (both operands in shared memory),
+ * 1 = kind::f16 M128 K16 (A in tensor memory, B MN-major in shared memory, n <= 128), 2 =
+ * kind::f16 M128 K16 (both in shared memory); n in {64, 128, 256}; chains in {1, 2, 4};
+ * issuers*chains*n <= 256.  Multiply-accumulates per MMA: 128*n*K. */
+int sage_debug_mma_rate(int mode, int n, int chains, int issuers, int iters, int ctas, long long* cycles,
+                        int* status, void* stream);
 
 /* Waits for all work on stream, then returns and clears the device status word written by
  * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out).  Returns

@@ -58,7 +58,7 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_noalloc_scratch_bytes.argtypes = [_i, _i, _i, _i, _i]
         lib.sage_noalloc_scratch_bytes.restype = _sz
         lib.sage_debug_attn_trace.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _i, _p]
-        lib.sage_debug_mma_rate.argtypes = [_i, _i, _i, _i, _i, _p, _p, _p]
+        lib.sage_debug_mma_rate.argtypes = [_i, _i, _i, _i, _i, _i, _p, _p, _p]
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
                   "sage_debug_attn_trace", "sage_debug_mma_rate"):
@@ -160,7 +160,7 @@ def sage_debug_attn_trace(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float, g
 MMA_PROBE_KINDS = {0: ("i8", 32), 1: ("f16 A-from-TMEM", 16), 2: ("f16", 16)}
 
 
-def mma_rate(mode: int, n: int = 128, chains: int = 1, iters: int = 20000) -> dict:
+def mma_rate(mode: int, n: int = 128, chains: int = 1, issuers: int = 1, iters: int = 20000) -> dict:
     """Run the tensor-core probe on every SM; return MACs per SM clock and the whole-GPU
     rate in TOPS (2 ops per multiply-accumulate) timed with CUDA events."""
     dev = torch.cuda.current_device()
@@ -170,10 +170,10 @@ def mma_rate(mode: int, n: int = 128, chains: int = 1, iters: int = 20000) -> di
     kind, K = MMA_PROBE_KINDS[mode]
     st = torch.cuda.current_stream()
     lib = get_lib()
-    _check(lib.sage_debug_mma_rate(mode, n, chains, 64, sms, _ptr(cycles), _ptr(status), _stream(st)), "mma_rate")
+    _check(lib.sage_debug_mma_rate(mode, n, chains, issuers, 64, sms, _ptr(cycles), _ptr(status), _stream(st)), "mma_rate")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
-    _check(lib.sage_debug_mma_rate(mode, n, chains, iters, sms, _ptr(cycles), _ptr(status), _stream(st)),
+    _check(lib.sage_debug_mma_rate(mode, n, chains, issuers, iters, sms, _ptr(cycles), _ptr(status), _stream(st)),
            "mma_rate")
     e1.record(st)
     torch.cuda.synchronize()
@@ -181,7 +181,7 @@ def mma_rate(mode: int, n: int = 128, chains: int = 1, iters: int = 20000) -> di
         raise RuntimeError("mma_rate wait gave up")
     macs = 128 * n * K * iters
     cyc = float(cycles.double().median())
-    return {"mode": mode, "kind": kind, "shape": [128, n, K], "chains": chains,
+    return {"mode": mode, "kind": kind, "shape": [128, n, K], "chains": chains, "issuers": issuers,
             "macs_per_clk_per_sm": macs / cyc,
             "tops": 2.0 * macs * sms / (e0.elapsed_time(e1) * 1e-3) / 1e12}
 

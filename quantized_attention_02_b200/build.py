@@ -31,7 +31,7 @@ SOURCES = {
     "noalloc.cu": [],
     "mma_rate.cu": [],
 }
-HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "prep_kernels.cuh"]
+HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -45,7 +45,7 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_SK = OFF_V + STAGES * V_BYTES;           // per-token key scales
   static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 4 * NQT + 1 + NQT;
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 6 * NQT;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int USED = OFF_MISC + 16;
   // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
@@ -151,9 +151,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_s_full = bars + 1 + 3 * STAGES;
   uint64_t* bar_p_full = bar_s_full + 2;  // P~ of keys 64..127 (the whole tile) written
   uint64_t* bar_o_done = bar_s_full + 4;
-  uint64_t* bar_drain = bar_s_full + 6;
-  uint64_t* bar_seq = bar_s_full + 7;     // softmax group t finished the exp2 phase of a key tile
-  uint64_t* bar_p_lo = bar_s_full + 9;    // P~ of keys 0..63 written
+  uint64_t* bar_drain = bar_s_full + 6;   // one per MMA warp
+  uint64_t* bar_seq = bar_s_full + 8;     // softmax group t finished the exp2 phase of a key tile
+  uint64_t* bar_p_lo = bar_s_full + 10;   // P~ of keys 0..63 written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_k_full + s, 1);
       mbar_init(bar_v_full + s, 1);
-      mbar_init(bar_kv_empty + s, 1);
+      mbar_init(bar_kv_empty + s, n_tiles);  // one commit from each MMA warp
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + t, 1);
@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar_o_done + t, 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_drain + 1, 1);
     mbar_init(bar_seq, 128);
     mbar_init(bar_seq + 1, 128);
     mbar_init(bar_p_lo, 128);
@@ -259,24 +260,27 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    // The whole warp runs this loop (uniform control flow and descriptors); elect.sync lets
-    // one lane issue each tcgen05 instruction.
-    {
+  } else if (warp == 1 || warp == 2) {
+    // ================================================================ MMA warps
+    // Warp 1 issues the products of query tile 0, warp 2 those of tile 1: one tcgen05.mma stream
+    // per warp leaves the tensor core idle between back-to-back instructions (about 110-140
+    // cycles each), two independent streams keep it busy.  The whole warp runs the loop
+    // (uniform control flow and descriptors); elect.sync lets one lane issue each instruction.
+    const int t = warp - 1;
+    if (t < n_tiles) {
       constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
       constexpr uint32_t IDESC_PV = make_idesc(1 /*f32*/, 0 /*f16*/, 0 /*f16*/, 0, 1 /*V is MN-major*/, 128, D);
       constexpr SwizzleMode QK_SWZ = D == 128 ? kSwizzle128B : kSwizzle64B;
       constexpr uint32_t QK_SBO = D == 128 ? 1024 : 512;  // 8 rows of D bytes
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      const uint32_t q_base = smem_u32(sQ) + t * L::Q_BYTES, k_base = smem_u32(sK), v_base = smem_u32(sV);
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
       };
 
-      auto issue_qk = [&](int t, int s) {
+      auto issue_qk = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
-          const uint64_t a = make_smem_desc(q_base + t * L::Q_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
+          const uint64_t a = make_smem_desc(q_base + kk * 32, 16, QK_SBO, QK_SWZ);
           const uint64_t b = make_smem_desc(k_base + s * L::K_BYTES + kk * 32, 16, QK_SBO, QK_SWZ);
           mma_i8_ss_warp(tmem + L::s_col(t), a, b, IDESC_QK, kk > 0 ? 1u : 0u);
         }
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       // P.V for keys [16*k0, 16*k1) of the tile: 16 keys per MMA = 16 rows of 128 B in the V box
       // (LBO jumps to the next 64 columns); P~ columns hold two fp16 keys each
-      auto issue_pv = [&](int t, int s, bool first, int k0, int k1) {
+      auto issue_pv = [&](int s, bool first, int k0, int k1) {
 #pragma unroll
         for (int kk = k0; kk < k1; ++kk) {
           const uint64_t b = make_smem_desc(v_base + s * L::V_BYTES + kk * 16 * 128, L::V_BOX, 1024, kSwizzle128B);
@@ -295,39 +299,36 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = wait(bar_q, 0) && wait(bar_k_full, 0);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < n_tiles; ++t) issue_qk(t, 0);
+        issue_qk(0);
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
+      for (int j = 0; ok && j < n_iter[t]; ++j) {
         const int s = j % STAGES;
         if (!wait(bar_v_full + s, (j / STAGES) & 1)) break;
-        for (int t = 0; t < n_tiles && ok; ++t) {
-          if (j >= n_iter[t]) continue;
-          // the first half of P~ is signalled separately, so that its P.V overlaps the
-          // exp2 work on the second half
-          if (!wait(bar_p_lo + t, j & 1)) { ok = false; break; }
+        // the first half of P~ is signalled separately, so that its P.V overlaps the exp2
+        // work on the second half
+        if (!wait(bar_p_lo + t, j & 1)) break;
+        tc_fence_after();
+        if (j == 0) issue_pv(s, true, 0, L::BN / 32);
+        else issue_pv(s, false, 0, L::BN / 32);
+        if (!wait(bar_p_full + t, j & 1)) break;
+        tc_fence_after();
+        issue_pv(s, false, L::BN / 32, L::BN / 16);
+        mma_commit_warp(bar_o_done + t);
+        if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
+        if (j + 1 < n_iter[t]) {
+          // S_t(j+1) overwrites P~_t(j): tcgen05 MMAs issued by one thread execute in issue
+          // order, so the P.V above has read P~_t before this product writes S_t.
+          const int s1 = (j + 1) % STAGES;
+          if (!wait(bar_k_full + s1, ((j + 1) / STAGES) & 1)) break;
           tc_fence_after();
-          if (j == 0) issue_pv(t, s, true, 0, L::BN / 32);
-          else issue_pv(t, s, false, 0, L::BN / 32);
-          if (!wait(bar_p_full + t, j & 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, s, false, L::BN / 32, L::BN / 16);
-          mma_commit_warp(bar_o_done + t);
-          if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
-          if (j + 1 < n_iter[t]) {
-            // S_t(j+1) overwrites P~_t(j): tcgen05 MMAs issued by one thread execute in
-            // issue order, so the P.V above has read P~_t before this product writes S_t.
-            const int s1 = (j + 1) % STAGES;
-            if (!wait(bar_k_full + s1, ((j + 1) / STAGES) & 1)) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(t, s1);
-            if (lane == 0) stamp((7 + 2 * t) * n_kv_total + j);
-          }
+          issue_qk(s1);
+          if (lane == 0) stamp((7 + 2 * t) * n_kv_total + j);
         }
-        mma_commit_warp(bar_kv_empty + s);
+        mma_commit_warp(bar_kv_empty + s);  // this tile's products reading stage s are issued
       }
       // all MMAs issued by this warp must finish before TMEM is released
-      mma_commit_warp(bar_drain);
-      mbar_drain(bar_drain, 0);
+      mma_commit_warp(bar_drain + t);
+      mbar_drain(bar_drain + t, 0);
     }
     }
   } else {
@@ -519,6 +520,8 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
+#include "attn_v3.cuh"
+
 // ---------------------------------------------------------------- debug: INT32 S = q8 k8^T
 // One CTA per (128-row query tile, head).  Thread 0 issues the TMA loads and the same
 // kind::i8 MMA as the fused kernel; warps 4-7 copy S from TMEM to global memory.
@@ -638,6 +641,23 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE = false>
+static cudaError_t launch_attn_v3(const AttnArgs& a, cudaStream_t st) {
+  using L = V3Layout;
+  auto kern = sage_attn_v3_kernel<CAUSAL, PER_TOKEN, TRACE>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int n_pairs = (a.N / L::BM + 1) / 2;
+  dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
+  kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.sq, a.sk, a.BH, a.N, a.sm_scale_log2,
+                                          a.trace, a.trace_ctas);
+  return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
   if (a.causal) return a.per_token ? launch_attn_t<D, true, true>(a, st) : launch_attn_t<D, true, false>(a, st);
@@ -647,10 +667,14 @@ static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   if (a.trace) {  // traced builds exist for per-block granularity only
     if (a.per_token) return cudaErrorNotSupported;
-    if (a.D == 128) return a.causal ? launch_attn_t<128, true, false, true>(a, st) : launch_attn_t<128, false, false, true>(a, st);
+    if (a.D == 128) return a.causal ? launch_attn_v3<true, false, true>(a, st) : launch_attn_v3<false, false, true>(a, st);
     return a.causal ? launch_attn_t<64, true, false, true>(a, st) : launch_attn_t<64, false, false, true>(a, st);
   }
-  return a.D == 128 ? launch_attn_d<128>(a, st) : launch_attn_d<64>(a, st);
+  if (a.D == 128) {
+    if (a.causal) return a.per_token ? launch_attn_v3<true, true>(a, st) : launch_attn_v3<true, false>(a, st);
+    return a.per_token ? launch_attn_v3<false, true>(a, st) : launch_attn_v3<false, false>(a, st);
+  }
+  return launch_attn_d<64>(a, st);
 }
 
 template <int D>

@@ -1,0 +1,526 @@
+// attn_v3.cuh -- the fused attention kernel for head dimension 128, with P.V computed
+// transposed: O^T[d, q] += V^T[d, keys] . P~^T[keys, q], one product stream per query tile
+// (M = 128 = d, N = 128 queries, K = 16 keys), each issued by its own warp.
+//
+// Why this shape: one warp issuing tcgen05.mma gets about one instruction per 110-140 cycles
+// whatever N is (up to 256), so at N = 128 a single issuing warp keeps the tensor core about half
+// busy; several issuing warps overlap.  Here three warps issue: Q.K^T for both query tiles, and
+// one P.V stream per tile.  Transposed, P~ is the B operand and lives in shared memory in the
+// 128-byte-swizzled K-major layout the tensor core reads, and O^T has the head dimension on the
+// TMEM lanes, so a separate correction warpgroup (thread = head dimension) rescales the O^T
+// columns of the queries whose softmax offset moved, off the softmax warps' path.
+//
+// Included by attn_kernels.cu inside namespace sage (one translation unit with the PTX helpers).
+#pragma once
+
+struct V3Layout {
+  static constexpr int D = 128;
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int SK = 3;                // K stages
+  static constexpr int SV = 2;                // V stages
+  static constexpr int Q_BYTES = BM * D;      // int8 tile
+  static constexpr int K_BYTES = BN * D;      // int8 tile
+  static constexpr int V_BOX = BN * 128;      // one 64-column fp16 box (128-byte rows)
+  static constexpr int V_BYTES = BN * D * 2;  // two boxes
+  static constexpr int P_ATOM = 256 * 128;    // 64 keys x 256 query rows of fp16 P~
+  static constexpr int P_BYTES = 2 * P_ATOM;  // 128 keys
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + SK * K_BYTES;
+  static constexpr int OFF_P = OFF_V + SV * V_BYTES;
+  static constexpr int OFF_ALPHA = OFF_P + P_BYTES;       // [2][256] fp32 rescale factors
+  static constexpr int OFF_L = OFF_ALPHA + 2 * 256 * 4;   // [256] fp32 row sums
+  static constexpr int OFF_FLAG = OFF_L + 256 * 4;        // [2][3] int rescale votes
+  static constexpr int OFF_BAR = OFF_FLAG + 32;
+  // q, k_full/empty, v_full/empty, then per tile: s_full, s_free, p_lo, p_hi, o_lo, o_done, vote,
+  // corr_done, l_ready, drain, plus the Q.K^T warp's drain and 1 epilogue barrier
+  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 10 * 2 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr int THREADS = 512;
+};
+static_assert(V3Layout::SMEM <= 227 * 1024, "shared memory budget");
+
+// exp2 on the FMA pipe for a pair of arguments (Cody-Waite style range reduction plus a
+// polynomial), to take part of the exp2 work off the MUFU unit:
+//   t -> max(t, -126); n = round_to_nearest(t) via the 1.5 * 2^23 add; f = t - n in [-1/2, 1/2];
+//   2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 with coefficients fitted here to the minimax relative error on
+//   [-1/2, 1/2] (max relative error 7.5e-5, below half an fp16 ulp); 2^n by adding n to the
+//   exponent field (n << 23, taken from the low bits of the magic sum).
+__device__ __forceinline__ float2 exp2_poly2(float2 t) {
+  constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f, c2 = 0.2426108568906784f,
+                  c3 = 0.055171459913253784f;
+  t.x = fmaxf(t.x, -126.f);
+  t.y = fmaxf(t.y, -126.f);
+  const float2 y = __fadd2_rn(t, make_float2(kMagicF, kMagicF));
+  const float2 n = __fadd2_rn(y, make_float2(-kMagicF, -kMagicF));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), t);
+  float2 p = __ffma2_rn(f, make_float2(c3, c3), make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(y.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(y.y) << 23)));
+}
+
+// CTA-wide vote helpers -----------------------------------------------------------------
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Warp roles (16 warps):
+//   0   TMA producer: Q tiles once, then K and V tiles through their rings
+//   1 / 3  MMA warps: O^T_t += V^T . P~_t^T for query tile 0 / 1 (warp 1 also allocates TMEM)
+//   2   MMA warp: S_t = Q_t . K^T for both query tiles
+//   4-7 / 8-11  softmax of query tile 0 / 1 (thread = query row = TMEM lane of S)
+//   12-15       correction and epilogue (thread = head dimension d = TMEM lane of O^T):
+//               rescales the O^T columns of rows whose offset moved, then normalizes by 1/l,
+//               stages O in shared memory and TMA-stores it.
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE>
+__global__ void __launch_bounds__(512, 1)
+    sage_attn_v3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                        const float* __restrict__ sq, const float* __restrict__ sk, int BH, int N,
+                        float sm_scale_log2, long long* __restrict__ trace, int trace_ctas) {
+  using L = V3Layout;
+  constexpr int D = L::D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sP = smem + L::OFF_P;
+  float* sAlpha = reinterpret_cast<float*>(smem + L::OFF_ALPHA);  // [2][256] per-query rescale factor
+  float* sL = reinterpret_cast<float*>(smem + L::OFF_L);          // [256] 1 / row sum
+  int* sFlag = reinterpret_cast<int*>(smem + L::OFF_FLAG);        // [2 tiles][3 slots] rescale votes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_k_full = bar_q + 1;
+  uint64_t* bar_k_empty = bar_k_full + L::SK;
+  uint64_t* bar_v_full = bar_k_empty + L::SK;
+  uint64_t* bar_v_empty = bar_v_full + L::SV;
+  uint64_t* bar_s_full = bar_v_empty + L::SV;  // [2] Q.K^T of tile t done
+  uint64_t* bar_s_free = bar_s_full + 2;       // [2] softmax t has read S_t
+  uint64_t* bar_p_lo = bar_s_free + 2;         // [2] P~ keys 0..63 of tile t in shared memory
+  uint64_t* bar_p_hi = bar_p_lo + 2;           // [2] P~ keys 64..127 of tile t in shared memory
+  uint64_t* bar_o_lo = bar_p_hi + 2;           // [2] the keys-0..63 half of a P.V with tile t done
+  uint64_t* bar_o_done = bar_o_lo + 2;         // [2] a whole P.V with tile t's queries done
+  uint64_t* bar_vote = bar_o_done + 2;         // [2] softmax t published its rescale factors
+  uint64_t* bar_corr = bar_vote + 2;           // [2] O^T columns of tile t corrected
+  uint64_t* bar_l = bar_corr + 2;              // [2] softmax t published 1 / l
+  uint64_t* bar_drain = bar_l + 2;             // [3] MMA warps' completion at exit
+  uint64_t* bar_epi = bar_drain + 3;           // correction group internal sync
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: head-major, heavy query-tile pairs first
+  const int n_qtiles = N / L::BM;
+  const int n_pairs = (n_qtiles + 1) / 2;
+  const int bh = static_cast<int>(blockIdx.x) / n_pairs;
+  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
+  const int tile0 = 2 * pair;
+  const int n_tiles = min(2, n_qtiles - tile0);
+  const int n_kv_total = N / L::BN;
+  int n_iter[2];
+  n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
+  n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
+  const int n_kv = max(n_iter[0], n_iter[1]);
+  const int row_base = bh * N;
+
+  long long* trace_row = nullptr;
+  if constexpr (TRACE) {
+    if (static_cast<int>(blockIdx.x) < trace_ctas) {
+      trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * n_kv_total);
+      if (threadIdx.x == 0) trace_row[0] = clock64();
+    }
+  }
+  // trace slots as documented at sage_debug_attn_trace; MMA event 0 = the P.V containing
+  // tile t's queries issued, event 1 = Q.K^T of tile t issued (for key tile j + 1)
+  auto stamp = [&](int slot) {
+    if constexpr (TRACE) {
+      if (trace_row) trace_row[2 + slot] = clock64();
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < L::SK; ++s) {
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_k_empty + s, 1);
+    }
+    for (int s = 0; s < L::SV; ++s) {
+      mbar_init(bar_v_full + s, 1);
+      mbar_init(bar_v_empty + s, n_tiles);  // one commit from each P.V warp
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + t, 1);
+      mbar_init(bar_s_free + t, 128);
+      mbar_init(bar_p_lo + t, 128);
+      mbar_init(bar_p_hi + t, 128);
+      mbar_init(bar_o_lo + t, 1);
+      mbar_init(bar_o_done + t, 1);
+      mbar_init(bar_vote + t, 128);
+      mbar_init(bar_corr + t, 128);
+      mbar_init(bar_l + t, 128);
+      mbar_init(bar_drain + t, 1);
+    }
+    mbar_init(bar_drain + 2, 1);
+    mbar_init(bar_epi, 128);
+    for (int i = 0; i < 6; ++i) sFlag[i] = 0;
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S_0 [0,128), S_1 [128,256), O^T [256,512) with column 256 + q for the CTA's
+  // query q (tile 0: q < 128, tile 1: q >= 128); O^T lane = head dimension d.
+  auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+  };
+
+  // Registers: launched with 128 per thread (512 x 128); the control and correction groups hand
+  // part of theirs to the softmax groups: 128 x 88 + 256 x 168 + 128 x 88.  Each setmaxnreg is
+  // executed by a whole warpgroup and dominates that group's code.
+  if (warp < 4) {
+  reg_dealloc<88>();
+  if (warp == 0) {
+    // ============================================================ TMA producer: Q once, K and V
+    if (lane == 0) {
+      int k_issued[L::SK], v_issued[L::SV];
+      for (int s = 0; s < L::SK; ++s) k_issued[s] = 0;
+      for (int s = 0; s < L::SV; ++s) v_issued[s] = 0;
+      mbar_arrive_expect_tx(bar_q, n_tiles * L::Q_BYTES);
+      for (int t = 0; t < n_tiles; ++t)
+        tma_load_2d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, row_base + (tile0 + t) * L::BM);
+      for (int j = 0; j < n_kv; ++j) {
+        const int key_row = row_base + j * L::BN;
+        const int sk_ = j % L::SK, sv_ = j % L::SV;
+        if (j >= L::SK && !mbar_wait(bar_k_empty + sk_, (j / L::SK - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar_k_full + sk_, L::K_BYTES);
+        tma_load_2d(sK + sk_ * L::K_BYTES, &tm_k, bar_k_full + sk_, 0, key_row);
+        k_issued[sk_] = j / L::SK + 1;
+        if (j >= L::SV && !mbar_wait(bar_v_empty + sv_, (j / L::SV - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar_v_full + sv_, L::V_BYTES);
+        tma_load_2d(sV + sv_ * L::V_BYTES, &tm_v, bar_v_full + sv_, 0, key_row);
+        tma_load_2d(sV + sv_ * L::V_BYTES + L::V_BOX, &tm_v, bar_v_full + sv_, 64, key_row);
+        v_issued[sv_] = j / L::SV + 1;
+      }
+      if (*abort_flag) {  // let copies in flight land before the CTA exits
+        mbar_drain(bar_q, 0);
+        for (int s = 0; s < L::SK; ++s)
+          if (k_issued[s] > 0) mbar_drain(bar_k_full + s, (k_issued[s] - 1) & 1);
+        for (int s = 0; s < L::SV; ++s)
+          if (v_issued[s] > 0) mbar_drain(bar_v_full + s, (v_issued[s] - 1) & 1);
+      }
+    }
+  } else if (warp == 1 || warp == 3) {
+    // ============================================================ MMA: O^T_t += V^T . P~_t^T
+    // Warp 1 serves query tile 0, warp 3 tile 1: each product has M = 128 (head dims),
+    // N = 128 (the tile's queries), K = 16 keys, and the two tiles' streams overlap on the
+    // tensor core.  The whole warp runs the loop; elect.sync lets one lane issue.
+    const int t = warp == 1 ? 0 : 1;
+    if (t < n_tiles) {
+      const uint32_t v_base = smem_u32(sV), p_base = smem_u32(sP) + t * 128 * 128;
+      constexpr uint32_t IDESC_PV = make_idesc(1 /*f32*/, 0, 0, 1 /*A = V^T MN-major*/, 0, 128, 128);
+      const uint32_t d_tmem = tmem + 256 + 128 * t;
+      bool ok = true;
+      for (int j = 0; ok && j < n_iter[t]; ++j) {
+        const int s = j % L::SV;
+        if (!wait_warp(bar_v_full + s, (j / L::SV) & 1)) break;
+        // rescaled O^T columns must be in place before this product accumulates into them
+        if (j > 0 && !wait_warp(bar_corr + t, (j - 1) & 1)) break;
+        for (int half = 0; half < 2; ++half) {
+          if (!wait_warp(half == 0 ? bar_p_lo + t : bar_p_hi + t, j & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = half * 4 + k4;  // 16 keys per MMA
+            // A = V^T: keys kk*16.. of the V tile (16 rows of 128 B), LBO = next 64 head dims
+            const uint64_t a = make_smem_desc(v_base + s * L::V_BYTES + kk * 16 * 128, L::V_BOX, 1024, kSwizzle128B);
+            // B = P~_t^T: 64-key atom `half`, 32-byte step k4 inside the 128-byte swizzled rows
+            const uint64_t b = make_smem_desc(p_base + half * L::P_ATOM + k4 * 32, 16, 1024, kSwizzle128B);
+            mma_f16_ss_warp(d_tmem, a, b, IDESC_PV, (j == 0 && kk == 0) ? 0u : 1u);
+          }
+          mma_commit_warp(half == 0 ? bar_o_lo + t : bar_o_done + t);
+        }
+        if (!ok) break;
+        mma_commit_warp(bar_v_empty + s);  // one of the n_tiles arrivals that free stage s
+        if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
+      }
+      mma_commit_warp(bar_drain + t);
+      mbar_drain(bar_drain + t, 0);
+    }
+  } else if (warp == 2) {
+    // ============================================================ MMA: S_t = Q_t . K^T
+    const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
+    constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
+    bool ok = wait_warp(bar_q, 0);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int s = j % L::SK;
+      if (!wait_warp(bar_k_full + s, (j / L::SK) & 1)) break;
+      for (int t = 0; t < n_tiles; ++t) {
+        if (j >= n_iter[t]) continue;
+        if (j > 0 && !wait_warp(bar_s_free + t, (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = make_smem_desc(q_base + t * L::Q_BYTES + kk * 32, 16, 1024, kSwizzle128B);
+          const uint64_t b = make_smem_desc(k_base + s * L::K_BYTES + kk * 32, 16, 1024, kSwizzle128B);
+          mma_i8_ss_warp(tmem + 128 * t, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_warp(bar_s_full + t);
+        if (lane == 0 && j > 0) stamp((7 + 2 * t) * n_kv_total + j - 1);
+      }
+      if (!ok) break;
+      mma_commit_warp(bar_k_empty + s);
+    }
+    mma_commit_warp(bar_drain + 2);
+    mbar_drain(bar_drain + 2, 0);
+  }
+  } else if (warp < 12) {
+    reg_alloc<168>();
+    // ============================================================ softmax warpgroups
+    const int t = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // query row in the tile = TMEM lane of S
+    if (t < n_tiles) {
+      const int q_tile = tile0 + t;
+      const int q_row = q_tile * L::BM + r;
+      const int qi = t * 128 + r;  // the CTA's query index (row of P~, column of O^T)
+      const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+      const uint32_t tS = tmem + lane_addr + 128 * t;
+      const uint32_t p_row = smem_u32(sP) + qi * 128;
+      const float sq_r = PER_TOKEN ? __ldg(sq + row_base + q_row) : __ldg(sq + bh * n_qtiles + q_tile);
+      const float a_r = sq_r * sm_scale_log2;
+      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : N / 64);
+
+      float qm = 0x1p-126f;
+      if constexpr (!PER_TOKEN) {
+        float skmax = 0.f;
+        for (int i = lane; i < N / 64; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) skmax = fmaxf(skmax, __shfl_xor_sync(0xffffffffu, skmax, off));
+        qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
+      }
+
+      float m_use = 0.f;
+      float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+      bool ok = true;
+      for (int j = 0; j < n_iter[t]; ++j) {
+        if (!wait_warp(bar_s_full + t, j & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (r == 0) stamp((3 * t) * n_kv_total + j);
+        const bool diag = CAUSAL && (j == q_tile);
+        const float* skj = sk_head + j * L::BN;  // per-token key scales (global, L1/L2 resident)
+
+        // ---- row maximum of the dequantized scores (log2 units), S read in two halves
+        float mx = -INFINITY;
+        float cb0 = 0.f, cb1 = 0.f;
+        if constexpr (!PER_TOKEN) {
+          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
+          cb1 = trim_scale(a_r * __ldg(sk_head + 2 * j + 1));
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t x[64];
+          tmem_ld64_sync(tS + 64 * h, x);
+          if constexpr (PER_TOKEN) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[64 * h + c]);
+              if (!(diag && 64 * h + c > r)) mx = fmaxf(mx, v);
+            }
+          } else {
+            if (diag) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                if (64 * h + c > r) x[c] = 0x80000000u;
+            }
+            const int im = imax64(x);
+            if (im != INT_MIN) mx = fmaxf(mx, (h ? cb1 : cb0) * static_cast<float>(im));
+          }
+        }
+
+        // ---- offset update; the correction group rescales O^T columns of rows whose offset moved
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_use = round_up_to(mx, qm);
+        } else if (mx > m_use + 8.f) {
+          const float m_new = round_up_to(mx, qm);
+          alpha = fast_exp2(m_use - m_new);
+          m_use = m_new;
+          rescale = true;
+        }
+        if (j > 0) {
+          sAlpha[(j & 1) * 256 + qi] = alpha;
+          int* flag = sFlag + t * 3;
+          if (r == 0) flag[(j + 1) % 3] = 0;  // slot of iteration j+1, last read by iteration j-2's correction
+          if (__any_sync(0xffffffffu, rescale) && lane == 0) atomicOr(flag + j % 3, 1);
+          mbar_arrive(bar_vote + t);
+          if (rescale) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
+          }
+        }
+        const float nb0 = -fmaf(kMagicF, cb0, m_use);  // exact: see offset_quantum
+        const float nb1 = -fmaf(kMagicF, cb1, m_use);
+        if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
+
+        // ---- P~ = exp2(s - m_use) in fp16, 32 keys at a time from TMEM (the next chunk's load in
+        // flight while this one is computed), into shared memory
+        uint32_t xs[2][32];
+        tmem_ld32_async(tS, xs[0]);
+#pragma unroll
+        for (int cb = 0; cb < 128; cb += 32) {
+          uint32_t (&x)[32] = xs[(cb >> 5) & 1];
+          tmem_wait_ld_into(x);
+          if (cb < 96) {
+            tmem_ld32_async(tS + cb + 32, xs[((cb >> 5) + 1) & 1]);
+          } else {
+            tc_fence_before();
+            mbar_arrive(bar_s_free + t);  // S_t fully read: the next Q.K^T may overwrite it
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int c = cb + i;
+            float2 tt;
+            if constexpr (PER_TOKEN) {
+              tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[c], -m_use);
+              tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[c + 1], -m_use);
+            } else {
+              const float cs = c < 64 ? cb0 : cb1;
+              const float nb = c < 64 ? nb0 : nb1;
+              // kMagic + S as float (exact), then one rounding: fl(S * c' - m_use)
+              tt = __ffma2_rn(make_float2(__uint_as_float(x[i] + kMagicBits), __uint_as_float(x[i + 1] + kMagicBits)),
+                              make_float2(cs, cs), make_float2(nb, nb));
+            }
+            // one pair in four on the FMA pipe (exp2_poly2), the rest on the MUFU unit
+            float2 p = ((i >> 1) & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
+            if (diag) {
+              if (c > r) p.x = 0.f;
+              if (c + 1 > r) p.y = 0.f;
+            }
+            lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
+            pk[i >> 1] = pack_half2(p.x, p.y);
+          }
+          // the P~ buffer half is reused: the previous P.V must have read it
+          if (j > 0 && (cb == 0 || cb == 64)) {
+            if (!wait_warp(cb == 0 ? bar_o_lo + t : bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
+          }
+          // keys cb..cb+31 = four 16-byte chunks of 8 keys in 64-key atom cb/64
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int chunk = ((cb & 63) >> 3) + g;
+            st_shared_v4(p_row + (cb >> 6) * L::P_ATOM + ((chunk ^ (qi & 7)) << 4), pk[4 * g], pk[4 * g + 1],
+                         pk[4 * g + 2], pk[4 * g + 3]);
+          }
+          if (cb == 32 || cb == 96) {
+            fence_proxy_async_shared();
+            mbar_arrive(cb == 32 ? bar_p_lo + t : bar_p_hi + t);
+          }
+        }
+        if (!ok) break;
+        if (r == 0) stamp((3 * t + 2) * n_kv_total + j);
+      }
+      if (ok) {
+        const float2 l2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+        sL[qi] = 1.f / (l2.x + l2.y);
+        mbar_arrive(bar_l + t);
+      }
+    }
+  } else {
+    reg_dealloc<88>();
+    // ============================================================ correction and epilogue
+    const int quad = warp & 3;
+    const int d = quad * 32 + lane;  // TMEM lane of O^T
+    const uint32_t tOT = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 256;
+    bool ok = true;
+    for (int j = 1; ok && j < n_kv; ++j) {
+      for (int t = 0; t < n_tiles; ++t) {
+        if (j >= n_iter[t]) continue;
+        if (!wait_warp(bar_vote + t, (j - 1) & 1)) { ok = false; break; }
+        if (sFlag[t * 3 + j % 3]) {
+          // O^T holds the products up to key tile j-1: wait for the last of them
+          if (!wait_warp(bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const float* alpha = sAlpha + (j & 1) * 256 + t * 128;
+#pragma unroll
+          for (int cb = 0; cb < 128; cb += 32) {
+            uint32_t ov[32];
+            tmem_ld32_sync(tOT + t * 128 + cb, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha[cb + i]);
+            tmem_st32(tOT + t * 128 + cb, ov);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        mbar_arrive(bar_corr + t);
+      }
+    }
+    // epilogue per tile: O[q][d] = O^T[d][q] / l_q -> fp16, staged in the tile's own P~ rows
+    // (two [128 q][64 d] pieces, d = lane's head dimension), then TMA-stored
+    int epi_phase = 0;
+    for (int t = 0; ok && t < n_tiles; ++t) {
+      if (!wait_warp(bar_o_done + t, (n_iter[t] - 1) & 1) || !wait_warp(bar_l + t, 0)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t stage = smem_u32(sP) + (d >> 6) * L::P_ATOM + t * 128 * 128 + (d & 63) * 2;
+      const float* inv_l = sL + t * 128;
+#pragma unroll
+      for (int cb = 0; cb < 128; cb += 32) {
+        uint32_t ov[32];
+        tmem_ld32_sync(tOT + t * 128 + cb, ov);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          st_shared_u16(stage + (cb + i) * 128, __half_as_ushort(__float2half_rn(__uint_as_float(ov[i]) * inv_l[cb + i])));
+      }
+      fence_proxy_async_shared();
+      mbar_arrive(bar_epi);
+      if (!wait_warp(bar_epi, epi_phase & 1)) { ok = false; break; }
+      ++epi_phase;
+      if (d == 0) {
+        const int y = row_base + (tile0 + t) * L::BM;
+        tma_store_2d(&tm_o, sP + t * 128 * 128, 0, y);
+        tma_store_2d(&tm_o, sP + L::P_ATOM + t * 128 * 128, 64, y);
+        bulk_commit_and_wait_read();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (TRACE) {
+    if (trace_row && threadIdx.x == 0) trace_row[1] = clock64();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}

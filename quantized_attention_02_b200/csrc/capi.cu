@@ -56,6 +56,11 @@ bool make_v_map(CUtensorMap* map, const void* base, long long rows, int D) {
   return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, D, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// O written by TMA stores of [128 rows x 64 columns] fp16 boxes from unswizzled shared memory.
+bool make_o_map(CUtensorMap* map, const void* base, long long rows, int D) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape checks shared by every entry point.
@@ -81,13 +86,15 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
                         cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0) {
   const int BH = B * H;
   const long long rows = static_cast<long long>(BH) * N;
-  CUtensorMap tq, tk, tv;
-  if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d) || !make_v_map(&tv, v, rows, d))
+  CUtensorMap tq, tk, tv, to;
+  if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d) || !make_v_map(&tv, v, rows, d) ||
+      !make_o_map(&to, o, rows, d))
     return SAGE_ERR_CUDA;
   sage::AttnArgs a{};
   a.tm_q = &tq;
   a.tm_k = &tk;
   a.tm_v = &tv;
+  a.tm_o = &to;
   a.sq = sq;
   a.sk = sk;
   a.o = static_cast<__half*>(o);

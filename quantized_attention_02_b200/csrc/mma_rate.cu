@@ -33,17 +33,18 @@ constexpr uint32_t idesc(uint32_t d_fmt, uint32_t a_fmt, uint32_t b_fmt, uint32_
   return (d_fmt << 4) | (a_fmt << 7) | (b_fmt << 10) | (b_mn << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int chains, int iters, long long* cycles,
-                                                          int* status) {
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int chains, int issuers, int iters,
+                                                          long long* cycles, int* status) {
   extern __shared__ uint8_t raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;              // 16 KB
   uint8_t* sB = smem + 16384;      // 32 KB
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 49152);
-  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 49160);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 49152);  // one per issuing warp
+  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 49168);
   for (int i = threadIdx.x; i < 49152 / 16; i += blockDim.x) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bars)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bars + 1)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zero fill visible to the tensor core
@@ -56,34 +57,53 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int c
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *slot;
 
-  if (threadIdx.x == 0) {
+  // Each issuing warp runs the loop with warp-uniform operands (elect.sync picks the lane that
+  // issues) into its own accumulator columns; with two issuers each does half of the MMAs.
+  const int w = threadIdx.x >> 5;
+  if (w < issuers) {
+    uint64_t* bar = bars + w;
+    const int my_iters = iters / issuers;
     const uint32_t a = smem_u32(sA), b = smem_u32(sB);
+    const uint32_t mask = static_cast<uint32_t>(chains - 1);  // chains is 1, 2 or 4
+    uint32_t id = 0;
+    if (mode == 0) id = idesc(2, 1, 1, 0, 128, n);
+    else if (mode == 1) id = idesc(1, 0, 0, 1, 128, n);
+    else id = idesc(1, 0, 0, 0, 128, n);
+    // descriptors for the four K-steps, computed once; the loop body is unrolled by four
+    uint64_t da[4], db[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      da[k] = desc(a + k * 32, 16, 1024, 2);
+      db[k] = mode == 1 ? desc(b + k * 2048, 16384, 1024, 2) : desc(b + k * 32, 16, 1024, 2);
+    }
     const long long t0 = clock64();
-    for (int i = 0; i < iters; ++i) {
-      const int c = i % chains;
-      const uint32_t acc = i >= chains ? 1u : 0u;
-      const uint32_t d = tmem + 256 + c * n;
-      if (mode == 0) {
-        const uint32_t id = idesc(2, 1, 1, 0, 128, n);
-        const uint64_t da = desc(a + (i & 3) * 32, 16, 1024, 2), db = desc(b + (i & 3) * 32, 16, 1024, 2);
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-                     "l"(da), "l"(db), "r"(id), "r"(acc) : "memory");
-      } else if (mode == 1) {
-        const uint32_t id = idesc(1, 0, 0, 1, 128, n);
-        const uint64_t db = desc(b + (i & 7) * 2048, 16384, 1024, 2);
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-                     "r"(tmem + (i & 7) * 8), "l"(db), "r"(id), "r"(acc) : "memory");
-      } else {
-        const uint32_t id = idesc(1, 0, 0, 0, 128, n);
-        const uint64_t da = desc(a + (i & 3) * 32, 16, 1024, 2), db = desc(b + (i & 3) * 32, 16, 1024, 2);
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-                     "l"(da), "l"(db), "r"(id), "r"(acc) : "memory");
+    for (int i = 0; i < my_iters; i += 4) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t c = static_cast<uint32_t>(i + k) & mask;
+        const uint32_t acc = static_cast<uint32_t>(i + k) > mask ? 1u : 0u;
+        const uint32_t d = tmem + 256 + (c + static_cast<uint32_t>(w * chains)) * static_cast<uint32_t>(n);
+        if (mode == 1) {
+          asm volatile("{\n\t.reg .pred p, e;\n\t.reg .b32 ln;\n\telect.sync ln|e, 0xffffffff;\n\t"
+                       "setp.ne.b32 p, %4, 0;\n\t"
+                       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+                       "r"(tmem + k * 8), "l"(db[k]), "r"(id), "r"(acc) : "memory");
+        } else if (mode == 0) {
+          asm volatile("{\n\t.reg .pred p, e;\n\t.reg .b32 ln;\n\telect.sync ln|e, 0xffffffff;\n\t"
+                       "setp.ne.b32 p, %4, 0;\n\t"
+                       "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+                       "l"(da[k]), "l"(db[k]), "r"(id), "r"(acc) : "memory");
+        } else {
+          asm volatile("{\n\t.reg .pred p, e;\n\t.reg .b32 ln;\n\telect.sync ln|e, 0xffffffff;\n\t"
+                       "setp.ne.b32 p, %4, 0;\n\t"
+                       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+                       "l"(da[k]), "l"(db[k]), "r"(id), "r"(acc) : "memory");
+        }
       }
     }
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+    asm volatile("{\n\t.reg .pred e;\n\t.reg .b32 ln;\n\telect.sync ln|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+                     smem_u32(bar))
                  : "memory");
     uint32_t done = 0;
     const long long tw = clock64();
@@ -95,7 +115,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int c
         break;
       }
     }
-    cycles[blockIdx.x] = clock64() - t0;
+    if (threadIdx.x == 0) cycles[blockIdx.x] = clock64() - t0;  // issuer 0 (both run concurrently)
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -108,11 +128,13 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int mode, int n, int c
 }  // namespace probe
 }  // namespace sage
 
-extern "C" int sage_debug_mma_rate(int mode, int n, int chains, int iters, int ctas, long long* cycles, int* status,
-                                   void* stream) {
-  if (mode < 0 || mode > 2 || iters <= 0 || iters > (1 << 24) || ctas <= 0 || !cycles || !status)
+extern "C" int sage_debug_mma_rate(int mode, int n, int chains, int issuers, int iters, int ctas, long long* cycles,
+                                   int* status, void* stream) {
+  if (mode < 0 || mode > 2 || iters <= 0 || iters > (1 << 24) || iters % 4 != 0 || ctas <= 0 || !cycles || !status)
     return SAGE_ERR_INVALID;
-  if ((n != 64 && n != 128 && n != 256) || chains < 1 || chains > 4 || chains * n > 256) return SAGE_ERR_INVALID;
+  if ((n != 64 && n != 128 && n != 256) || (chains != 1 && chains != 2 && chains != 4) || (issuers != 1 && issuers != 2) ||
+      issuers * chains * n > 256 || iters % (4 * issuers) != 0)
+    return SAGE_ERR_INVALID;
   if (mode == 1 && n > 128) return SAGE_ERR_INVALID;  // B box of the P.V shape holds 128 columns
   constexpr int SMEM = 49152 + 64 + 1024;
   static bool configured = false;
@@ -124,7 +146,7 @@ extern "C" int sage_debug_mma_rate(int mode, int n, int chains, int iters, int c
   }
   // 120 KB of shared memory per CTA keeps one CTA (and one 512-column TMEM allocation) per SM
   (void)SMEM;
-  sage::probe::mma_rate_kernel<<<ctas, 128, 120 * 1024, static_cast<cudaStream_t>(stream)>>>(mode, n, chains, iters,
-                                                                                              cycles, status);
+  sage::probe::mma_rate_kernel<<<ctas, 128, 120 * 1024, static_cast<cudaStream_t>(stream)>>>(mode, n, chains, issuers,
+                                                                                              iters, cycles, status);
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
