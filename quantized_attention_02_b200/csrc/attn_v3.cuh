@@ -81,9 +81,9 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
 }
 
 // Warp roles (16 warps):
-//   0   TMA producer: Q tiles once, then K and V tiles through their rings
+//   0   TMA producer: Q tiles once, then V tiles through their ring
 //   1 / 3  MMA warps: O^T_t += V^T . P~_t^T for query tile 0 / 1 (warp 1 also allocates TMEM)
-//   2   MMA warp: S_t = Q_t . K^T for both query tiles
+//   2   MMA warp: S_t = Q_t . K^T for both query tiles; also loads the K ring (TMA)
 //   4-7 / 8-11  softmax of query tile 0 / 1 (thread = query row = TMEM lane of S)
 //   12-15       correction and epilogue (thread = head dimension d = TMEM lane of O^T):
 //               rescales the O^T columns of rows whose offset moved, then normalizes by 1/l,
@@ -209,21 +209,17 @@ __global__ void __launch_bounds__(512, 1)
   if (warp < 4) {
   reg_dealloc<88>();
   if (warp == 0) {
-    // ============================================================ TMA producer: Q once, K and V
+    // ============================================================ TMA producer: Q once, then V
+    // (the Q.K^T warp loads K itself, so that a V stage still in use never holds back a K load)
     if (lane == 0) {
-      int k_issued[L::SK], v_issued[L::SV];
-      for (int s = 0; s < L::SK; ++s) k_issued[s] = 0;
+      int v_issued[L::SV];
       for (int s = 0; s < L::SV; ++s) v_issued[s] = 0;
       mbar_arrive_expect_tx(bar_q, n_tiles * L::Q_BYTES);
       for (int t = 0; t < n_tiles; ++t)
         tma_load_2d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, row_base + (tile0 + t) * L::BM);
       for (int j = 0; j < n_kv; ++j) {
         const int key_row = row_base + j * L::BN;
-        const int sk_ = j % L::SK, sv_ = j % L::SV;
-        if (j >= L::SK && !mbar_wait(bar_k_empty + sk_, (j / L::SK - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar_k_full + sk_, L::K_BYTES);
-        tma_load_2d(sK + sk_ * L::K_BYTES, &tm_k, bar_k_full + sk_, 0, key_row);
-        k_issued[sk_] = j / L::SK + 1;
+        const int sv_ = j % L::SV;
         if (j >= L::SV && !mbar_wait(bar_v_empty + sv_, (j / L::SV - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar_v_full + sv_, L::V_BYTES);
         tma_load_2d(sV + sv_ * L::V_BYTES, &tm_v, bar_v_full + sv_, 0, key_row);
@@ -232,8 +228,6 @@ __global__ void __launch_bounds__(512, 1)
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
         mbar_drain(bar_q, 0);
-        for (int s = 0; s < L::SK; ++s)
-          if (k_issued[s] > 0) mbar_drain(bar_k_full + s, (k_issued[s] - 1) & 1);
         for (int s = 0; s < L::SV; ++s)
           if (v_issued[s] > 0) mbar_drain(bar_v_full + s, (v_issued[s] - 1) & 1);
       }
@@ -276,12 +270,27 @@ __global__ void __launch_bounds__(512, 1)
       mbar_drain(bar_drain + t, 0);
     }
   } else if (warp == 2) {
-    // ============================================================ MMA: S_t = Q_t . K^T
+    // ============================================================ MMA: S_t = Q_t . K^T, and the
+    // K ring's loads: key tile jj goes to stage jj % SK once Q.K^T of the tile before it there
+    // (jj - SK) is complete.
     const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
     constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
+    int k_loaded = 0;  // key tiles 0 .. k_loaded-1 requested
+    auto load_k = [&](int jj) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_k_full + jj % L::SK, L::K_BYTES);
+        tma_load_2d(sK + (jj % L::SK) * L::K_BYTES, &tm_k, bar_k_full + jj % L::SK, 0, row_base + jj * L::BN);
+      }
+      k_loaded = jj + 1;
+    };
+    for (int jj = 0; jj < min(L::SK - 1, n_kv); ++jj) load_k(jj);
     bool ok = wait_warp(bar_q, 0);
     for (int j = 0; ok && j < n_kv; ++j) {
       const int s = j % L::SK;
+      if (j + L::SK - 1 < n_kv) {  // refill the stage key tile j - 1 used
+        if (j > 0 && !wait_warp(bar_k_empty + (j - 1) % L::SK, ((j - 1) / L::SK) & 1)) break;
+        load_k(j + L::SK - 1);
+      }
       if (!wait_warp(bar_k_full + s, (j / L::SK) & 1)) break;
       for (int t = 0; t < n_tiles; ++t) {
         if (j >= n_iter[t]) continue;
@@ -301,6 +310,9 @@ __global__ void __launch_bounds__(512, 1)
     }
     mma_commit_warp(bar_drain + 2);
     mbar_drain(bar_drain + 2, 0);
+    if (*abort_flag && lane == 0) {  // let K copies in flight land before the CTA exits
+      for (int jj = max(0, k_loaded - L::SK); jj < k_loaded; ++jj) mbar_drain(bar_k_full + jj % L::SK, (jj / L::SK) & 1);
+    }
   }
   } else if (warp < 12) {
     reg_alloc<168>();
@@ -378,6 +390,9 @@ __global__ void __launch_bounds__(512, 1)
           rescale = true;
         }
         if (j > 0) {
+          // the correction group has consumed the previous vote (its barrier phase, factors and
+          // flag slot are reused): bounds how far this group runs ahead of it
+          if (j > 1 && !wait_warp(bar_corr + t, (j - 2) & 1)) { ok = false; break; }
           sAlpha[(j & 1) * 256 + qi] = alpha;
           int* flag = sFlag + t * 3;
           if (r == 0) flag[(j + 1) % 3] = 0;  // slot of iteration j+1, last read by iteration j-2's correction
@@ -393,16 +408,20 @@ __global__ void __launch_bounds__(512, 1)
         if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
 
         // ---- P~ = exp2(s - m_use) in fp16, 32 keys at a time from TMEM (the next chunk's load in
-        // flight while this one is computed), into shared memory
+        // flight while this one is computed), into shared memory.  The last chunk is waited for
+        // together with the third, so that S_t is released (and the next Q.K^T can start) one
+        // chunk before the end.
         uint32_t xs[2][32];
         tmem_ld32_async(tS, xs[0]);
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 32) {
           uint32_t (&x)[32] = xs[(cb >> 5) & 1];
-          tmem_wait_ld_into(x);
-          if (cb < 96) {
+          if (cb < 96) tmem_wait_ld_into(x);
+          if (cb < 64) {
             tmem_ld32_async(tS + cb + 32, xs[((cb >> 5) + 1) & 1]);
-          } else {
+          } else if (cb == 64) {
+            tmem_ld32_async(tS + 96, xs[1]);
+            tmem_wait_ld_into(xs[1]);
             tc_fence_before();
             mbar_arrive(bar_s_free + t);  // S_t fully read: the next Q.K^T may overwrite it
           }
