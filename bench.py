@@ -301,7 +301,7 @@ def run_ours(args, w: W.Workload):
                        "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
                        "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default)",
                        "parallelism": f"independent batch per rank x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "sage_attn_kernel", "achieved": round(achieved, 2),
+            "roofline": {"bound": "tensor", "kernel": ("sage_attn_v3_kernel" if w.d == 128 else "sage_attn_kernel"), "achieved": round(achieved, 2),
                          "peak": round(peak, 2), "unit": "TOPS", "frac": round(achieved / peak, 4),
                          "traffic": traffic,
                          "peak_note": (f"mixed INT8+FP16 roofline from the {src} sustained bf16 peak "
