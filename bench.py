@@ -270,17 +270,6 @@ def run_ours(args, w: W.Workload):
     if sa.sage_last_device_error(stream) != 0:
         raise RuntimeError("a kernel wait timed out during timing")
 
-    # ---- tensor-core rate probe (the MMA shapes of the fused kernel), for the roofline notes
-    probe = {}
-    try:
-        for mode, n, chains in ((0, 128, 1), (0, 128, 2), (0, 256, 1), (0, 64, 4), (1, 128, 1), (1, 128, 2),
-                                (1, 64, 4), (2, 128, 1), (2, 128, 2), (2, 256, 1)):
-            r = sa.mma_rate(mode, n, chains)
-            probe[f"{r['kind']} N{n} x{chains}"] = {"macs_per_clk_per_sm": round(r["macs_per_clk_per_sm"], 1),
-                                                    "tops": round(r["tops"], 1)}
-    except Exception as exc:  # the probe is informational only
-        probe = {"error": str(exc)}
-
     result = None
     if rank == 0:
         peaks, src = load_peaks()
@@ -314,7 +303,6 @@ def run_ours(args, w: W.Workload):
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
-            "mma_probe": probe,
             "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
         }

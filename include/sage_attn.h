@@ -113,7 +113,9 @@ int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, c
                           float sm_scale, int granularity, long long* trace, int trace_ctas,
                           void* stream);
 
-/* Debug: tensor-core throughput probe for the MMA shapes of the fused kernel.  Launches
+/* Debug: tensor-core issue probe for the MMA shapes of the fused kernel (the loop computes the
+ * destination and accumulate flag per instruction; its rate is a lower bound on the tensor rate,
+ * not the peak).  Launches
  * `ctas` CTAs (use the SM count; one per SM); in each, `issuers` warps (1 or 2) issue back-to-back
  * MMAs, iters/issuers each (iters a multiple of 4*issuers, <= 2^24), each warp rotating over its
  * own `chains` accumulators, on zero-filled operands; issuer 0 writes the CTA's SM-clock cycles

@@ -1,5 +1,10 @@
-// mma_rate.cu -- tensor-core throughput probe for the two MMA shapes the fused attention
-// kernel issues, used to measure the INT8 and FP16 peaks its roofline is quoted against.
+// mma_rate.cu -- tensor-core issue probe for the MMA shapes the fused attention kernel uses.
+//
+// What it measures is the rate of this loop: one warp issuing one MMA per iteration with the
+// destination column and the accumulate flag computed per instruction.  That loop reaches about
+// one instruction per 110-140 SM cycles whatever N is, which is below the tensor core's rate for
+// N <= 128 (straight-line issue of the same shapes runs at the datasheet per-SM rate), so its
+// results are a lower bound on the tensor rate, not the peak.
 //
 // One CTA per SM; one thread issues `iters` back-to-back tcgen05 MMAs of one kind, rotating
 // over `chains` independent TMEM accumulators (operands in shared memory, zero-filled), then
