@@ -18,8 +18,8 @@
 //     warps 8-11  softmax for query tile 1
 //   TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D); P~_t (fp16,
 //   64 columns) overwrites the first half of S_t once S_t has been read.
-//   The MMA issue order per key tile j is  PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that while
-//   one softmax warpgroup works the tensor core serves the other tile (ping-pong).
+//   The MMA issue order per key tile j is  PV0(j), QK0(j+1), PV1(j), QK1(j+1): the tensor core
+//   alternates between the two tiles' work.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -45,7 +45,7 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_SK = OFF_V + STAGES * V_BYTES;           // per-token key scales
   static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 6 * NQT;
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 5 * NQT;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int USED = OFF_MISC + 16;
   // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
@@ -152,8 +152,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_p_full = bar_s_full + 2;  // P~ of keys 64..127 (the whole tile) written
   uint64_t* bar_o_done = bar_s_full + 4;
   uint64_t* bar_drain = bar_s_full + 6;   // one per MMA warp
-  uint64_t* bar_seq = bar_s_full + 8;     // softmax group t finished the exp2 phase of a key tile
-  uint64_t* bar_p_lo = bar_s_full + 10;   // P~ of keys 0..63 written
+  uint64_t* bar_p_lo = bar_s_full + 8;    // P~ of keys 0..63 written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -204,8 +203,6 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar_drain, 1);
     mbar_init(bar_drain + 1, 1);
-    mbar_init(bar_seq, 128);
-    mbar_init(bar_seq + 1, 128);
     mbar_init(bar_p_lo, 128);
     mbar_init(bar_p_lo + 1, 128);
     *abort_flag = 0;
@@ -438,15 +435,6 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
 
-        // ---- the two softmax groups take turns on the exp2 unit: group 0 runs key tile j
-        // after group 1 finished tile j-1, group 1 after group 0 finished tile j
-        if (n_tiles > 1) {
-          bool go = true;
-          if (t == 0 && j > 0) go = mbar_wait(bar_seq + 1, (j - 1) & 1, abort_flag);
-          if (t == 1 && j < n_iter[0]) go = mbar_wait(bar_seq, j & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, go)) { ok = false; break; }
-        }
-
         // ---- P~ = exp2(s - m_use) in fp16; the row sum takes the unrounded values
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 32) {
@@ -480,7 +468,6 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive(bar_p_lo + t);
           }
         }
-        if (n_tiles > 1) mbar_arrive(bar_seq + t);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p_full + t);
