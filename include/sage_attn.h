@@ -21,8 +21,10 @@
  *     layout.  km is fp32 [B][H][d].  Scales are fp32 [B][H][G] with
  *     G = sage_scale_count(N, granularity, is_q).
  *   - granularity SAGE_PER_TOKEN: one scale per token (G = N);
- *     SAGE_PER_BLOCK: one scale per 128 consecutive Q tokens / 64 consecutive K tokens.
- *   - d must be 64 or 128; N must be a positive multiple of 128; B, H >= 1;
+ *     SAGE_PER_BLOCK: one scale per 128 consecutive Q tokens / 64 consecutive K tokens
+ *     (groups start at token 0 of each (b,h); the last group holds the remaining tokens).
+ *   - d must be 64 or 128; N >= 1 (any value; sage_debug_qk_int32 alone needs a multiple of
+ *     128); B, H >= 1;
  *     B*H*N*d must stay below 2^31.  sm_scale must be finite and > 0.
  *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls only enqueue work:
  *     they never synchronize the host.  Arguments are validated before anything is
@@ -99,9 +101,10 @@ int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq,
 int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, int H, int N, int d,
                         void* stream);
 
-/* Debug / tracing: sage_attn_fwd_quantized (per-block granularity only) built with SM clock
+/* Debug / tracing: sage_attn_fwd_quantized (per-block granularity and N a multiple of 128
+ * only, else SAGE_ERR_UNSUPPORTED) built with SM clock
  * stamps (clock64) of its pipeline events, for the first trace_ctas CTAs.  Output equals the
- * untraced kernel's.  trace: int64 [trace_ctas][2 + 10*T] with T = N/128 key tiles, zeroed by
+ * untraced kernel's.  trace: int64 [trace_ctas][2 + 10*T] with T = ceil(N/128) key tiles, zeroed by
  * the caller; per CTA: [0] start, [1] end, then for key tile j:
  *   [2 + (3t+e)*T + j]   softmax warpgroup of query tile t (0/1), event e: 0 = S ready,
  *                        1 = row max and offset done, 2 = P~ written and signalled;

@@ -24,6 +24,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "attn_kernels.cuh"
 #include "sm100_ptx.cuh"
@@ -129,7 +130,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 
 // TRACE builds record SM clock stamps of the pipeline events of the first trace_ctas CTAs
 // (layout documented at sage_debug_attn_trace in include/sage_attn.h).
-template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE>
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED>
 __global__ void __launch_bounds__(384, 1)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ sq,
@@ -161,22 +162,22 @@ __global__ void __launch_bounds__(384, 1)
 
   // ---- work unit: consecutive CTAs share a head (its K/V stay in L2); within a head the
   // query-tile pairs with the most key tiles (causal) come first
-  const int n_qtiles = N / L::BM;
+  const int n_qtiles = (N + L::BM - 1) / L::BM;  // the last tile may be partial (rows past N: zeros)
   const int n_pairs = (n_qtiles + 1) / 2;
   const int bh = static_cast<int>(blockIdx.x) / n_pairs;
   const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
   const int tile0 = 2 * pair;
   const int n_tiles = min(2, n_qtiles - tile0);
-  const int n_kv_total = N / L::BN;
+  const int n_kv_total = (N + L::BN - 1) / L::BN;
   int n_iter[2];
   n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
   n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
   const int n_kv = max(n_iter[0], n_iter[1]);
-  const int row_base = bh * N;  // first row of this head in the [BH*N, D] views
+  const int row_base = bh * N;  // first row of this head in the [BH*N, D] arrays
   long long* trace_row = nullptr;
   if constexpr (TRACE) {
     if (static_cast<int>(blockIdx.x) < trace_ctas) {
-      trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * (N / L::BN));
+      trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * n_kv_total);
       if (threadIdx.x == 0) trace_row[0] = clock64();
     }
   }
@@ -232,19 +233,26 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
       mbar_arrive_expect_tx(bar_q, n_tiles * L::Q_BYTES);
       for (int t = 0; t < n_tiles; ++t)
-        tma_load_2d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, row_base + (tile0 + t) * L::BM);
+        tma_load_3d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, (tile0 + t) * L::BM, bh);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % STAGES;
         const int it = j / STAGES;
         if (j >= STAGES && !mbar_wait(bar_kv_empty + s, (it - 1) & 1, abort_flag)) break;
-        const int key_row = row_base + j * L::BN;
-        mbar_arrive_expect_tx(bar_k_full + s, L::K_BYTES + (PER_TOKEN ? L::BN * 4 : 0));
-        tma_load_2d(sK + s * L::K_BYTES, &tm_k, bar_k_full + s, 0, key_row);
-        if constexpr (PER_TOKEN) bulk_load(sSK + s * L::BN, sk + key_row, L::BN * 4, bar_k_full + s);
+        const int key_row = j * L::BN;  // token row within the head
+        // per-token key scales: one bulk copy when the 128 scales exist and start on a 16-byte
+        // boundary, else plain loads (zeros past N) stored before the arrival that publishes them
+        const bool bulk_sk = PER_TOKEN && (N % 4 == 0) && key_row + L::BN <= N;
+        if (PER_TOKEN && !bulk_sk) {
+          for (int c = 0; c < L::BN; ++c)
+            sSK[s * L::BN + c] = key_row + c < N ? __ldg(sk + row_base + key_row + c) : 0.f;
+        }
+        mbar_arrive_expect_tx(bar_k_full + s, L::K_BYTES + (bulk_sk ? L::BN * 4 : 0));
+        tma_load_3d(sK + s * L::K_BYTES, &tm_k, bar_k_full + s, 0, key_row, bh);
+        if (bulk_sk) bulk_load(sSK + s * L::BN, sk + row_base + key_row, L::BN * 4, bar_k_full + s);
         mbar_arrive_expect_tx(bar_v_full + s, L::V_BYTES);
 #pragma unroll
         for (int b = 0; b < D / 64; ++b)
-          tma_load_2d(sV + s * L::V_BYTES + b * L::V_BOX, &tm_v, bar_v_full + s, 64 * b, key_row);
+          tma_load_3d(sV + s * L::V_BYTES + b * L::V_BOX, &tm_v, bar_v_full + s, 64 * b, key_row, bh);
         issued[s] = it + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
@@ -340,9 +348,11 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
       const uint32_t tS = tmem + lane_addr + L::s_col(t);
       const uint32_t tO = tmem + lane_addr + L::o_col(t);
-      const float sq_r = PER_TOKEN ? __ldg(sq + row_base + q_row) : __ldg(sq + bh * n_qtiles + q_tile);
+      // rows past N (a partial last tile) compute on zeros and are never stored
+      const float sq_r = PER_TOKEN ? (q_row < N ? __ldg(sq + row_base + q_row) : 0.f) : __ldg(sq + bh * n_qtiles + q_tile);
       const float a_r = sq_r * sm_scale_log2;  // log2-unit value of one integer step, before sk
-      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : N / 64);
+      const int n_kgroups = (N + 63) / 64;  // per-block key scales per head
+      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : n_kgroups);
 
       // Offset quantum: the exponent offset m_use is kept a multiple of qm, a power of two at
       // least 4 ulps of kMagic * c for every key scale c of this row.  Then kMagic * c' + m_use
@@ -350,9 +360,9 @@ __global__ void __launch_bounds__(384, 1)
       // integer-to-float conversion by the magic-number add costs no extra rounding.
       float qm = 0x1p-126f;
       if constexpr (!PER_TOKEN) {
-        // largest key scale of the head: the warp's lanes split the N/64 scales, then reduce
+        // largest key scale of the head: the warp's lanes split the key scales, then reduce
         float skmax = 0.f;
-        for (int i = lane; i < N / 64; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
+        for (int i = lane; i < n_kgroups; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) skmax = fmaxf(skmax, __shfl_xor_sync(0xffffffffu, skmax, off));
         qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
@@ -369,15 +379,24 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld64_sync(tS + 0, *reinterpret_cast<uint32_t(*)[64]>(x + 0));
         tmem_ld64_sync(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(x + 64));
 
-        const bool diag = CAUSAL && (j == q_tile);
+        // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
+        // c > cmax of this tile are left out of the maximum and get P~ = 0
+        const int kvalid = N - j * L::BN;
+        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
+        const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
         const int s = j % STAGES;
         float mx;            // row maximum of the dequantized scores (log2 units)
         float cb0 = 0.f, cb1 = 0.f, nb0 = 0.f, nb1 = 0.f;
         const float* skj = sSK + s * L::BN;
         if constexpr (PER_TOKEN) {
           // f = kMagic + S exactly (|S| < 2^22), as float bits; masked keys -inf
+          if (diag) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] = (diag && c > r) ? 0xFF800000u : x[c] + kMagicBits;
+            for (int c = 0; c < 128; ++c) x[c] = c > cmax ? 0xFF800000u : x[c] + kMagicBits;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) x[c] += kMagicBits;
+          }
           if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
           mx = -INFINITY;
 #pragma unroll
@@ -386,17 +405,17 @@ __global__ void __launch_bounds__(384, 1)
         } else {
           // integer maxima of the two 64-key halves (one key scale each); masked keys INT_MIN
           cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
-          cb1 = trim_scale(a_r * __ldg(sk_head + 2 * j + 1));
+          cb1 = 2 * j + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * j + 1)) : 0.f;
           if (diag) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
-              if (c > r) x[c] = 0x80000000u;
+              if (c > cmax) x[c] = 0x80000000u;
           }
           const int im0 = imax64(x);
           if (diag) {
 #pragma unroll
             for (int c = 64; c < 128; ++c)
-              if (c > r) x[c] = 0x80000000u;
+              if (c > cmax) x[c] = 0x80000000u;
           }
           const int im1 = imax64(x + 64);
           const float m0 = im0 == INT_MIN ? -INFINITY : cb0 * static_cast<float>(im0);
@@ -435,7 +454,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
 
-        // ---- P~ = exp2(s - m_use) in fp16; the row sum takes the unrounded values
+        // ---- P~ = exp2(s - m_use) in fp16; the row sum takes the unrounded values.  Tiles that
+        // mask keys take exp_pass_masked below instead.
+        auto exp_pass = [&]() {
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 32) {
           uint32_t pk[16];
@@ -453,11 +474,7 @@ __global__ void __launch_bounds__(384, 1)
               tt = __ffma2_rn(make_float2(__uint_as_float(x[c] + kMagicBits), __uint_as_float(x[c + 1] + kMagicBits)),
                               make_float2(cs, cs), make_float2(nb, nb));
             }
-            float2 p = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
-            if (diag) {
-              if (c > r) p.x = 0.f;
-              if (c + 1 > r) p.y = 0.f;
-            }
+            const float2 p = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
             lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
             pk[i >> 1] = pack_half2(p.x, p.y);
           }
@@ -468,6 +485,44 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive(bar_p_lo + t);
           }
         }
+        };
+        // ---- the same for a tile with masked keys (c > cmax: the causal diagonal, a partial last
+        // tile), at most one per row: a rolled loop over 8-key steps that re-reads S from TMEM
+        // 8 columns at a time (P~ of a step lands on columns already read), so that this rare
+        // case adds little code next to the unrolled pass
+        auto exp_pass_masked = [&]() {
+#pragma unroll 1
+          for (int c8 = 0; c8 < 16; ++c8) {
+            uint32_t y[8];
+            tmem_ld8_sync(tS + 8 * c8, y);
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              const int c = 8 * c8 + i;
+              float2 tt;
+              if constexpr (PER_TOKEN) {
+                tt.x = fmaf(static_cast<float>(static_cast<int>(y[i])), a_r * skj[c], -m_use);
+                tt.y = fmaf(static_cast<float>(static_cast<int>(y[i + 1])), a_r * skj[c + 1], -m_use);
+              } else {
+                const float cs = c < 64 ? cb0 : cb1;
+                const float nb = c < 64 ? nb0 : nb1;
+                tt = __ffma2_rn(make_float2(__uint_as_float(y[i] + kMagicBits), __uint_as_float(y[i + 1] + kMagicBits)),
+                                make_float2(cs, cs), make_float2(nb, nb));
+              }
+              const float2 p = make_float2(c > cmax ? 0.f : fast_exp2(tt.x), c + 1 > cmax ? 0.f : fast_exp2(tt.y));
+              lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
+              pk[i >> 1] = pack_half2(p.x, p.y);
+            }
+            tmem_st4(tS + 4 * c8, pk);
+            if (c8 == 7) {  // keys 0..63 done: let their P.V start
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar_p_lo + t);
+            }
+          }
+        };
+        if (diag) exp_pass_masked();
+        else exp_pass();
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p_full + t);
@@ -489,8 +544,10 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 16; ++i)
             hv[i] = pack_half2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+          if (q_row < N) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+          }
         }
       }
     }
@@ -610,17 +667,17 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // ---------------------------------------------------------------- launchers
-template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE = false>
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<D>;
-  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN, TRACE>;
+  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN, TRACE, RAGGED>;
   static bool configured = false;  // attribute set once per instantiation (idempotent)
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int n_qtiles = a.N / L::BM;
+  const int n_qtiles = (a.N + L::BM - 1) / L::BM;
   const int n_pairs = (n_qtiles + 1) / 2;
   dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
   kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sq, a.sk, a.o, a.BH, a.N, a.sm_scale_log2,
@@ -628,40 +685,48 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool CAUSAL, bool PER_TOKEN, bool TRACE = false>
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false>
 static cudaError_t launch_attn_v3(const AttnArgs& a, cudaStream_t st) {
   using L = V3Layout;
-  auto kern = sage_attn_v3_kernel<CAUSAL, PER_TOKEN, TRACE>;
+  auto kern = sage_attn_v3_kernel<CAUSAL, PER_TOKEN, TRACE, RAGGED>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int n_pairs = (a.N / L::BM + 1) / 2;
+  const int n_pairs = ((a.N + L::BM - 1) / L::BM + 1) / 2;
   dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
   kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.sq, a.sk, a.BH, a.N, a.sm_scale_log2,
                                           a.trace, a.trace_ctas);
   return cudaGetLastError();
 }
 
-template <int D>
+// RAGGED instantiations carry the key masking of a partial last key tile; whole-tile problems
+// (N a multiple of 128) use the others, whose non-causal forms have no masking code at all.
+template <int D, bool RAGGED>
 static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
-  if (a.causal) return a.per_token ? launch_attn_t<D, true, true>(a, st) : launch_attn_t<D, true, false>(a, st);
-  return a.per_token ? launch_attn_t<D, false, true>(a, st) : launch_attn_t<D, false, false>(a, st);
+  if (a.causal)
+    return a.per_token ? launch_attn_t<D, true, true, false, RAGGED>(a, st) : launch_attn_t<D, true, false, false, RAGGED>(a, st);
+  return a.per_token ? launch_attn_t<D, false, true, false, RAGGED>(a, st) : launch_attn_t<D, false, false, false, RAGGED>(a, st);
+}
+
+template <bool RAGGED>
+static cudaError_t launch_attn_128(const AttnArgs& a, cudaStream_t st) {
+  if (a.causal)
+    return a.per_token ? launch_attn_v3<true, true, false, RAGGED>(a, st) : launch_attn_v3<true, false, false, RAGGED>(a, st);
+  return a.per_token ? launch_attn_v3<false, true, false, RAGGED>(a, st) : launch_attn_v3<false, false, false, RAGGED>(a, st);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
-  if (a.trace) {  // traced builds exist for per-block granularity only
-    if (a.per_token) return cudaErrorNotSupported;
+  const bool ragged = a.N % 128 != 0;
+  if (a.trace) {  // traced builds exist for per-block granularity and whole tiles only
+    if (a.per_token || ragged) return cudaErrorNotSupported;
     if (a.D == 128) return a.causal ? launch_attn_v3<true, false, true>(a, st) : launch_attn_v3<false, false, true>(a, st);
     return a.causal ? launch_attn_t<64, true, false, true>(a, st) : launch_attn_t<64, false, false, true>(a, st);
   }
-  if (a.D == 128) {
-    if (a.causal) return a.per_token ? launch_attn_v3<true, true>(a, st) : launch_attn_v3<true, false>(a, st);
-    return a.per_token ? launch_attn_v3<false, true>(a, st) : launch_attn_v3<false, false>(a, st);
-  }
-  return launch_attn_d<64>(a, st);
+  if (a.D == 128) return ragged ? launch_attn_128<true>(a, st) : launch_attn_128<false>(a, st);
+  return ragged ? launch_attn_d<64, true>(a, st) : launch_attn_d<64, false>(a, st);
 }
 
 template <int D>

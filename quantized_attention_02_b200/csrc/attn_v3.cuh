@@ -70,12 +70,6 @@ __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit_and_wait_read() {
   asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
 }
@@ -88,7 +82,7 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
 //   12-15       correction and epilogue (thread = head dimension d = TMEM lane of O^T):
 //               rescales the O^T columns of rows whose offset moved, then normalizes by 1/l,
 //               stages O in shared memory and TMA-stores it.
-template <bool CAUSAL, bool PER_TOKEN, bool TRACE>
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED>
 __global__ void __launch_bounds__(512, 1)
     sage_attn_v3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -129,13 +123,13 @@ __global__ void __launch_bounds__(512, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work unit: head-major, heavy query-tile pairs first
-  const int n_qtiles = N / L::BM;
+  const int n_qtiles = (N + L::BM - 1) / L::BM;  // the last tile may be partial (rows past N: zeros)
   const int n_pairs = (n_qtiles + 1) / 2;
   const int bh = static_cast<int>(blockIdx.x) / n_pairs;
   const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) % n_pairs;
   const int tile0 = 2 * pair;
   const int n_tiles = min(2, n_qtiles - tile0);
-  const int n_kv_total = N / L::BN;
+  const int n_kv_total = (N + L::BN - 1) / L::BN;
   int n_iter[2];
   n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
   n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
@@ -216,14 +210,14 @@ __global__ void __launch_bounds__(512, 1)
       for (int s = 0; s < L::SV; ++s) v_issued[s] = 0;
       mbar_arrive_expect_tx(bar_q, n_tiles * L::Q_BYTES);
       for (int t = 0; t < n_tiles; ++t)
-        tma_load_2d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, row_base + (tile0 + t) * L::BM);
+        tma_load_3d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, (tile0 + t) * L::BM, bh);
       for (int j = 0; j < n_kv; ++j) {
-        const int key_row = row_base + j * L::BN;
+        const int key_row = j * L::BN;  // token row within the head
         const int sv_ = j % L::SV;
         if (j >= L::SV && !mbar_wait(bar_v_empty + sv_, (j / L::SV - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar_v_full + sv_, L::V_BYTES);
-        tma_load_2d(sV + sv_ * L::V_BYTES, &tm_v, bar_v_full + sv_, 0, key_row);
-        tma_load_2d(sV + sv_ * L::V_BYTES + L::V_BOX, &tm_v, bar_v_full + sv_, 64, key_row);
+        tma_load_3d(sV + sv_ * L::V_BYTES, &tm_v, bar_v_full + sv_, 0, key_row, bh);
+        tma_load_3d(sV + sv_ * L::V_BYTES + L::V_BOX, &tm_v, bar_v_full + sv_, 64, key_row, bh);
         v_issued[sv_] = j / L::SV + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
@@ -279,7 +273,7 @@ __global__ void __launch_bounds__(512, 1)
     auto load_k = [&](int jj) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar_k_full + jj % L::SK, L::K_BYTES);
-        tma_load_2d(sK + (jj % L::SK) * L::K_BYTES, &tm_k, bar_k_full + jj % L::SK, 0, row_base + jj * L::BN);
+        tma_load_3d(sK + (jj % L::SK) * L::K_BYTES, &tm_k, bar_k_full + jj % L::SK, 0, jj * L::BN, bh);
       }
       k_loaded = jj + 1;
     };
@@ -327,14 +321,16 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
       const uint32_t tS = tmem + lane_addr + 128 * t;
       const uint32_t p_row = smem_u32(sP) + qi * 128;
-      const float sq_r = PER_TOKEN ? __ldg(sq + row_base + q_row) : __ldg(sq + bh * n_qtiles + q_tile);
+      // rows past N (a partial last tile) compute on zeros and are never stored
+      const float sq_r = PER_TOKEN ? (q_row < N ? __ldg(sq + row_base + q_row) : 0.f) : __ldg(sq + bh * n_qtiles + q_tile);
       const float a_r = sq_r * sm_scale_log2;
-      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : N / 64);
+      const int n_kgroups = (N + 63) / 64;  // per-block key scales per head
+      const float* sk_head = sk + static_cast<size_t>(bh) * (PER_TOKEN ? N : n_kgroups);
 
       float qm = 0x1p-126f;
       if constexpr (!PER_TOKEN) {
         float skmax = 0.f;
-        for (int i = lane; i < N / 64; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
+        for (int i = lane; i < n_kgroups; i += 32) skmax = fmaxf(skmax, __ldg(sk_head + i));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) skmax = fmaxf(skmax, __shfl_xor_sync(0xffffffffu, skmax, off));
         qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
@@ -347,7 +343,12 @@ __global__ void __launch_bounds__(512, 1)
         if (!wait_warp(bar_s_full + t, j & 1)) { ok = false; break; }
         tc_fence_after();
         if (r == 0) stamp((3 * t) * n_kv_total + j);
-        const bool diag = CAUSAL && (j == q_tile);
+        // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
+        // c > cmax of this tile are left out of the maximum and get P~ = 0
+        const int kvalid = N - j * L::BN;
+        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
+        const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
+        const int klast = min(kvalid, L::BN) - 1;  // per-token key scales are read up to here
         const float* skj = sk_head + j * L::BN;  // per-token key scales (global, L1/L2 resident)
 
         // ---- row maximum of the dequantized scores (log2 units), S read in two halves
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(512, 1)
         float cb0 = 0.f, cb1 = 0.f;
         if constexpr (!PER_TOKEN) {
           cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
-          cb1 = trim_scale(a_r * __ldg(sk_head + 2 * j + 1));
+          cb1 = 2 * j + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * j + 1)) : 0.f;
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -364,14 +365,14 @@ __global__ void __launch_bounds__(512, 1)
           if constexpr (PER_TOKEN) {
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-              const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[64 * h + c]);
-              if (!(diag && 64 * h + c > r)) mx = fmaxf(mx, v);
+              const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[min(64 * h + c, klast)]);
+              if (!(diag && 64 * h + c > cmax)) mx = fmaxf(mx, v);
             }
           } else {
             if (diag) {
 #pragma unroll
               for (int c = 0; c < 64; ++c)
-                if (64 * h + c > r) x[c] = 0x80000000u;
+                if (64 * h + c > cmax) x[c] = 0x80000000u;
             }
             const int im = imax64(x);
             if (im != INT_MIN) mx = fmaxf(mx, (h ? cb1 : cb0) * static_cast<float>(im));
@@ -410,7 +411,8 @@ __global__ void __launch_bounds__(512, 1)
         // ---- P~ = exp2(s - m_use) in fp16, 32 keys at a time from TMEM (the next chunk's load in
         // flight while this one is computed), into shared memory.  The last chunk is waited for
         // together with the third, so that S_t is released (and the next Q.K^T can start) one
-        // chunk before the end.
+        // chunk before the end.  Tiles that mask keys take exp_pass_masked below instead.
+        auto exp_pass = [&]() -> bool {
         uint32_t xs[2][32];
         tmem_ld32_async(tS, xs[0]);
 #pragma unroll
@@ -431,8 +433,8 @@ __global__ void __launch_bounds__(512, 1)
             const int c = cb + i;
             float2 tt;
             if constexpr (PER_TOKEN) {
-              tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[c], -m_use);
-              tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[c + 1], -m_use);
+              tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[min(c, klast)], -m_use);
+              tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[min(c + 1, klast)], -m_use);
             } else {
               const float cs = c < 64 ? cb0 : cb1;
               const float nb = c < 64 ? nb0 : nb1;
@@ -441,17 +443,13 @@ __global__ void __launch_bounds__(512, 1)
                               make_float2(cs, cs), make_float2(nb, nb));
             }
             // one pair in four on the FMA pipe (exp2_poly2), the rest on the MUFU unit
-            float2 p = ((i >> 1) & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
-            if (diag) {
-              if (c > r) p.x = 0.f;
-              if (c + 1 > r) p.y = 0.f;
-            }
+            const float2 p = ((i >> 1) & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
             lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
             pk[i >> 1] = pack_half2(p.x, p.y);
           }
           // the P~ buffer half is reused: the previous P.V must have read it
           if (j > 0 && (cb == 0 || cb == 64)) {
-            if (!wait_warp(cb == 0 ? bar_o_lo + t : bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
+            if (!wait_warp(cb == 0 ? bar_o_lo + t : bar_o_done + t, (j - 1) & 1)) return false;
           }
           // keys cb..cb+31 = four 16-byte chunks of 8 keys in 64-key atom cb/64
 #pragma unroll
@@ -465,7 +463,51 @@ __global__ void __launch_bounds__(512, 1)
             mbar_arrive(cb == 32 ? bar_p_lo + t : bar_p_hi + t);
           }
         }
-        if (!ok) break;
+        return true;
+        };
+        // ---- the same for a tile with masked keys (c > cmax: the causal diagonal, a partial last
+        // tile), at most one per row: a rolled loop over 8-key steps, S re-read 8 columns at a
+        // time, so that this rare case adds little code next to the unrolled pass
+        auto exp_pass_masked = [&]() -> bool {
+#pragma unroll 1
+          for (int c8 = 0; c8 < 16; ++c8) {
+            uint32_t x[8];
+            tmem_ld8_sync(tS + 8 * c8, x);
+            if (c8 == 15) {
+              tc_fence_before();
+              mbar_arrive(bar_s_free + t);  // S_t fully read
+            }
+            if (j > 0 && (c8 == 0 || c8 == 8)) {
+              if (!wait_warp(c8 == 0 ? bar_o_lo + t : bar_o_done + t, (j - 1) & 1)) return false;
+            }
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              const int c = 8 * c8 + i;
+              float2 tt;
+              if constexpr (PER_TOKEN) {
+                tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[min(c, klast)], -m_use);
+                tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[min(c + 1, klast)], -m_use);
+              } else {
+                const float cs = c < 64 ? cb0 : cb1;
+                const float nb = c < 64 ? nb0 : nb1;
+                tt = __ffma2_rn(make_float2(__uint_as_float(x[i] + kMagicBits), __uint_as_float(x[i + 1] + kMagicBits)),
+                                make_float2(cs, cs), make_float2(nb, nb));
+              }
+              const float2 p = make_float2(c > cmax ? 0.f : fast_exp2(tt.x), c + 1 > cmax ? 0.f : fast_exp2(tt.y));
+              lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
+              pk[i >> 1] = pack_half2(p.x, p.y);
+            }
+            // keys 8*c8 .. 8*c8+7 = 16-byte chunk (c8 mod 8) of 64-key atom c8/8
+            st_shared_v4(p_row + (c8 >> 3) * L::P_ATOM + (((c8 & 7) ^ (qi & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            if (c8 == 7 || c8 == 15) {
+              fence_proxy_async_shared();
+              mbar_arrive(c8 == 7 ? bar_p_lo + t : bar_p_hi + t);
+            }
+          }
+          return true;
+        };
+        if (!(diag ? exp_pass_masked() : exp_pass())) { ok = false; break; }
         if (r == 0) stamp((3 * t + 2) * n_kv_total + j);
       }
       if (ok) {
@@ -525,9 +567,9 @@ __global__ void __launch_bounds__(512, 1)
       if (!wait_warp(bar_epi, epi_phase & 1)) { ok = false; break; }
       ++epi_phase;
       if (d == 0) {
-        const int y = row_base + (tile0 + t) * L::BM;
-        tma_store_2d(&tm_o, sP + t * 128 * 128, 0, y);
-        tma_store_2d(&tm_o, sP + L::P_ATOM + t * 128 * 128, 64, y);
+        const int y = (tile0 + t) * L::BM;  // rows past N are clipped by the tensor map
+        tma_store_3d(&tm_o, sP + t * 128 * 128, 0, y, bh);
+        tma_store_3d(&tm_o, sP + L::P_ATOM + t * 128 * 128, 64, y, bh);
         bulk_commit_and_wait_read();
       }
     }

@@ -47,18 +47,39 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_qk_map(CUtensorMap* map, const int8_t* base, long long rows, int D) {
-  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, D, D,
-                  D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+// [BH, N, D] as a 3-D tensor (D innermost, then the N tokens of a head, then heads), box
+// [box_cols x 128 tokens x 1 head]: a box never reaches into the next head; token rows past N
+// read as zeros and are not written by stores.
+bool make_map3(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes, int N, int BH, int D,
+               int box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem_bytes,
+                                 static_cast<cuuint64_t>(N) * D * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_v_map(CUtensorMap* map, const void* base, long long rows, int D) {
-  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, D, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+bool make_qk_map3(CUtensorMap* map, const int8_t* base, int N, int BH, int D) {
+  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, BH, D, D,
+                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+bool make_v_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
+  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // O written by TMA stores of [128 rows x 64 columns] fp16 boxes from unswizzled shared memory.
-bool make_o_map(CUtensorMap* map, const void* base, long long rows, int D) {
-  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+bool make_o_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
+  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+bool make_qk_map(CUtensorMap* map, const int8_t* base, long long rows, int D) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, D, D,
+                  D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -67,7 +88,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_shape(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SAGE_ERR_INVALID;
   if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return SAGE_ERR_UNSUPPORTED;
   const long long elems = static_cast<long long>(B) * H * N * d;
   if (elems >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
@@ -85,10 +105,9 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
                         int B, int H, int N, int d, int causal, float sm_scale, int granularity,
                         cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0) {
   const int BH = B * H;
-  const long long rows = static_cast<long long>(BH) * N;
   CUtensorMap tq, tk, tv, to;
-  if (!make_qk_map(&tq, q8, rows, d) || !make_qk_map(&tk, k8, rows, d) || !make_v_map(&tv, v, rows, d) ||
-      !make_o_map(&to, o, rows, d))
+  if (!make_qk_map3(&tq, q8, N, BH, d) || !make_qk_map3(&tk, k8, N, BH, d) || !make_v_map3(&tv, v, N, BH, d) ||
+      !make_o_map3(&to, o, N, BH, d))
     return SAGE_ERR_CUDA;
   sage::AttnArgs a{};
   a.tm_q = &tq;
@@ -118,7 +137,7 @@ const char* sage_status_string(int status) {
   switch (status) {
     case SAGE_OK: return "ok";
     case SAGE_ERR_INVALID: return "invalid argument";
-    case SAGE_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128, N a multiple of 128)";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128; the INT32 debug entry also needs N a multiple of 128)";
     case SAGE_ERR_CUDA: return "CUDA runtime error";
     case SAGE_ERR_TIMEOUT: return "a kernel wait timed out";
     case SAGE_ERR_NOMEM: return "workspace allocation failed";
@@ -215,6 +234,7 @@ int sage_debug_qk_int32(const int8_t* q8, const int8_t* k8, int32_t* s, int B, i
   if (!q8 || !k8 || !s) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
+  if (N % 128 != 0) return SAGE_ERR_UNSUPPORTED;  // whole 128 x 128 tiles only
   if (static_cast<long long>(B) * H * N * N >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(s)) return SAGE_ERR_INVALID;
   const long long rows = static_cast<long long>(B) * H * N;

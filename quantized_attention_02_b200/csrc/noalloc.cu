@@ -69,7 +69,6 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   if (granularity != SAGE_PER_TOKEN && granularity != SAGE_PER_BLOCK) return SAGE_ERR_INVALID;
   if (!(sm_scale > 0.f) || sm_scale > 3.4e38f) return SAGE_ERR_INVALID;  // also rejects NaN and inf
   if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return SAGE_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N * d >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
   for (const void* p : {q, k, static_cast<const void*>(v), static_cast<const void*>(o)})
     if (reinterpret_cast<uintptr_t>(p) & 15u) return SAGE_ERR_INVALID;

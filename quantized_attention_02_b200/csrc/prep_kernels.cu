@@ -109,11 +109,15 @@ __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
 
 // Quantize groups of G tokens (G = 1: per token).  T = D/8 threads cover one token row with
 // one 16-byte vector each; a 256-thread CTA covers P = 256/T tokens per pass.
-//   G == 1 : each T-lane team is its own group (team-wide shuffle max);
+//   G == 1 : each T-lane team is its own group (team-wide shuffle max); teams past the last
+//            row compute on zeros and store nothing;
 //   G  > 1 : the CTA is one group of G tokens held in registers (G/P passes), CTA-wide max.
+//            Groups tile each head separately: ceil(N/G) groups per head, the last one holding
+//            the N mod G remaining tokens when G does not divide N.
 template <int D, int G, bool SMOOTH>
 __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x, const float* __restrict__ km,
-                                                    int8_t* __restrict__ q, float* __restrict__ scale, int N) {
+                                                    int8_t* __restrict__ q, float* __restrict__ scale, int N,
+                                                    long long rows) {
   constexpr int T = D / 8;
   constexpr int P = 256 / T;
   const int piece = threadIdx.x % T;
@@ -121,11 +125,12 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
 
   if constexpr (G == 1) {
     const size_t row = static_cast<size_t>(blockIdx.x) * P + threadIdx.x / T;
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + row * D + c0));
+    const bool live = row < static_cast<size_t>(rows);  // whole T-lane teams; all lanes stay for the shuffles
+    const uint4 w = live ? __ldg(reinterpret_cast<const uint4*>(x + row * D + c0)) : make_uint4(0, 0, 0, 0);
     float v[8];
     unpack8(w, v);
     if constexpr (SMOOTH) {
-      const float* mu = km + (row / N) * D + c0;
+      const float* mu = km + (live ? row / N : 0) * D + c0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = __fsub_rn(v[i], __ldg(mu + i));
     }
@@ -139,16 +144,21 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
       s = __fdiv_rn(a, 127.0f);
       inv = __fdiv_rn(127.0f, a);
     }
-    *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v, inv);
-    if (piece == 0) scale[row] = s;
+    if (live) {
+      *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v, inv);
+      if (piece == 0) scale[row] = s;
+    }
   } else {
     static_assert(G % P == 0, "group must be a whole number of passes");
     constexpr int PASSES = G / P;
-    const size_t row0 = static_cast<size_t>(blockIdx.x) * G;  // groups tile the rows of each head
+    const int n_groups = (N + G - 1) / G;
+    const int bh = static_cast<int>(blockIdx.x) / n_groups;
+    const int tok0 = (static_cast<int>(blockIdx.x) % n_groups) * G;  // first token of the group in its head
+    const size_t row0 = static_cast<size_t>(bh) * N + tok0;
     const int tok = threadIdx.x / T;
     float mu[8];
     if constexpr (SMOOTH) {
-      const float* m = km + (row0 / N) * D + c0;
+      const float* m = km + static_cast<size_t>(bh) * D + c0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) mu[i] = __ldg(m + i);
     }
@@ -157,12 +167,13 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
       const size_t row = row0 + p * P + tok;
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(x + row * D + c0));
+      const bool live = tok0 + p * P + tok < N;
+      const uint4 w = live ? __ldg(reinterpret_cast<const uint4*>(x + row * D + c0)) : make_uint4(0, 0, 0, 0);
       unpack8(w, v[p]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if constexpr (SMOOTH) v[p][i] = __fsub_rn(v[p][i], mu[i]);
-        a = fmaxf(a, fabsf(v[p][i]));
+        if (live) a = fmaxf(a, fabsf(v[p][i]));
       }
     }
 #pragma unroll
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
       const size_t row = row0 + p * P + tok;
-      *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v[p], inv);
+      if (tok0 + p * P + tok < N) *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v[p], inv);
     }
     if (threadIdx.x == 0) scale[blockIdx.x] = s;
   }
@@ -204,8 +215,8 @@ static cudaError_t launch_quant_g(const __half* x, const float* km, int8_t* q, f
                                   cudaStream_t st) {
   constexpr int T = D / 8, P = 256 / T;
   const long long rows = static_cast<long long>(BH) * N;
-  const long long blocks = (G == 1) ? rows / P : rows / G;
-  quant_kernel<D, G, SMOOTH><<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, km, q, s, N);
+  const long long blocks = (G == 1) ? (rows + P - 1) / P : static_cast<long long>(BH) * ((N + G - 1) / G);
+  quant_kernel<D, G, SMOOTH><<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, km, q, s, N, rows);
   return cudaGetLastError();
 }
 
