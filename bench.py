@@ -288,7 +288,7 @@ def run_ours(args, w: W.Workload):
             "scaling": "weak", "vs_baseline": None, "dtype": "int8+f16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
-                       "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default)",
+                       "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default); no flush needed",
                        "parallelism": f"independent batch per rank x{world}"},
             "roofline": {"bound": "tensor", "kernel": ("sage_attn_v3_kernel" if w.d == 128 else "sage_attn_kernel"), "achieved": round(achieved, 2),
                          "peak": round(peak, 2), "unit": "TOPS", "frac": round(achieved / peak, 4),

@@ -10,6 +10,7 @@
 // intrinsics (never contracted into an FMA), in the order the C ABI documents.
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "prep_kernels.cuh"
 
@@ -126,7 +127,9 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
   if constexpr (G == 1) {
     const size_t row = static_cast<size_t>(blockIdx.x) * P + threadIdx.x / T;
     const bool live = row < static_cast<size_t>(rows);  // whole T-lane teams; all lanes stay for the shuffles
-    const uint4 w = live ? __ldg(reinterpret_cast<const uint4*>(x + row * D + c0)) : make_uint4(0, 0, 0, 0);
+    // the load always reads an existing row (the last one for teams past the end), then is zeroed
+    uint4 w = __ldg(reinterpret_cast<const uint4*>(x + (live ? row : static_cast<size_t>(rows) - 1) * D + c0));
+    if (!live) w = make_uint4(0u, 0u, 0u, 0u);
     float v[8];
     unpack8(w, v);
     if constexpr (SMOOTH) {
@@ -164,11 +167,18 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
     }
     float v[PASSES][8];
     float a = 0.f;
+    // a whole group (every group but a partial last one of its head) compiles without the
+    // per-token guards, so that its PASSES loads are all in flight together
+    const bool whole = tok0 + G <= N;
+    auto load_pass = [&](auto whole_tag) {
+    constexpr bool WHOLE = decltype(whole_tag)::value;
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
-      const size_t row = row0 + p * P + tok;
-      const bool live = tok0 + p * P + tok < N;
-      const uint4 w = live ? __ldg(reinterpret_cast<const uint4*>(x + row * D + c0)) : make_uint4(0, 0, 0, 0);
+      const bool live = WHOLE || tok0 + p * P + tok < N;
+      // every pass loads (the group's first token for rows past N, then zeroed): no branch
+      // between the loads, so all PASSES of them are in flight together
+      uint4 w = __ldg(reinterpret_cast<const uint4*>(x + (row0 + (live ? p * P + tok : 0)) * D + c0));
+      if (!live) w = make_uint4(0, 0, 0, 0);
       unpack8(w, v[p]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -176,6 +186,9 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
         if (live) a = fmaxf(a, fabsf(v[p][i]));
       }
     }
+    };
+    if (whole) load_pass(std::true_type{});
+    else load_pass(std::false_type{});
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
     __shared__ float wmax[8];
@@ -192,7 +205,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
       const size_t row = row0 + p * P + tok;
-      if (tok0 + p * P + tok < N) *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v[p], inv);
+      if (whole || tok0 + p * P + tok < N) *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v[p], inv);
     }
     if (threadIdx.x == 0) scale[blockIdx.x] = s;
   }
