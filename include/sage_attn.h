@@ -164,6 +164,29 @@ size_t sage_noalloc_scratch_bytes(int B, int H, int N, int d, int granularity);
 int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                           int causal, float sm_scale, int granularity, void* stream);
 
+/* The whole forward pass with Q, K, V and O in HOST memory: the host->device copies of the
+ * inputs and the device->host copy of O overlap the compute.  (Not an operation of the
+ * pages: a serving convenience built from the three steps above.)
+ *
+ * The B*H heads are processed in chunks of heads_per_chunk consecutive heads (0 = automatic,
+ * about sixteen chunks).  For chunk c, its slice of Q, K, V is copied in on an internal
+ * stream, the three steps run on `stream`, and its slice of O is copied out on a second
+ * internal stream, while chunk c+1 is copied in and chunk c-1 copied out; events order every
+ * reuse of the two sets of device buffers.  The output is bit-identical to sage_attn_fwd on
+ * the same tensors (every head is an independent problem and runs the same kernels).
+ *
+ * q, k, v: fp16 [B][H][N][d] host memory, read; o: fp16 [B][H][N][d] host memory, written.
+ * Any host allocation works; page-locked memory (cudaMallocHost / cudaHostRegister) is
+ * needed for the copies to overlap.  The caller keeps all four buffers alive and unchanged
+ * (o unread) until `stream` has passed the call: like every entry point here, the call only
+ * enqueues work (with pageable memory the runtime may block the host during a copy).  The
+ * device workspace (2 x chunk slices of Q, K, V, O plus INT8 copies and scales) is
+ * allocated and freed stream-ordered on `stream`.  Same size, scale and granularity rules
+ * and statuses as sage_attn_fwd; heads_per_chunk < 0 gives SAGE_ERR_INVALID; a failed
+ * workspace allocation SAGE_ERR_NOMEM. */
+int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                       int causal, float sm_scale, int granularity, int heads_per_chunk, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -59,9 +59,10 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_noalloc_scratch_bytes.restype = _sz
         lib.sage_debug_attn_trace.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _i, _p]
         lib.sage_debug_mma_rate.argtypes = [_i, _i, _i, _i, _i, _i, _p, _p, _p]
+        lib.sage_attn_fwd_host.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p]
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
-                  "sage_debug_attn_trace", "sage_debug_mma_rate"):
+                  "sage_debug_attn_trace", "sage_debug_mma_rate", "sage_attn_fwd_host"):
             getattr(lib, n).restype = _i
         _lib = lib
     return _lib
@@ -194,6 +195,33 @@ def sage_attn_fwd_noalloc(q, k, v, o, causal: bool, sm_scale: float, granularity
     _check(get_lib().sage_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
                                      float(sm_scale), int(granularity), _stream(stream)),
            "sage_attn_fwd_noalloc")
+
+
+def _host_ptr(t):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if t.is_cuda:
+        raise ValueError("sage_attn_fwd_host takes host tensors (pinned memory lets the copies overlap)")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if t.dtype != torch.float16:
+        raise ValueError("expected float16")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def sage_attn_fwd_host(q, k, v, o, causal: bool, sm_scale: float, granularity: int, heads_per_chunk: int = 0,
+                       stream=None) -> None:
+    """Whole forward pass on HOST tensors [B, H, N, d] (fp16): copies in, compute and copies
+    out overlap across chunks of heads.  Asynchronous on `stream` (the current CUDA stream by
+    default): synchronize it before reading o or changing q, k, v."""
+    B, H, N, d = _shape(q)
+    for t in (k, v, o):
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v, o must have the same shape")
+    _check(get_lib().sage_attn_fwd_host(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(o), B, H, N, d,
+                                        int(bool(causal)), float(sm_scale), int(granularity), int(heads_per_chunk),
+                                        _stream(stream)),
+           "sage_attn_fwd_host")
 
 
 def sage_noalloc_scratch_bytes(B: int, H: int, N: int, d: int, granularity: int) -> int:

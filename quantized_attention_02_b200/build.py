@@ -29,6 +29,7 @@ SOURCES = {
     "prep_kernels.cu": ["--fmad=false"],
     "attn_kernels.cu": [],
     "noalloc.cu": [],
+    "host_pipeline.cu": [],
     "mma_rate.cu": [],
 }
 HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh"]

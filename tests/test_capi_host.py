@@ -93,6 +93,20 @@ def test_null_pointers_and_bad_scalars(sa):
     assert L.sage_debug_qk_int32(FAKE, FAKE, None, 1, 1, 128, 64, s) == -1
 
 
+def test_host_pipeline_validation(sa):
+    # every failure below is found before any CUDA call (no GPU is needed)
+    L = sa.get_lib()
+    s = ctypes.c_void_p(0)
+    ok_args = (1, 2, 256, 64, 0, 0.1, 1)
+    assert L.sage_attn_fwd_host(None, FAKE, FAKE, FAKE, *ok_args, 0, s) == -1
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, None, *ok_args, 0, s) == -1
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, *ok_args, -1, s) == -1       # heads_per_chunk < 0
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 96, 0, 0.1, 1, 0, s) == -2  # d
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 0, 64, 0, 0.1, 1, 0, s) == -1    # N
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 64, 0, float("nan"), 1, 0, s) == -1
+    assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 64, 0, 0.1, 5, 0, s) == -1  # granularity
+
+
 def test_binding_rejects_cpu_tensors(sa):
     import torch
     q = torch.zeros(1, 1, 128, 64, dtype=torch.float16)
