@@ -152,6 +152,24 @@ def oracle_sample(w: W.Workload, budget_s: float = 12.0):
     return ops / t / 1e12, cores, desc
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value: the job is done when every rank is.  Every rank must call
+    this (it is a collective when world > 1)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(world: int, ops_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: every rank's work over the slowest rank's time (weak scaling:
+    each rank runs its own independent batch)."""
+    return world * ops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, w: W.Workload):
     import torch.distributed as dist
@@ -202,11 +220,7 @@ def run_ours(args, w: W.Workload):
         torch.cuda.synchronize(dev)
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # ---- the fused kernel alone (already-quantized inputs), same stream, for the roofline
     sa.sage_smooth_k(k, km, stream)
@@ -260,11 +274,7 @@ def run_ours(args, w: W.Workload):
         e2e_step()
     x1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = x0.elapsed_time(x1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / e2e_steps, world, dev)
     if sa.sage_last_device_error(stream) != 0:
         raise RuntimeError("a kernel wait timed out during timing")
 
@@ -272,7 +282,7 @@ def run_ours(args, w: W.Workload):
     if rank == 0:
         peaks, src = load_peaks()
         ops = w.ops()
-        value = world * ops / (ms_max * 1e-3) / 1e12
+        value = job_tops(world, ops, ms_max)
         p_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
         p_burst = float(peaks["bf16_tflops"])
         peak = mixed_peak_tops(p_sus)
@@ -297,7 +307,7 @@ def run_ours(args, w: W.Workload):
                                        f"(frac {achieved / mixed_peak_tops(p_burst):.4f})"),
                          "kernel_ms": round(kernel_ms, 4)},
             "cpu_baseline": {"value": cpu_tops, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
-            "e2e": {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "e2e": {"value": round(job_tops(world, ops, e2e_ms), 2), "unit": UNIT,
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
