@@ -72,6 +72,16 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = None
         self._nvml = None
+        # samples count only inside the timed window (open_window .. close_window): the sampler
+        # starts before the warm-up so that its set-up never overlaps the timed steps
+        self.window = [float("inf")]
+        self.window_closed = False
+
+    def open_window(self):
+        self.window[0] = time.perf_counter()
+
+    def close_window(self):
+        self.window_closed = True
 
     def _run(self):
         nv = self._nvml
@@ -82,12 +92,15 @@ class ClockSampler:
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((sm, mx, pw, bits))
+                if self.window[0] <= time.perf_counter() and not self.window_closed:
+                    self.samples.append((sm, mx, pw, bits))
             except Exception:
                 pass
             self._stop.wait(0.05)
 
     def __enter__(self):
+        if self._t is not None:  # already sampling
+            return self
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -201,6 +214,8 @@ def run_ours(args, w: W.Workload):
     def step():
         sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
 
+    clocks = ClockSampler(dev.index if world == 1 else local)
+    clocks.__enter__()  # sampling thread up before the warm-up; samples count from the timed window only
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -208,16 +223,17 @@ def run_ours(args, w: W.Workload):
         raise RuntimeError("a kernel wait timed out during warm-up")
 
     # ---- headline: K whole steps, inputs resident (each input 2*B*H*N*d bytes > L2)
-    clocks = ClockSampler(dev.index if world == 1 else local)
-    barrier()
-    torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with clocks:
+        barrier()
+        torch.cuda.synchronize(dev)
+        clocks.open_window()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.close_window()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)

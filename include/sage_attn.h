@@ -82,7 +82,9 @@ int sage_quant_qk(const void* q, const void* k, const float* km, int8_t* q8, int
 /* The whole forward pass as a user calls it: smooth K, quantize Q and K, fused attention.
  * q, k, v: fp16 [B,H,N,d] (in); o: fp16 [B,H,N,d] (out).  causal: keys j > i masked
  * (top-left aligned).  Workspace (int8 Q/K, scales, km: 2*B*H*N*d bytes plus scales) is
- * allocated and freed stream-ordered (cudaMallocAsync / cudaFreeAsync) inside the call. */
+ * allocated and freed stream-ordered inside the call, from a memory pool the library owns
+ * (one per device) that keeps freed memory reserved for the next call: the largest workspace
+ * used so far stays reserved until the process exits. */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                   int causal, float sm_scale, int granularity, void* stream);
 

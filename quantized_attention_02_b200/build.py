@@ -32,7 +32,7 @@ SOURCES = {
     "host_pipeline.cu": [],
     "mma_rate.cu": [],
 }
-HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh"]
+HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh", "workspace.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -12,6 +12,7 @@
 #include "attn_kernels.cuh"
 #include "prep_kernels.cuh"
 #include "sage_attn.h"
+#include "workspace.cuh"
 
 namespace {
 
@@ -131,6 +132,41 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
 
 }  // namespace
 
+namespace sage {
+
+cudaError_t workspace_alloc(void** p, size_t bytes, cudaStream_t st) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+      cudaMemPoolProps props{};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t created = nullptr;
+      if ((e = cudaMemPoolCreate(&created, &props)) != cudaSuccess) return e;
+      unsigned long long keep = ~0ull;  // never hand freed memory back at synchronizations
+      if ((e = cudaMemPoolSetAttribute(created, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) {
+        cudaMemPoolDestroy(created);
+        return e;
+      }
+      pools[dev] = created;
+    }
+    pool = pools[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, st);
+}
+
+}  // namespace sage
+
 extern "C" {
 
 const char* sage_status_string(int status) {
@@ -212,7 +248,7 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   const size_t off_km = off_sk + up(nsk * 4);
   const size_t total = off_km + up(static_cast<size_t>(BH) * d * 4);
   void* ws = nullptr;
-  if (cudaMallocAsync(&ws, total, st) != cudaSuccess) {
+  if (sage::workspace_alloc(&ws, total, st) != cudaSuccess) {
     cudaGetLastError();
     return SAGE_ERR_NOMEM;
   }

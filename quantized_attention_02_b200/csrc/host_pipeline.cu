@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "sage_attn.h"
+#include "workspace.cuh"
 
 namespace {
 
@@ -106,7 +107,7 @@ int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int
 
   const size_t per_slot = slot_bytes(hc, N, d, granularity);
   void* ws = nullptr;
-  if (cudaMallocAsync(&ws, per_slot * n_slots, st) != cudaSuccess) {
+  if (sage::workspace_alloc(&ws, per_slot * n_slots, st) != cudaSuccess) {
     cudaGetLastError();
     return SAGE_ERR_NOMEM;
   }

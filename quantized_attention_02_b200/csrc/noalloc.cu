@@ -1,7 +1,7 @@
 // noalloc.cu -- sage_attn_fwd_noalloc: the whole forward pass without any allocation.
 //
 // sage_attn_fwd needs a workspace for the INT8 copies of Q and K, their scales and the K
-// mean, and gets it with cudaMallocAsync.  Some callers cannot allocate device memory at
+// mean, and gets it with a stream-ordered allocation.  Some callers cannot allocate device memory at
 // call time: code running inside a CUDA-graph capture that must not add allocation nodes,
 // embedded or real-time hosts whose memory budget is fixed after start-up, plugins of
 // frameworks that own every allocation themselves.  For them this entry point uses a
