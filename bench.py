@@ -77,11 +77,26 @@ class ClockSampler:
         self.window = [float("inf")]
         self.window_closed = False
 
+    def _sample_now(self):
+        nv = self._nvml
+        if nv is None:
+            return
+        try:
+            h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                 nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                                 nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                 nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+        except Exception:
+            pass
+
     def open_window(self):
+        self._sample_now()  # right before the first timed step (short runs get a sample too)
         self.window[0] = time.perf_counter()
 
     def close_window(self):
         self.window_closed = True
+        self._sample_now()  # right after the last timed step completed
 
     def _run(self):
         nv = self._nvml
