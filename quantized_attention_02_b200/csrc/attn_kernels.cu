@@ -398,10 +398,16 @@ __global__ void __launch_bounds__(384, 1)
             for (int c = 0; c < 128; ++c) x[c] += kMagicBits;
           }
           if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
-          mx = -INFINITY;
+          // max of S * sk over the row's keys (masked: -inf), then times a_r >= 0
+          float m3 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            mx = fmaxf(mx, (__uint_as_float(x[c]) - kMagicF) * (a_r * skj[c]));
+          for (int c = 0; c < 128; c += 2) {
+            const float2 v = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
+                                                   make_float2(-kMagicF, -kMagicF)),
+                                        *reinterpret_cast<const float2*>(skj + c));
+            m3 = fmaxf(m3, fmaxf(v.x, v.y));
+          }
+          mx = m3 == -INFINITY ? -INFINITY : a_r * m3;
         } else {
           // integer maxima of the two 64-key halves (one key scale each); masked keys INT_MIN
           cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
@@ -465,8 +471,11 @@ __global__ void __launch_bounds__(384, 1)
             const int c = cb + i;
             float2 tt;
             if constexpr (PER_TOKEN) {
-              tt.x = fmaf(__uint_as_float(x[c]) - kMagicF, a_r * skj[c], -m_use);
-              tt.y = fmaf(__uint_as_float(x[c + 1]) - kMagicF, a_r * skj[c + 1], -m_use);
+              // fl(fl(S * sk) * a_r - m_use)
+              const float2 v = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
+                                                     make_float2(-kMagicF, -kMagicF)),
+                                          *reinterpret_cast<const float2*>(skj + c));
+              tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
             } else {
               const float cs = c < 64 ? cb0 : cb1;
               const float nb = c < 64 ? nb0 : nb1;
@@ -501,8 +510,9 @@ __global__ void __launch_bounds__(384, 1)
               const int c = 8 * c8 + i;
               float2 tt;
               if constexpr (PER_TOKEN) {
-                tt.x = fmaf(static_cast<float>(static_cast<int>(y[i])), a_r * skj[c], -m_use);
-                tt.y = fmaf(static_cast<float>(static_cast<int>(y[i + 1])), a_r * skj[c + 1], -m_use);
+                const float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(y[i])), static_cast<float>(static_cast<int>(y[i + 1]))),
+                                            *reinterpret_cast<const float2*>(skj + c));
+                tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
               } else {
                 const float cs = c < 64 ? cb0 : cb1;
                 const float nb = c < 64 ? nb0 : nb1;

@@ -31,10 +31,12 @@ struct V3Layout {
   static constexpr int OFF_ALPHA = OFF_P + P_BYTES;       // [2][256] fp32 rescale factors
   static constexpr int OFF_L = OFF_ALPHA + 2 * 256 * 4;   // [256] fp32 row sums
   static constexpr int OFF_FLAG = OFF_L + 256 * 4;        // [2][3] int rescale votes
-  static constexpr int OFF_BAR = OFF_FLAG + 32;
+  static constexpr int OFF_SKS = OFF_FLAG + 32;           // [2 tiles][2][128] fp32 per-token key scales
+  static constexpr int OFF_BAR = OFF_SKS + 2 * 2 * 128 * 4;
   // q, k_full/empty, v_full/empty, then per tile: s_full, s_free, p_lo, p_hi, o_lo, o_done, vote,
-  // corr_done, l_ready, drain, plus the Q.K^T warp's drain and 1 epilogue barrier
-  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 10 * 2 + 2;
+  // corr_done, l_ready, drain, key scales staged, plus the Q.K^T warp's drain and 1 epilogue
+  // barrier
+  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 11 * 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 512;
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_l = bar_corr + 2;              // [2] softmax t published 1 / l
   uint64_t* bar_drain = bar_l + 2;             // [3] MMA warps' completion at exit
   uint64_t* bar_epi = bar_drain + 3;           // correction group internal sync
+  uint64_t* bar_sks = bar_epi + 1;             // [2] per-token key scales of softmax t's next key tile staged
+  float* sSKs = reinterpret_cast<float*>(smem + L::OFF_SKS);  // [2 tiles][2][128] per-token key scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -175,6 +179,8 @@ __global__ void __launch_bounds__(512, 1)
     }
     mbar_init(bar_drain + 2, 1);
     mbar_init(bar_epi, 128);
+    mbar_init(bar_sks, 128);
+    mbar_init(bar_sks + 1, 128);
     for (int i = 0; i < 6; ++i) sFlag[i] = 0;
     *abort_flag = 0;
     fence_barrier_init();
@@ -336,6 +342,19 @@ __global__ void __launch_bounds__(512, 1)
         qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
       }
 
+      // per-token key scales: thread r fetches scale r of a key tile (zero past N) and the group
+      // publishes the 128 of them in shared memory, double-buffered, for all its rows; the fetch
+      // for key tile j+1 is issued early in iteration j and stored at its end
+      float* sks_t = sSKs + t * 256;
+      auto key_scale = [&](int jj) -> float {
+        const int key = jj * L::BN + r;
+        return key < N ? __ldg(sk_head + key) : 0.f;
+      };
+      if constexpr (PER_TOKEN) {
+        sks_t[r] = key_scale(0);
+        mbar_arrive(bar_sks + t);
+      }
+
       float m_use = 0.f;
       float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       bool ok = true;
@@ -343,13 +362,17 @@ __global__ void __launch_bounds__(512, 1)
         if (!wait_warp(bar_s_full + t, j & 1)) { ok = false; break; }
         tc_fence_after();
         if (r == 0) stamp((3 * t) * n_kv_total + j);
+        const float* skj = sks_t + (j & 1) * 128;  // per-token key scales of key tile j (shared memory)
+        float sk_next = 0.f;
+        if constexpr (PER_TOKEN) {
+          if (j + 1 < n_iter[t]) sk_next = key_scale(j + 1);
+          if (!wait_warp(bar_sks + t, j & 1)) { ok = false; break; }
+        }
         // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
         // c > cmax of this tile are left out of the maximum and get P~ = 0
         const int kvalid = N - j * L::BN;
         const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
         const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
-        const int klast = min(kvalid, L::BN) - 1;  // per-token key scales are read up to here
-        const float* skj = sk_head + j * L::BN;  // per-token key scales (global, L1/L2 resident)
 
         // ---- row maximum of the dequantized scores (log2 units), S read in two halves
         float mx = -INFINITY;
@@ -363,11 +386,20 @@ __global__ void __launch_bounds__(512, 1)
           uint32_t x[64];
           tmem_ld64_sync(tS + 64 * h, x);
           if constexpr (PER_TOKEN) {
+            // max of S * sk over the row's keys (a_r >= 0 multiplies it afterwards)
+            float m3 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const float v = static_cast<float>(static_cast<int>(x[c])) * (a_r * skj[min(64 * h + c, klast)]);
-              if (!(diag && 64 * h + c > cmax)) mx = fmaxf(mx, v);
+            for (int c = 0; c < 64; c += 2) {
+              const int cc = 64 * h + c;
+              float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(x[c])), static_cast<float>(static_cast<int>(x[c + 1]))),
+                                    *reinterpret_cast<const float2*>(skj + cc));
+              if (diag) {
+                if (cc > cmax) v.x = -INFINITY;
+                if (cc + 1 > cmax) v.y = -INFINITY;
+              }
+              m3 = fmaxf(m3, fmaxf(v.x, v.y));
             }
+            if (m3 != -INFINITY) mx = fmaxf(mx, a_r * m3);
           } else {
             if (diag) {
 #pragma unroll
@@ -433,8 +465,10 @@ __global__ void __launch_bounds__(512, 1)
             const int c = cb + i;
             float2 tt;
             if constexpr (PER_TOKEN) {
-              tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[min(c, klast)], -m_use);
-              tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[min(c + 1, klast)], -m_use);
+              // fl(fl(S * sk) * a_r - m_use)
+              const float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(x[i])), static_cast<float>(static_cast<int>(x[i + 1]))),
+                                          *reinterpret_cast<const float2*>(skj + c));
+              tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
             } else {
               const float cs = c < 64 ? cb0 : cb1;
               const float nb = c < 64 ? nb0 : nb1;
@@ -486,8 +520,9 @@ __global__ void __launch_bounds__(512, 1)
               const int c = 8 * c8 + i;
               float2 tt;
               if constexpr (PER_TOKEN) {
-                tt.x = fmaf(static_cast<float>(static_cast<int>(x[i])), a_r * skj[min(c, klast)], -m_use);
-                tt.y = fmaf(static_cast<float>(static_cast<int>(x[i + 1])), a_r * skj[min(c + 1, klast)], -m_use);
+                const float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(x[i])), static_cast<float>(static_cast<int>(x[i + 1]))),
+                                            *reinterpret_cast<const float2*>(skj + c));
+                tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
               } else {
                 const float cs = c < 64 ? cb0 : cb1;
                 const float nb = c < 64 ? nb0 : nb1;
@@ -508,6 +543,12 @@ __global__ void __launch_bounds__(512, 1)
           return true;
         };
         if (!(diag ? exp_pass_masked() : exp_pass())) { ok = false; break; }
+        if constexpr (PER_TOKEN) {  // key scales of tile j+1 into the other buffer
+          if (j + 1 < n_iter[t]) {
+            sks_t[((j + 1) & 1) * 128 + r] = sk_next;
+            mbar_arrive(bar_sks + t);
+          }
+        }
         if (r == 0) stamp((3 * t + 2) * n_kv_total + j);
       }
       if (ok) {
