@@ -8,12 +8,12 @@
 namespace sage {
 
 struct AttnArgs {
-  const CUtensorMap* tm_q;  // int8 [BH*N, D], box {D, 128}, 128 B (D=128) / 64 B (D=64) swizzle
-  const CUtensorMap* tm_k;  // int8 [BH*N, D], same boxes
-  const CUtensorMap* tm_v;  // fp16 [BH*N, D], box {64, 128}, 128 B swizzle
-  const CUtensorMap* tm_o;  // fp16 [BH*N, D], box {64, 128}, no swizzle (TMA store of O, D = 128)
-  const float* sq;          // [BH, N] per token or [BH, N/128] per block
-  const float* sk;          // [BH, N] per token or [BH, N/64] per block
+  const CUtensorMap* tm_q;  // int8 [BH][N][D] (3-D), box {D, 128, 1}, 128 B (D=128) / 64 B (D=64) swizzle
+  const CUtensorMap* tm_k;  // int8 [BH][N][D] (3-D), same boxes
+  const CUtensorMap* tm_v;  // fp16 [BH][N][D] (3-D), box {64, 128, 1}, 128 B swizzle
+  const CUtensorMap* tm_o;  // fp16 [BH][N][D] (3-D), box {64, 128, 1}, no swizzle (TMA store of O, D = 128)
+  const float* sq;          // [BH, N] per token or [BH, ceil(N/128)] per block
+  const float* sk;          // [BH, N] per token or [BH, ceil(N/64)] per block
   __half* o;                // fp16 [BH, N, D]
   int BH, N, D;
   bool causal, per_token;

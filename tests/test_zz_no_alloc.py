@@ -2,8 +2,8 @@
 
 Some callers cannot let a library allocate while they run: a CUDA-graph capture that must
 stay free of allocation nodes, a host whose device-memory budget is fixed at start-up, a
-framework plugin whose host owns every allocation.  sage_attn_fwd gets its workspace with
-cudaMallocAsync, so it is not usable there; sage_attn_fwd_noalloc runs the same kernels on
+framework plugin whose host owns every allocation.  sage_attn_fwd gets its workspace with a
+stream-ordered allocation, so it is not usable there; sage_attn_fwd_noalloc runs the same kernels on
 a fixed scratch array compiled into the library.
 
 This file is collected last on purpose: it must pass on its own in a fresh process (where
@@ -39,6 +39,7 @@ def test_noalloc_matches_sage_attn_fwd_on_two_calls_in_a_row():
     cases = [
         W.Workload("noalloc_a", 1, 4, 1024, 128, True, True, n_out=8, out_mag=30.0),
         W.Workload("noalloc_b", 2, 3, 512, 64, False, False, n_out=4, out_mag=20.0),
+        W.Workload("noalloc_c_ragged", 1, 2, 777, 128, True, False, n_out=4, out_mag=20.0),
     ]
     stream = torch.cuda.current_stream()
     for w in cases:  # two calls in a row; the second finds the first one's scratch contents
