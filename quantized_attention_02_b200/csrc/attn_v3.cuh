@@ -33,10 +33,10 @@ struct V3Layout {
   static constexpr int OFF_FLAG = OFF_L + 256 * 4;        // [2][3] int rescale votes
   static constexpr int OFF_SKS = OFF_FLAG + 32;           // [2 tiles][2][128] fp32 per-token key scales
   static constexpr int OFF_BAR = OFF_SKS + 2 * 2 * 128 * 4;
-  // q, k_full/empty, v_full/empty, then per tile: s_full, s_free, p_lo, p_hi, o_done, vote,
+  // q, k_full/empty, v_full/empty, then per tile: s_full, s_free, p_lo, p_hi, o_done, 2 votes,
   // corr_done, l_ready, drain, key scales staged, plus the Q.K^T warp's drain and 1 epilogue
   // barrier
-  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 10 * 2 + 2;
+  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 11 * 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 512;
@@ -112,8 +112,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_p_lo = bar_s_free + 2;         // [2] P~ keys 0..63 of tile t in shared memory
   uint64_t* bar_p_hi = bar_p_lo + 2;           // [2] P~ keys 64..127 of tile t in shared memory
   uint64_t* bar_o_done = bar_p_hi + 2;         // [2] a whole P.V with tile t's queries done
-  uint64_t* bar_vote = bar_o_done + 2;         // [2] softmax t published its rescale factors
-  uint64_t* bar_corr = bar_vote + 2;           // [2] O^T columns of tile t corrected
+  uint64_t* bar_vote = bar_o_done + 2;         // [2 tiles][2] softmax t published its rescale factors
+                                               // (key tile j uses bar_vote[2t + (j & 1)])
+  uint64_t* bar_corr = bar_vote + 4;           // [2] O^T columns of tile t corrected
   uint64_t* bar_l = bar_corr + 2;              // [2] softmax t published 1 / l
   uint64_t* bar_drain = bar_l + 2;             // [3] MMA warps' completion at exit
   uint64_t* bar_epi = bar_drain + 3;           // correction group internal sync
@@ -170,7 +171,8 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_p_lo + t, 128);
       mbar_init(bar_p_hi + t, 128);
       mbar_init(bar_o_done + t, 1);
-      mbar_init(bar_vote + t, 128);
+      mbar_init(bar_vote + 2 * t, 128);
+      mbar_init(bar_vote + 2 * t + 1, 128);
       mbar_init(bar_corr + t, 128);
       mbar_init(bar_l + t, 128);
       mbar_init(bar_drain + t, 1);
@@ -421,14 +423,15 @@ __global__ void __launch_bounds__(512, 1)
           rescale = true;
         }
         if (j > 0) {
-          // the correction group has consumed the previous vote (its barrier phase, factors and
-          // flag slot are reused): bounds how far this group runs ahead of it
-          if (j > 1 && !wait_warp(bar_corr + t, (j - 2) & 1)) { ok = false; break; }
+          // Run-ahead bound, without a wait: this vote's barrier, factor slot and flag slot were
+          // last used by key tile j-2, and the correction group has consumed that vote, because
+          // the P.V of key tile j-2 (which waits for that correction) completed before this
+          // group's exp2 pass of key tile j-1 began.
           sAlpha[(j & 1) * 256 + qi] = alpha;
           int* flag = sFlag + t * 3;
           if (r == 0) flag[(j + 1) % 3] = 0;  // slot of iteration j+1, last read by iteration j-2's correction
           if (__any_sync(0xffffffffu, rescale) && lane == 0) atomicOr(flag + j % 3, 1);
-          mbar_arrive(bar_vote + t);
+          mbar_arrive(bar_vote + 2 * t + (j & 1));
           if (rescale) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
@@ -564,7 +567,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int j = 1; ok && j < n_kv; ++j) {
       for (int t = 0; t < n_tiles; ++t) {
         if (j >= n_iter[t]) continue;
-        if (!wait_warp(bar_vote + t, (j - 1) & 1)) { ok = false; break; }
+        if (!wait_warp(bar_vote + 2 * t + (j & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
         if (sFlag[t * 3 + j % 3]) {
           // O^T holds the products up to key tile j-1: wait for the last of them
           if (!wait_warp(bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
