@@ -140,9 +140,10 @@ int sage_last_device_error(void* stream);
 /* ---------------------------------------------------------------------------------------
  * Allocation-free variant of sage_attn_fwd.  The SageAttention page has no counterpart of
  * this entry point: it exists for callers that cannot allocate device memory while they
- * run -- e.g. code being captured into a CUDA graph that must not contain allocations, or
- * hosts whose device-memory budget is fixed at start-up -- and so cannot use the
- * stream-ordered workspace of sage_attn_fwd.
+ * run -- hosts whose device-memory budget is fixed at start-up (embedded and real-time
+ * services), and plugins of frameworks that own every device allocation themselves and
+ * forbid a library from calling the CUDA allocator -- and so cannot use the stream-ordered
+ * workspace of sage_attn_fwd.
  *
  * Same arguments, results and validation as sage_attn_fwd (bit-identical output), but the
  * workspace (INT8 Q/K, scales, K mean) lives in a scratch array compiled into the library:

@@ -2,9 +2,9 @@
 //
 // sage_attn_fwd needs a workspace for the INT8 copies of Q and K, their scales and the K
 // mean, and gets it with a stream-ordered allocation.  Some callers cannot allocate device memory at
-// call time: code running inside a CUDA-graph capture that must not add allocation nodes,
-// embedded or real-time hosts whose memory budget is fixed after start-up, plugins of
-// frameworks that own every allocation themselves.  For them this entry point uses a
+// call time: embedded or real-time hosts whose memory budget is fixed after start-up, and
+// plugins of frameworks that own every allocation themselves and do not let a library call
+// the CUDA allocator.  For them this entry point uses a
 // fixed scratch area that lives in the library itself: a file-scope __device__ array that
 // every GPU which loads the library holds (kScratchBytes) until the process exits.
 //

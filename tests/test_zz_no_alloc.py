@@ -1,8 +1,8 @@
 """sage_attn_fwd_noalloc: the forward pass for callers that cannot allocate device memory.
 
-Some callers cannot let a library allocate while they run: a CUDA-graph capture that must
-stay free of allocation nodes, a host whose device-memory budget is fixed at start-up, a
-framework plugin whose host owns every allocation.  sage_attn_fwd gets its workspace with a
+Some callers cannot let a library allocate while they run: a host whose device-memory
+budget is fixed at start-up, or a framework plugin whose host owns every device allocation
+and does not let the library call the CUDA allocator.  sage_attn_fwd gets its workspace with a
 stream-ordered allocation, so it is not usable there; sage_attn_fwd_noalloc runs the same kernels on
 a fixed scratch array compiled into the library.
 
@@ -42,21 +42,24 @@ def test_noalloc_matches_sage_attn_fwd_on_two_calls_in_a_row():
         W.Workload("noalloc_c_ragged", 1, 2, 777, 128, True, False, n_out=4, out_mag=20.0),
     ]
     stream = torch.cuda.current_stream()
-    for w in cases:  # two calls in a row; the second finds the first one's scratch contents
-        q, k, v = (t.cuda() for t in W.make_qkv(w))
+    for w in cases:
         gran = sa.SAGE_PER_BLOCK if w.per_block else sa.SAGE_PER_TOKEN
         assert sa.sage_noalloc_scratch_bytes(w.B, w.H, w.N, w.d, gran) <= 64 << 20
-        o_ref = torch.empty_like(q)
-        sa.sage_attn_fwd(q, k, v, o_ref, w.causal, w.sm_scale, gran, stream)
-        o = torch.empty_like(q)
-        rc = lib.sage_attn_fwd_noalloc(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                       ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
-                                       w.B, w.H, w.N, w.d, int(w.causal), float(w.sm_scale), gran,
-                                       ctypes.c_void_p(stream.cuda_stream))
-        assert rc == sa.SAGE_OK, sa.sage_status_string(rc)
-        torch.cuda.synchronize()
-        assert sa.sage_last_device_error() == 0
-        _close(o, o_ref, float(v.abs().max()))
+        # two calls in a row on different inputs: the second one finds the first one's
+        # codes and scales in the shared scratch array and must not depend on them
+        for seed in (0, 1):
+            q, k, v = (t.cuda() for t in W.make_qkv(w, seed=seed))
+            o_ref = torch.empty_like(q)
+            sa.sage_attn_fwd(q, k, v, o_ref, w.causal, w.sm_scale, gran, stream)
+            o = torch.empty_like(q)
+            rc = lib.sage_attn_fwd_noalloc(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                           ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                           w.B, w.H, w.N, w.d, int(w.causal), float(w.sm_scale), gran,
+                                           ctypes.c_void_p(stream.cuda_stream))
+            assert rc == sa.SAGE_OK, sa.sage_status_string(rc)
+            torch.cuda.synchronize()
+            assert sa.sage_last_device_error() == 0
+            _close(o, o_ref, float(v.abs().max()))
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
