@@ -37,6 +37,8 @@ import workloads as W  # noqa: E402
 
 METRIC = "SageAttn fwd TOPS (4N²d·BH/time) at N=16k,d=128; % of INT8+FP16 roofline"
 UNIT = "TOPS"
+# kernels one sage_attn_fwd call launches: K channel means, Q and K quantization, fused attention
+KERNELS_PER_STEP = 4
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -342,7 +344,7 @@ def run_ours(args, w: W.Workload):
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }
     if world > 1:

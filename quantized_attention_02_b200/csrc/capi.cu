@@ -209,12 +209,8 @@ int sage_quant_qk(const void* q, const void* k, const float* km, int8_t* q8, int
   if ((rc = check_gran(granularity))) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8)) return SAGE_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool pt = granularity == SAGE_PER_TOKEN;
-  const int BH = B * H;
-  cudaError_t e = sage::launch_quant(static_cast<const __half*>(q), nullptr, q8, sq, BH, N, d, pt ? 1 : 128, st);
-  if (e != cudaSuccess) return SAGE_ERR_CUDA;
-  e = sage::launch_quant(static_cast<const __half*>(k), km, k8, sk, BH, N, d, pt ? 1 : 64, st);
-  return cuda_status(e);
+  return cuda_status(sage::launch_quant_qk(static_cast<const __half*>(q), static_cast<const __half*>(k), km, q8, k8,
+                                           sq, sk, B * H, N, d, granularity == SAGE_PER_TOKEN, st));
 }
 
 int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v,

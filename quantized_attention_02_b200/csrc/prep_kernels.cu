@@ -8,7 +8,9 @@
 // Both are bit-exact by construction: the mean comes from an exact fixed-point sum, and
 // every floating-point step is a single IEEE-rounded operation written with the _rn
 // intrinsics (never contracted into an FMA), in the order the C ABI documents.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
+#include <algorithm>
 #include <cstdint>
 #include <type_traits>
 
@@ -16,72 +18,122 @@
 
 namespace sage {
 
-// fp16 bits -> the value times 2^24 as an exact integer.  A normal fp16 is
-// (1024 + mantissa) * 2^(exponent - 25); a subnormal is mantissa * 2^-24.
-// Infinity / NaN (exponent 31) map to a finite value (results are then unspecified).
-__device__ __forceinline__ long long half_bits_to_fixed(uint32_t h) {
-  const uint32_t e = (h >> 10) & 31u;
-  const uint32_t m = h & 1023u;
-  const long long mag = e ? (static_cast<long long>(m | 1024u) << (e - 1)) : static_cast<long long>(m);
-  return (h & 0x8000u) ? -mag : mag;
+namespace cg = cooperative_groups;
+
+// Exact channel sums without 64-bit integer work per element.  Every finite fp16 value x is
+// a multiple of 2^-24 with |x| < 2^16.  One rounding add of C = 1.5 * 2^17 (the sum stays in
+// [2^17, 2^18), where the fp32 spacing is 2^-6) gives t = C + h with h = x rounded to a
+// multiple of 2^-6; bits(t) - bits(C) = h * 2^6 exactly (an integer, |.| < 2^22); h = t - C and
+// lo = x - h are exact in fp32 (lo is a multiple of 2^-24 with |lo| <= 2^-7).  So
+//   x * 2^24 = (h * 2^6) * 2^18 + lo * 2^24
+// and a thread sums the h * 2^6 in int32 and the lo in fp32 -- both exact for up to 64 tokens
+// (|sum h * 2^6| < 2^28, |sum lo| <= 1/2 on the 2^-24 grid) -- then moves them into int64.
+// Per element that is fp32 adds (packed two at a time) and one integer add, instead of a
+// 64-bit shift-and-add.  Infinity / NaN inputs give unspecified (finite-time) results.
+constexpr float kSplitC = 196608.0f;          // 1.5 * 2^17
+constexpr int kSplitBits = 0x48400000;        // bits of kSplitC
+constexpr int kSplitFlushTokens = 64;         // tokens a thread adds between flushes
+
+__device__ __forceinline__ void split_acc(uint32_t word, int& h0, int& h1, float2& lo) {
+  const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&word));
+  const float2 t = __fadd2_rn(x, make_float2(kSplitC, kSplitC));
+  const float2 h = __fadd2_rn(t, make_float2(-kSplitC, -kSplitC));
+  lo = __fadd2_rn(lo, __fadd2_rn(x, make_float2(-h.x, -h.y)));
+  h0 += __float_as_int(t.x) - kSplitBits;
+  h1 += __float_as_int(t.y) - kSplitBits;
 }
 
-// One CTA of 1024 threads per (32-channel chunk, head): thread = (token phase 0..255, 16-byte
-// piece 0..3 of the 64-byte chunk row).  Each thread keeps four 16-byte loads in flight
-// (tokens t, t+256, t+512, t+768) so that the whole GPU has enough bytes in flight to run
-// at HBM speed even with few heads.
-template <int D>
-__global__ void __launch_bounds__(1024) smooth_k_kernel(const __half* __restrict__ k, float* __restrict__ km,
-                                                        int N) {
-  constexpr int PHASES = 256;
-  const int chunk = blockIdx.x;  // 32 channels
-  const int bh = blockIdx.y;
-  const int piece = threadIdx.x & 3;
-  const int tok0 = threadIdx.x >> 2;
-  const __half* base = k + (static_cast<size_t>(bh) * N) * D + chunk * 32 + piece * 8;
+// One thread-block cluster of C CTAs per head (C = 1, 2, 4 or 8, chosen from N at launch so
+// that every CTA gets at least 2048 tokens).  CTA r of the cluster sums the contiguous
+// token slice [r*S, min(N, (r+1)*S)), S = ceil(N / C), reading whole rows: a team of T = D/8
+// threads covers one token row with one 16-byte load each (coalesced), a 512-thread CTA covers
+// 512/T rows per pass and keeps four passes of loads in flight.  The per-CTA channel sums
+// (exact int64) meet in the cluster's rank-0 CTA through distributed shared memory, which
+// writes the mean: one read of K, no atomics, no workspace, and the integer total does not
+// depend on the order of the additions.
+constexpr int kSmoothMaxCtas = 8;
+constexpr int kSmoothThreads = 512;
+constexpr int kSmoothTokensPerCta = 2048;
 
+template <int D>
+__global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* __restrict__ k,
+                                                                  float* __restrict__ km, int N) {
+  constexpr int T = D / 8;                 // threads per token row
+  constexpr int R = kSmoothThreads / T;    // rows per pass
+  constexpr int U = 4;                     // passes in flight
+  constexpr int WARPS = kSmoothThreads / 32;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int n_ctas = static_cast<int>(cluster.num_blocks());  // the cluster spans grid x
+  const int bh = blockIdx.y;
+  const int piece = threadIdx.x % T;       // channels piece*8 .. piece*8+7
+  const int row = threadIdx.x / T;
+  const int slice = (N + n_ctas - 1) / n_ctas;
+  const int t0 = rank * slice;
+  const int t1 = min(N, t0 + slice);
+  const __half* base = k + (static_cast<size_t>(bh) * N) * D + piece * 8;
+
+  constexpr int ITERS = kSplitFlushTokens / U;  // loop iterations between flushes
   long long acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0;
-
-  for (int t = tok0; t < N; t += 4 * PHASES) {
-    uint4 w[4];
+  for (int t = t0 + row; t < t1;) {
+    int hs[8];
+    float2 ls[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      w[u] = (t + u * PHASES < N) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * PHASES) * D))
-                                  : make_uint4(0u, 0u, 0u, 0u);  // +0.0 contributes nothing
+    for (int i = 0; i < 8; ++i) hs[i] = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+    for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
+    for (int it = 0; it < ITERS && t < t1; ++it, t += U * R) {
+      uint4 w[U];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] += half_bits_to_fixed(words[i] & 0xFFFFu);
-        acc[2 * i + 1] += half_bits_to_fixed(words[i] >> 16);
+      for (int u = 0; u < U; ++u)
+        w[u] = (t + u * R < t1) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D))
+                                : make_uint4(0u, 0u, 0u, 0u);  // +0.0 contributes nothing
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_acc(words[i], hs[2 * i], hs[2 * i + 1], ls[i]);
       }
     }
+    // flush: x * 2^24 summed = (sum h*2^6) * 2^18 + (sum lo) * 2^24, both parts exact integers
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += (static_cast<long long>(hs[2 * i]) << 18) + __float2int_rn(__fmul_rn(ls[i].x, 16777216.0f));
+      acc[2 * i + 1] += (static_cast<long long>(hs[2 * i + 1]) << 18) + __float2int_rn(__fmul_rn(ls[i].y, 16777216.0f));
+    }
   }
-  // lanes sharing `piece` differ in lane bits 2..4
+  // lanes of a warp with the same piece differ by multiples of T
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+    for (int off = T; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
   }
-  __shared__ long long part[32][4][8];
+  __shared__ long long part[WARPS][T][8];
+  __shared__ long long csum[D];  // this CTA's channel sums, read by rank 0 of the cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane < 4) {
+  if (lane < T) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[warp][lane][i] = acc[i];
   }
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int p = threadIdx.x >> 3, i = threadIdx.x & 7;  // channel = chunk*32 + p*8 + i
+  if (threadIdx.x < D) {
+    const int p = threadIdx.x >> 3, i = threadIdx.x & 7;  // channel = p*8 + i = threadIdx.x
     long long s = 0;
 #pragma unroll
-    for (int w = 0; w < 32; ++w) s += part[w][p][i];
+    for (int w = 0; w < WARPS; ++w) s += part[w][p][i];
+    csum[threadIdx.x] = s;
+  }
+  cluster.sync();
+  if (rank == 0 && threadIdx.x < D) {
+    long long s = 0;
+    for (int r = 0; r < n_ctas; ++r) s += *cluster.map_shared_rank(csum + threadIdx.x, r);
     const float s32 = __ll2float_rn(s);
     const float mean = __fdiv_rn(s32, static_cast<float>(N));
-    km[static_cast<size_t>(bh) * D + chunk * 32 + p * 8 + i] = __fmul_rn(mean, 5.9604644775390625e-08f);
+    km[static_cast<size_t>(bh) * D + threadIdx.x] = __fmul_rn(mean, 5.9604644775390625e-08f);
   }
+  cluster.sync();  // every CTA keeps its csum in place until rank 0 has read it
 }
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
@@ -94,17 +146,21 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   }
 }
 
-__device__ __forceinline__ int quant1(float x, float inv) {
-  int q = __float2int_rn(__fmul_rn(x, inv));  // round half to even
-  return max(-127, min(127, q));
-}
+// INT8 codes of 8 values: y = fl(x * inv), code = round_half_even(y).  The rounding is one add
+// of 1.5 * 2^23: for |y| < 2^22 the sum lies in [2^23, 2^24), where the fp32 spacing is 1, so it
+// rounds y to the nearest integer (ties to even) and the low byte of its bits is the code in
+// two's complement.  No clamp is needed: |x| <= a and inv = fl(127/a) give
+// |y| <= 127 (1 + 2^-24)^2 < 127.5, so |code| <= 127 (a = 0 gives inv = 0 and codes 0).
+constexpr float kRoundC = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
-  uint32_t lo = 0, hi = 0;
+  // scalar _rn intrinsics: the product must be rounded before the add (a contracted
+  // multiply-add would round x * inv + C once and break ties differently)
+  uint32_t b[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) lo |= (static_cast<uint32_t>(quant1(x[i], inv)) & 0xFFu) << (8 * i);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) hi |= (static_cast<uint32_t>(quant1(x[4 + i], inv)) & 0xFFu) << (8 * i);
+  for (int i = 0; i < 8; ++i) b[i] = __float_as_uint(__fadd_rn(__fmul_rn(x[i], inv), kRoundC));
+  const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
 }
 
@@ -115,17 +171,18 @@ __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
 //   G  > 1 : the CTA is one group of G tokens held in registers (G/P passes), CTA-wide max.
 //            Groups tile each head separately: ceil(N/G) groups per head, the last one holding
 //            the N mod G remaining tokens when G does not divide N.
+// `blk` is the block's index within its tensor's part of the grid.
 template <int D, int G, bool SMOOTH>
-__global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x, const float* __restrict__ km,
-                                                    int8_t* __restrict__ q, float* __restrict__ scale, int N,
-                                                    long long rows) {
+__device__ __forceinline__ void quant_block(const __half* __restrict__ x, const float* __restrict__ km,
+                                            int8_t* __restrict__ q, float* __restrict__ scale, int N,
+                                            long long rows, unsigned blk) {
   constexpr int T = D / 8;
   constexpr int P = 256 / T;
   const int piece = threadIdx.x % T;
   const int c0 = piece * 8;
 
   if constexpr (G == 1) {
-    const size_t row = static_cast<size_t>(blockIdx.x) * P + threadIdx.x / T;
+    const size_t row = static_cast<size_t>(blk) * P + threadIdx.x / T;
     const bool live = row < static_cast<size_t>(rows);  // whole T-lane teams; all lanes stay for the shuffles
     // the load always reads an existing row (the last one for teams past the end), then is zeroed
     uint4 w = __ldg(reinterpret_cast<const uint4*>(x + (live ? row : static_cast<size_t>(rows) - 1) * D + c0));
@@ -155,8 +212,8 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
     static_assert(G % P == 0, "group must be a whole number of passes");
     constexpr int PASSES = G / P;
     const int n_groups = (N + G - 1) / G;
-    const int bh = static_cast<int>(blockIdx.x) / n_groups;
-    const int tok0 = (static_cast<int>(blockIdx.x) % n_groups) * G;  // first token of the group in its head
+    const int bh = static_cast<int>(blk) / n_groups;
+    const int tok0 = (static_cast<int>(blk) % n_groups) * G;  // first token of the group in its head
     const size_t row0 = static_cast<size_t>(bh) * N + tok0;
     const int tok = threadIdx.x / T;
     float mu[8];
@@ -207,16 +264,35 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
       const size_t row = row0 + p * P + tok;
       if (whole || tok0 + p * P + tok < N) *reinterpret_cast<uint2*>(q + row * D + c0) = pack8(v[p], inv);
     }
-    if (threadIdx.x == 0) scale[blockIdx.x] = s;
+    if (threadIdx.x == 0) scale[blk] = s;
   }
+}
+
+template <int D, int G, bool SMOOTH>
+__global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x, const float* __restrict__ km,
+                                                    int8_t* __restrict__ q, float* __restrict__ scale, int N,
+                                                    long long rows) {
+  quant_block<D, G, SMOOTH>(x, km, q, scale, N, rows, blockIdx.x);
 }
 
 // ---------------------------------------------------------------- launchers
 template <int D>
 static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cudaStream_t st) {
-  dim3 grid(D / 32, BH);
-  smooth_k_kernel<D><<<grid, 1024, 0, st>>>(k, km, N);
-  return cudaGetLastError();
+  int ctas = 1;  // a power of two, at most kSmoothMaxCtas, with >= kSmoothTokensPerCta tokens per CTA
+  while (ctas < kSmoothMaxCtas && N / (2 * ctas) >= kSmoothTokensPerCta) ctas *= 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), static_cast<unsigned>(BH));  // one cluster (grid x) per head
+  cfg.blockDim = dim3(kSmoothThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, smooth_k_kernel<D>, k, km, N);
 }
 
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st) {
@@ -234,25 +310,25 @@ static cudaError_t launch_quant_g(const __half* x, const float* km, int8_t* q, f
 }
 
 template <int D>
-static cudaError_t launch_quant_d(const __half* x, const float* km, int8_t* q, float* s, int BH, int N,
-                                  int group, cudaStream_t st) {
-  const bool sm = km != nullptr;
-  switch (group) {
-    case 1:
-      return sm ? launch_quant_g<D, 1, true>(x, km, q, s, BH, N, st) : launch_quant_g<D, 1, false>(x, km, q, s, BH, N, st);
-    case 64:
-      return sm ? launch_quant_g<D, 64, true>(x, km, q, s, BH, N, st) : launch_quant_g<D, 64, false>(x, km, q, s, BH, N, st);
-    case 128:
-      return sm ? launch_quant_g<D, 128, true>(x, km, q, s, BH, N, st) : launch_quant_g<D, 128, false>(x, km, q, s, BH, N, st);
-    default:
-      return cudaErrorInvalidValue;
+static cudaError_t launch_quant_qk_d(const __half* q, const __half* k, const float* km, int8_t* q8, int8_t* k8,
+                                     float* sq, float* sk, int BH, int N, bool per_token, cudaStream_t st) {
+  // two launches: measured faster than one launch over both tensors (each kernel keeps its own
+  // register count, so the K groups run at a higher occupancy)
+  cudaError_t e;
+  if (per_token) {
+    e = launch_quant_g<D, 1, false>(q, nullptr, q8, sq, BH, N, st);
+    if (e != cudaSuccess) return e;
+    return km ? launch_quant_g<D, 1, true>(k, km, k8, sk, BH, N, st) : launch_quant_g<D, 1, false>(k, km, k8, sk, BH, N, st);
   }
+  e = launch_quant_g<D, 128, false>(q, nullptr, q8, sq, BH, N, st);
+  if (e != cudaSuccess) return e;
+  return km ? launch_quant_g<D, 64, true>(k, km, k8, sk, BH, N, st) : launch_quant_g<D, 64, false>(k, km, k8, sk, BH, N, st);
 }
 
-cudaError_t launch_quant(const __half* x, const float* km, int8_t* q, float* s, int BH, int N, int D, int group,
-                         cudaStream_t st) {
-  return D == 128 ? launch_quant_d<128>(x, km, q, s, BH, N, group, st)
-                  : launch_quant_d<64>(x, km, q, s, BH, N, group, st);
+cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, int8_t* q8, int8_t* k8, float* sq,
+                            float* sk, int BH, int N, int D, bool per_token, cudaStream_t st) {
+  return D == 128 ? launch_quant_qk_d<128>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st)
+                  : launch_quant_qk_d<64>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st);
 }
 
 }  // namespace sage

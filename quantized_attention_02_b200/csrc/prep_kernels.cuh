@@ -9,9 +9,10 @@ namespace sage {
 // km[bh, c] = mean over N tokens of k[bh, :, c]; k fp16 [BH, N, D], km fp32 [BH, D].
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st);
 
-// Quantize x fp16 [BH, N, D] in groups of `group` tokens (1, 64 or 128) to int8 q and fp32
-// scales s [BH, N/group].  km (fp32 [BH, D]) is subtracted first when not null.
-cudaError_t launch_quant(const __half* x, const float* km, int8_t* q, float* s, int BH, int N, int D, int group,
-                         cudaStream_t st);
+// Quantize q and k fp16 [BH, N, D] to int8 q8 / k8 with fp32 scales sq / sk (one launch per
+// tensor): per token (per_token), else in groups of 128 Q tokens and 64 K tokens.  km (fp32 [BH, D])
+// is subtracted from k first when not null.
+cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, int8_t* q8, int8_t* k8, float* sq,
+                            float* sk, int BH, int N, int D, bool per_token, cudaStream_t st);
 
 }  // namespace sage
