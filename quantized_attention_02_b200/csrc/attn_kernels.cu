@@ -10,16 +10,17 @@
 //                                         A operand read straight from tensor memory)
 //   O   = O / l                           stored as fp16
 //
-// CTA organisation (one CTA per SM: 512 TMEM columns and > 114 KB of shared memory):
+// CTA organisation (one CTA per SM: 512 TMEM columns and > 114 KB of shared memory), for head
+// dimension 64 (128 has its own kernel, attn_v3.cuh):
 //   work unit = (head, pair of 128-row query tiles); 12 warps:
 //     warp 0      TMA producer: Q tiles once, then K / V tiles through a STAGES-deep ring
-//     warp 1      TMEM allocator and single-thread MMA issuer
+//     warps 1, 2  MMA issuers of query tile 0 / 1 (warp 1 also allocates TMEM)
 //     warps 4-7   softmax for query tile 0 (thread = one query row = one TMEM lane)
 //     warps 8-11  softmax for query tile 1
-//   TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D); P~_t (fp16,
-//   64 columns) overwrites the first half of S_t once S_t has been read.
-//   The MMA issue order per key tile j is  PV0(j), QK0(j+1), PV1(j), QK1(j+1): the tensor core
-//   alternates between the two tiles' work.
+//   TMEM columns: S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384) P~0 [384,448) P~1 [448,512)
+//   (P~ fp16, two keys per column).  Per key tile j an MMA warp issues QK_t(j+1) as soon as the
+//   softmax has copied S_t(j) into registers (S_t is free), then PV_t(j) as the two halves of
+//   P~_t(j) arrive; the softmax waits for PV_t(j-1) before it writes P~_t(j) (one P~ buffer).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -46,13 +47,15 @@ struct AttnLayout {
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_SK = OFF_V + STAGES * V_BYTES;           // per-token key scales
   static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 5 * NQT;
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 6 * NQT;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int USED = OFF_MISC + 16;
   // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   static constexpr int SMEM = (USED + 1024 > 116 * 1024 ? USED + 1024 : 116 * 1024);
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t o_col(int t) { return 256u + D * t; }
+  __host__ __device__ static constexpr uint32_t p_col(int t) { return 256u + 2 * D + 64u * t; }
+  static_assert(256 + 2 * D + 128 <= 512, "S, O and P~ of two query tiles fit the 512 TMEM columns");
   static constexpr int THREADS = 384;
 };
 
@@ -154,6 +157,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_o_done = bar_s_full + 4;
   uint64_t* bar_drain = bar_s_full + 6;   // one per MMA warp
   uint64_t* bar_p_lo = bar_s_full + 8;    // P~ of keys 0..63 written
+  uint64_t* bar_s_free = bar_s_full + 10; // softmax t holds S_t(j) in registers: S_t may be overwritten
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -206,6 +210,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar_drain + 1, 1);
     mbar_init(bar_p_lo, 128);
     mbar_init(bar_p_lo + 1, 128);
+    mbar_init(bar_s_free, 128);
+    mbar_init(bar_s_free + 1, 128);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
@@ -271,6 +277,8 @@ __global__ void __launch_bounds__(384, 1)
     // per warp leaves the tensor core idle between back-to-back instructions (about 110-140
     // cycles each), two independent streams keep it busy.  The whole warp runs the loop
     // (uniform control flow and descriptors); elect.sync lets one lane issue each instruction.
+    // Per key tile j: QK(j+1) first (it only needs S_t free and K(j+1)), so that the next scores
+    // are ready when the softmax finishes tile j; then PV(j) from the P~ region.
     const int t = warp - 1;
     if (t < n_tiles) {
       constexpr uint32_t IDESC_QK = make_idesc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, L::BN);
@@ -297,7 +305,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = k0; kk < k1; ++kk) {
           const uint64_t b = make_smem_desc(v_base + s * L::V_BYTES + kk * 16 * 128, L::V_BOX, 1024, kSwizzle128B);
-          mma_f16_ts_warp(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          mma_f16_ts_warp(tmem + L::o_col(t), tmem + L::p_col(t) + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
         }
       };
 
@@ -308,6 +316,15 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int j = 0; ok && j < n_iter[t]; ++j) {
         const int s = j % STAGES;
+        if (j + 1 < n_iter[t]) {
+          // S_t(j+1) overwrites S_t(j) once the softmax holds S_t(j) in registers
+          const int s1 = (j + 1) % STAGES;
+          if (!wait(bar_k_full + s1, ((j + 1) / STAGES) & 1)) break;
+          if (!wait(bar_s_free + t, j & 1)) break;
+          tc_fence_after();
+          issue_qk(s1);
+          if (lane == 0) stamp((7 + 2 * t) * n_kv_total + j);
+        }
         if (!wait(bar_v_full + s, (j / STAGES) & 1)) break;
         // the first half of P~ is signalled separately, so that its P.V overlaps the exp2
         // work on the second half
@@ -320,15 +337,6 @@ __global__ void __launch_bounds__(384, 1)
         issue_pv(s, false, L::BN / 32, L::BN / 16);
         mma_commit_warp(bar_o_done + t);
         if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
-        if (j + 1 < n_iter[t]) {
-          // S_t(j+1) overwrites P~_t(j): tcgen05 MMAs issued by one thread execute in issue
-          // order, so the P.V above has read P~_t before this product writes S_t.
-          const int s1 = (j + 1) % STAGES;
-          if (!wait(bar_k_full + s1, ((j + 1) / STAGES) & 1)) break;
-          tc_fence_after();
-          issue_qk(s1);
-          if (lane == 0) stamp((7 + 2 * t) * n_kv_total + j);
-        }
         mma_commit_warp(bar_kv_empty + s);  // this tile's products reading stage s are issued
       }
       // all MMAs issued by this warp must finish before TMEM is released
@@ -348,6 +356,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
       const uint32_t tS = tmem + lane_addr + L::s_col(t);
       const uint32_t tO = tmem + lane_addr + L::o_col(t);
+      const uint32_t tP = tmem + lane_addr + L::p_col(t);
       // rows past N (a partial last tile) compute on zeros and are never stored
       const float sq_r = PER_TOKEN ? (q_row < N ? __ldg(sq + row_base + q_row) : 0.f) : __ldg(sq + bh * n_qtiles + q_tile);
       const float a_r = sq_r * sm_scale_log2;  // log2-unit value of one integer step, before sk
@@ -375,14 +384,18 @@ __global__ void __launch_bounds__(384, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
         if (r == 0) stamp((3 * t) * n_kv_total + j);
+        // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
+        // c > cmax of this tile are left out of the maximum and get P~ = 0.  Such a tile is
+        // always the last key tile of its query tile.
+        const int kvalid = N - j * L::BN;
+        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
         uint32_t x[128];
         tmem_ld64_sync(tS + 0, *reinterpret_cast<uint32_t(*)[64]>(x + 0));
         tmem_ld64_sync(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(x + 64));
-
-        // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
-        // c > cmax of this tile are left out of the maximum and get P~ = 0
-        const int kvalid = N - j * L::BN;
-        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
+        if (!diag) {  // S_t is in registers: the next Q.K^T may overwrite it (masked tiles re-read it)
+          tc_fence_before();
+          mbar_arrive(bar_s_free + t);
+        }
         const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
         const int s = j % STAGES;
         float mx;            // row maximum of the dequantized scores (log2 units)
@@ -440,11 +453,14 @@ __global__ void __launch_bounds__(384, 1)
           m_use = m_new;
           rescale = true;
         }
+        // P.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1)
+        if (j > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { ok = false; break; }
+          tc_fence_after();
+        }
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll
           for (int cb = 0; cb < D; cb += 32) {
             uint32_t ov[32];
@@ -487,7 +503,7 @@ __global__ void __launch_bounds__(384, 1)
             lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
             pk[i >> 1] = pack_half2(p.x, p.y);
           }
-          tmem_st16(tS + (cb >> 1), pk);
+          tmem_st16(tP + (cb >> 1), pk);
           if (cb == 32) {  // keys 0..63 done: let their P.V start
             tmem_wait_st();
             tc_fence_before();
@@ -497,8 +513,7 @@ __global__ void __launch_bounds__(384, 1)
         };
         // ---- the same for a tile with masked keys (c > cmax: the causal diagonal, a partial last
         // tile), at most one per row: a rolled loop over 8-key steps that re-reads S from TMEM
-        // 8 columns at a time (P~ of a step lands on columns already read), so that this rare
-        // case adds little code next to the unrolled pass
+        // 8 columns at a time, so that this rare case adds little code next to the unrolled pass
         auto exp_pass_masked = [&]() {
 #pragma unroll 1
           for (int c8 = 0; c8 < 16; ++c8) {
@@ -523,7 +538,7 @@ __global__ void __launch_bounds__(384, 1)
               lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
               pk[i >> 1] = pack_half2(p.x, p.y);
             }
-            tmem_st4(tS + 4 * c8, pk);
+            tmem_st4(tP + 4 * c8, pk);
             if (c8 == 7) {  // keys 0..63 done: let their P.V start
               tmem_wait_st();
               tc_fence_before();
@@ -531,8 +546,13 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         };
-        if (diag) exp_pass_masked();
-        else exp_pass();
+        if (diag) {
+          exp_pass_masked();
+          tc_fence_before();
+          mbar_arrive(bar_s_free + t);  // its re-reads of S_t are done
+        } else {
+          exp_pass();
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p_full + t);

@@ -82,8 +82,10 @@ SWEEP_D = (64, 128)
 HEADLINE = sweep(16384, 128, False)
 # a quarter of the headline problem (inputs still larger than L2) for profiler captures
 PROFILE = Workload("profile_b1h16_n16384_d128", 1, 16, 16384, 128, False, True, n_out=4, out_mag=20.0)
+# the video-DiT shape with a sixth of its heads: small enough for a full profiler capture
+PROFILE64 = Workload("profile_b1h16_n16384_d64", 1, 16, 16384, 64, False, True, bias_std=4.0)
 
-ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE)}
+ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
