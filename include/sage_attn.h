@@ -133,7 +133,9 @@ int sage_debug_mma_rate(int mode, int n, int chains, int issuers, int iters, int
                         int* status, void* stream);
 
 /* Waits for all work on stream, then returns and clears the device status word written by
- * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out).  Returns
+ * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out; 2, from
+ * sage_debug_attn_trace only: a CTA barrier let a thread through before every thread had
+ * arrived).  Returns
  * SAGE_ERR_CUDA (negative) if the synchronization itself failed. */
 int sage_last_device_error(void* stream);
 

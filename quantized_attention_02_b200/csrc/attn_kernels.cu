@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_s_free = bar_s_full + 10; // softmax t holds S_t(j) in registers: S_t may be overwritten
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  int* arrived = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);  // trace builds: threads at the final barrier
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(384, 1)
   if constexpr (TRACE) {
     if (static_cast<int>(blockIdx.x) < trace_ctas) {
       trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * n_kv_total);
-      if (threadIdx.x == 0) trace_row[0] = clock64();
+      if (threadIdx.x == 0) trace_row[0] = clock_stamp();
     }
   }
   // trace slots: [0] start, [1] end, then per key tile j: softmax group t events e (0 S ready,
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(384, 1)
   // 1 next Q.K^T issued) for tile t at 2 + (6 + 2t + e) n_kv_total + j
   auto stamp = [&](int slot) {
     if constexpr (TRACE) {
-      if (trace_row) trace_row[2 + slot] = clock64();
+      if (trace_row) trace_row[2 + slot] = clock_stamp();
     }
   };
 
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar_s_free, 128);
     mbar_init(bar_s_free + 1, 128);
     *abort_flag = 0;
+    *arrived = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();  // lane 0 of warp 0 initialised the barriers alone
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -583,10 +585,14 @@ __global__ void __launch_bounds__(384, 1)
     }
   }
 
+  // roles diverge inside warps (single-lane producers and stores): the thread-counting barrier
+  // holds the TMEM release until every thread of the CTA is done
   tc_fence_before();
-  __syncthreads();
-  if constexpr (TRACE) {
-    if (trace_row && threadIdx.x == 0) trace_row[1] = clock64();
+  if constexpr (TRACE) {  // also checks that the barrier held every thread
+    const long long t_end = cta_end_checked(arrived, threadIdx.x == 0);
+    if (trace_row && threadIdx.x == 0) trace_row[1] = t_end;
+  } else {
+    cta_sync();
   }
   if (warp == 1) {
     tc_fence_after();
@@ -636,7 +642,7 @@ __global__ void __launch_bounds__(256, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();  // lane 0 of warp 0 initialised the barriers alone
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -688,8 +694,10 @@ __global__ void __launch_bounds__(256, 1)
       mbar_arrive(bar_free);
     }
   }
+  // roles diverge inside warps (single-lane producers and stores): the thread-counting barrier
+  // holds the TMEM release until every thread of the CTA is done
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);

@@ -34,9 +34,8 @@ struct V3Layout {
   static constexpr int OFF_SKS = OFF_FLAG + 32;           // [2 tiles][2][128] fp32 per-token key scales
   static constexpr int OFF_BAR = OFF_SKS + 2 * 2 * 128 * 4;
   // q, k_full/empty, v_full/empty, then per tile: s_full, s_free, p_lo, p_hi, o_done, 2 votes,
-  // corr_done, l_ready, drain, key scales staged, plus the Q.K^T warp's drain and 1 epilogue
-  // barrier
-  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 11 * 2 + 2;
+  // corr_done, drain, key scales staged, plus the Q.K^T warp's drain
+  static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 10 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 512;
@@ -63,6 +62,10 @@ __device__ __forceinline__ float2 exp2_poly2(float2 t) {
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(y.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(y.y) << 23)));
 }
+
+// Barrier of one 128-thread warpgroup: named barrier `id` (1, 2, ...; 0 is the CTA barrier),
+// counted per thread, so warps may arrive diverged.
+__device__ __forceinline__ void group_sync(int id) { asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory"); }
 
 // CTA-wide vote helpers -----------------------------------------------------------------
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -115,13 +118,12 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_vote = bar_o_done + 2;         // [2 tiles][2] softmax t published its rescale factors
                                                // (key tile j uses bar_vote[2t + (j & 1)])
   uint64_t* bar_corr = bar_vote + 4;           // [2] O^T columns of tile t corrected
-  uint64_t* bar_l = bar_corr + 2;              // [2] softmax t published 1 / l
-  uint64_t* bar_drain = bar_l + 2;             // [3] MMA warps' completion at exit
-  uint64_t* bar_epi = bar_drain + 3;           // correction group internal sync
-  uint64_t* bar_sks = bar_epi + 1;             // [2] per-token key scales of softmax t's next key tile staged
+  uint64_t* bar_drain = bar_corr + 2;          // [3] MMA warps' completion at exit
+  uint64_t* bar_sks = bar_drain + 3;           // [2] per-token key scales of softmax t's next key tile staged
   float* sSKs = reinterpret_cast<float*>(smem + L::OFF_SKS);  // [2 tiles][2][128] per-token key scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  int* arrived = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);  // trace builds: threads at the final barrier
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -144,14 +146,14 @@ __global__ void __launch_bounds__(512, 1)
   if constexpr (TRACE) {
     if (static_cast<int>(blockIdx.x) < trace_ctas) {
       trace_row = trace + static_cast<size_t>(blockIdx.x) * (2 + 10 * n_kv_total);
-      if (threadIdx.x == 0) trace_row[0] = clock64();
+      if (threadIdx.x == 0) trace_row[0] = clock_stamp();
     }
   }
   // trace slots as documented at sage_debug_attn_trace; MMA event 0 = the P.V containing
   // tile t's queries issued, event 1 = Q.K^T of tile t issued (for key tile j + 1)
   auto stamp = [&](int slot) {
     if constexpr (TRACE) {
-      if (trace_row) trace_row[2 + slot] = clock64();
+      if (trace_row) trace_row[2 + slot] = clock_stamp();
     }
   };
 
@@ -174,15 +176,14 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar_vote + 2 * t, 128);
       mbar_init(bar_vote + 2 * t + 1, 128);
       mbar_init(bar_corr + t, 128);
-      mbar_init(bar_l + t, 128);
       mbar_init(bar_drain + t, 1);
     }
     mbar_init(bar_drain + 2, 1);
-    mbar_init(bar_epi, 128);
     mbar_init(bar_sks, 128);
     mbar_init(bar_sks + 1, 128);
     for (int i = 0; i < 6; ++i) sFlag[i] = 0;
     *abort_flag = 0;
+    *arrived = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(512, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();  // lane 0 of warp 0 initialised the barriers alone
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S_0 [0,128), S_1 [128,256), O^T [256,512) with column 256 + q for the CTA's
@@ -551,17 +552,42 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (r == 0) stamp((3 * t + 2) * n_kv_total + j);
       }
+      // ---- epilogue of this query tile by its own softmax group (both tiles in parallel):
+      // O[q][d] = O^T[d][q] / l_q -> fp16, staged in the tile's own P~ rows (two [128 q][64 d]
+      // pieces; this thread is TMEM lane d = r of O^T), then TMA-stored by one thread
+      // Every thread of the group reaches both group barriers on every path (a warp whose
+      // bounded wait gave up skips only the work), so a timeout cannot strand the group.
+      const float2 l2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+      sL[qi] = 1.f / (l2.x + l2.y);
+      group_sync(1 + t);  // the tile's 1 / l complete
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (n_iter[t] - 1) & 1, abort_flag));
       if (ok) {
-        const float2 l2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
-        sL[qi] = 1.f / (l2.x + l2.y);
-        mbar_arrive(bar_l + t);
+        tc_fence_after();
+        const uint32_t tOT = tmem + lane_addr + 256 + 128 * t;
+        const uint32_t stage = smem_u32(sP) + (r >> 6) * L::P_ATOM + t * 128 * 128 + (r & 63) * 2;
+        const float* inv_l = sL + t * 128;
+#pragma unroll
+        for (int cb = 0; cb < 128; cb += 64) {
+          uint32_t ov[64];
+          tmem_ld64_sync(tOT + cb, ov);
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            st_shared_u16(stage + (cb + i) * 128, __half_as_ushort(__float2half_rn(__uint_as_float(ov[i]) * inv_l[cb + i])));
+        }
+        fence_proxy_async_shared();
+      }
+      group_sync(1 + t);  // the whole tile staged
+      if (r == 0 && !*abort_flag) {
+        const int y = q_tile * L::BM;  // rows past N are clipped by the tensor map
+        tma_store_3d(&tm_o, sP + t * 128 * 128, 0, y, bh);
+        tma_store_3d(&tm_o, sP + L::P_ATOM + t * 128 * 128, 64, y, bh);
+        bulk_commit_and_wait_read();
       }
     }
   } else {
     reg_dealloc<88>();
-    // ============================================================ correction and epilogue
-    const int quad = warp & 3;
-    const int d = quad * 32 + lane;  // TMEM lane of O^T
+    // ============================================================ correction
+    const int quad = warp & 3;  // TMEM lanes (head dimensions) 32 quad .. 32 quad + 31 of O^T
     const uint32_t tOT = tmem + (static_cast<uint32_t>(quad * 32) << 16) + 256;
     bool ok = true;
     for (int j = 1; ok && j < n_kv; ++j) {
@@ -587,39 +613,16 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive(bar_corr + t);
       }
     }
-    // epilogue per tile: O[q][d] = O^T[d][q] / l_q -> fp16, staged in the tile's own P~ rows
-    // (two [128 q][64 d] pieces, d = lane's head dimension), then TMA-stored
-    int epi_phase = 0;
-    for (int t = 0; ok && t < n_tiles; ++t) {
-      if (!wait_warp(bar_o_done + t, (n_iter[t] - 1) & 1) || !wait_warp(bar_l + t, 0)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t stage = smem_u32(sP) + (d >> 6) * L::P_ATOM + t * 128 * 128 + (d & 63) * 2;
-      const float* inv_l = sL + t * 128;
-#pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) {
-        uint32_t ov[32];
-        tmem_ld32_sync(tOT + t * 128 + cb, ov);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          st_shared_u16(stage + (cb + i) * 128, __half_as_ushort(__float2half_rn(__uint_as_float(ov[i]) * inv_l[cb + i])));
-      }
-      fence_proxy_async_shared();
-      mbar_arrive(bar_epi);
-      if (!wait_warp(bar_epi, epi_phase & 1)) { ok = false; break; }
-      ++epi_phase;
-      if (d == 0) {
-        const int y = (tile0 + t) * L::BM;  // rows past N are clipped by the tensor map
-        tma_store_3d(&tm_o, sP + t * 128 * 128, 0, y, bh);
-        tma_store_3d(&tm_o, sP + L::P_ATOM + t * 128 * 128, 64, y, bh);
-        bulk_commit_and_wait_read();
-      }
-    }
   }
 
+  // roles diverge inside warps (single-lane producers and stores): the thread-counting barrier
+  // holds the TMEM release until every thread of the CTA is done
   tc_fence_before();
-  __syncthreads();
-  if constexpr (TRACE) {
-    if (trace_row && threadIdx.x == 0) trace_row[1] = clock64();
+  if constexpr (TRACE) {  // also checks that the barrier held every thread
+    const long long t_end = cta_end_checked(arrived, threadIdx.x == 0);
+    if (trace_row && threadIdx.x == 0) trace_row[1] = t_end;
+  } else {
+    cta_sync();
   }
   if (warp == 1) {
     tc_fence_after();

@@ -7,6 +7,26 @@
 // error can never hang the GPU.
 #pragma once
 
+// CTA-wide barrier that counts threads one by one (the non-.aligned form): correct even when a
+// warp reaches it diverged, e.g. right after a block that only lane 0 runs.  __syncthreads()
+// compiles to the .aligned form, which requires every warp to arrive converged.
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
+// Trace builds: the end of a CTA.  Every thread counts itself into *arrived (zeroed at set-up),
+// then the CTA barrier; thread 0 checks that the barrier let it through only once all blockDim.x
+// threads had arrived (else kDevBarrierEarly) and returns the SM clock, read in a loop whose exit
+// depends on the count, so that the read cannot be scheduled ahead of the barrier.
+__device__ __forceinline__ long long cta_end_checked(int* arrived, bool stamp_thread);
+
+// SM clock read for trace stamps.  The "memory" clobber keeps it in program order with the
+// surrounding memory operations and barriers, so a stamp taken after a barrier reads the clock
+// after the barrier.
+__device__ __forceinline__ long long clock_stamp() {
+  long long t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t)::"memory");
+  return t;
+}
+
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -20,6 +40,7 @@ namespace sage {
 enum DeviceError : int {
   kDevOk = 0,
   kDevTimeoutBarrier = 1,
+  kDevBarrierEarly = 2,  // trace builds: a CTA barrier let a thread through before all had arrived
 };
 __device__ int g_device_error = 0;
 
@@ -324,6 +345,21 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t d_fmt, uint32_t a_fmt
                                                   uint32_t N) {
   return (d_fmt << 4) | (a_fmt << 7) | (b_fmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
          ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ long long cta_end_checked(int* arrived, bool stamp_thread) {
+  atomicAdd(arrived, 1);
+  cta_sync();
+  long long t = 0;
+  if (stamp_thread) {
+    int n;
+    do {
+      t = clock_stamp();
+      n = *reinterpret_cast<volatile int*>(arrived);
+    } while (n < 0);
+    if (n != static_cast<int>(blockDim.x)) atomicExch(&g_device_error, kDevBarrierEarly);
+  }
+  return t;
 }
 
 }  // namespace sage

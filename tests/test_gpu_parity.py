@@ -240,8 +240,9 @@ def _exact_rows(qh, kh, vh, rows, w):
     return (e / e.sum(axis=1, keepdims=True)) @ vf
 
 
-def test_traced_kernel_matches_untraced_and_stamps_are_ordered(sa):
-    w = W.Workload("trace_b1h2_n1024_d128", 1, 2, 1024, 128, False, True, n_out=4, out_mag=20.0)
+@pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, True)])
+def test_traced_kernel_matches_untraced_and_stamps_are_ordered(sa, d, causal):
+    w = W.Workload(f"trace_b1h2_n1024_d{d}", 1, 2, 1024, d, causal, True, n_out=4, out_mag=20.0)
     q, k, v = (t.cuda() for t in W.make_qkv(w))
     km, q8, k8, sq, sk = sa.empty_quantized(q, 1)
     sa.sage_smooth_k(k, km)
@@ -249,17 +250,28 @@ def test_traced_kernel_matches_untraced_and_stamps_are_ordered(sa):
     o1, o2 = torch.empty_like(q), torch.empty_like(q)
     sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o1, w.causal, w.sm_scale, 1)
     T = w.N // 128
-    tr = torch.zeros((3, 2 + 10 * T), dtype=torch.int64, device="cuda")
-    sa.sage_debug_attn_trace(q8, k8, sq, sk, v, o2, w.causal, w.sm_scale, 1, tr, 3)
+    ctas = 8  # every CTA of the first head: causal pairs with 8, 6, 4 and 2 key tiles
+    tr = torch.zeros((ctas, 2 + 10 * T), dtype=torch.int64, device="cuda")
+    sa.sage_debug_attn_trace(q8, k8, sq, sk, v, o2, w.causal, w.sm_scale, 1, tr, ctas)
     torch.cuda.synchronize()
+    # 0: no wait timed out, and (2 otherwise) every CTA's final barrier held all its threads
     assert sa.sage_last_device_error() == 0
     assert torch.equal(o1, o2)
     tr = tr.cpu().numpy()
     assert np.all(tr[:, 1] > tr[:, 0])
+    # the end stamp is taken after the CTA's final barrier: every event of the CTA comes before it
+    assert np.all(tr[:, 2:].max(axis=1) <= tr[:, 1])
+    assert np.all(tr[:, 2:][tr[:, 2:] > 0] >= np.repeat(tr[:, :1], tr.shape[1] - 2, axis=1)[tr[:, 2:] > 0])
     for t in range(2):
         s_ready = tr[:, 2 + 3 * t * T: 2 + (3 * t + 1) * T]
         p_sig = tr[:, 2 + (3 * t + 2) * T: 2 + (3 * t + 3) * T]
-        assert np.all(p_sig > s_ready) and np.all(np.diff(s_ready, axis=1) > 0)
+        done = s_ready > 0  # key tiles this query tile processed (all of them when non-causal)
+        assert np.all((p_sig > s_ready)[done])
+        assert np.all(p_sig[~done] == 0)
+        for c in range(ctas):
+            assert np.all(np.diff(s_ready[c][done[c]]) > 0)
+        if not causal:
+            assert done.all()
 
 
 def test_mma_rate_probe_runs(sa):
