@@ -570,9 +570,20 @@ __global__ void __launch_bounds__(512, 1)
         for (int cb = 0; cb < 128; cb += 64) {
           uint32_t ov[64];
           tmem_ld64_sync(tOT + cb, ov);
+          // queries q, q+1 of this head dimension: packed multiply and packed fp16 conversion
+          // (each value rounded once, as a scalar multiply and conversion would), then one
+          // 16-bit store per query row
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            st_shared_u16(stage + (cb + i) * 128, __half_as_ushort(__float2half_rn(__uint_as_float(ov[i]) * inv_l[cb + i])));
+          for (int i = 0; i < 64; i += 4) {
+            const float4 il = *reinterpret_cast<const float4*>(inv_l + cb + i);
+            const float2 a = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(il.x, il.y));
+            const float2 b = __fmul2_rn(make_float2(__uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3])), make_float2(il.z, il.w));
+            const uint32_t ha = pack_half2(a.x, a.y), hb = pack_half2(b.x, b.y);
+            st_shared_u16(stage + (cb + i) * 128, static_cast<uint16_t>(ha));
+            st_shared_u16(stage + (cb + i + 1) * 128, static_cast<uint16_t>(ha >> 16));
+            st_shared_u16(stage + (cb + i + 2) * 128, static_cast<uint16_t>(hb));
+            st_shared_u16(stage + (cb + i + 3) * 128, static_cast<uint16_t>(hb >> 16));
+          }
         }
         fence_proxy_async_shared();
       }
