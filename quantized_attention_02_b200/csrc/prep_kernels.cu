@@ -171,7 +171,7 @@ __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
 //   G  > 1 : the CTA is one group of G tokens held in registers (G/P passes), CTA-wide max.
 //            Groups tile each head separately: ceil(N/G) groups per head, the last one holding
 //            the N mod G remaining tokens when G does not divide N.
-// `blk` is the block's index within its tensor's part of the grid.
+// Body of quant_kernel: `blk` is the CTA's group (per-block) or its block of P rows (per-token).
 template <int D, int G, bool SMOOTH>
 __device__ __forceinline__ void quant_block(const __half* __restrict__ x, const float* __restrict__ km,
                                             int8_t* __restrict__ q, float* __restrict__ scale, int N,
