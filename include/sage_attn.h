@@ -132,6 +132,15 @@ int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, c
 int sage_debug_mma_rate(int mode, int n, int chains, int issuers, int iters, int ctas, long long* cycles,
                         int* status, void* stream);
 
+/* Debug / failure detection: launches one warp that waits on an mbarrier nothing ever arrives
+ * on, with the same bounded wait (about 0.5 s of SM clocks) that every pipeline role of the
+ * attention kernels uses.  The wait gives up, records status 1 for sage_last_device_error()
+ * and the kernel returns: no trap, no fault, the context stays usable.  gave_up: device int,
+ * written 0 when the wait gave up (1 would mean it completed).  Returns SAGE_ERR_INVALID for a
+ * null pointer, SAGE_ERR_CUDA if the launch failed.  (Not an operation of the pages: a check of
+ * the library's own failure detection.) */
+int sage_debug_wait_timeout(int* gave_up, void* stream);
+
 /* Waits for all work on stream, then returns and clears the device status word written by
  * kernels whose bounded waits gave up (0 = none; 1 = an mbarrier wait timed out; 2, from
  * sage_debug_attn_trace only: a CTA barrier let a thread through before every thread had

@@ -59,10 +59,12 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_noalloc_scratch_bytes.restype = _sz
         lib.sage_debug_attn_trace.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _i, _p]
         lib.sage_debug_mma_rate.argtypes = [_i, _i, _i, _i, _i, _i, _p, _p, _p]
+        lib.sage_debug_wait_timeout.argtypes = [_p, _p]
         lib.sage_attn_fwd_host.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p]
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
-                  "sage_debug_attn_trace", "sage_debug_mma_rate", "sage_attn_fwd_host"):
+                  "sage_debug_attn_trace", "sage_debug_mma_rate", "sage_attn_fwd_host",
+                  "sage_debug_wait_timeout"):
             getattr(lib, n).restype = _i
         _lib = lib
     return _lib
@@ -230,6 +232,12 @@ def sage_noalloc_scratch_bytes(B: int, H: int, N: int, d: int, granularity: int)
 
 def sage_last_device_error(stream=None) -> int:
     return int(get_lib().sage_last_device_error(_stream(stream)))
+
+
+def sage_debug_wait_timeout(gave_up: torch.Tensor, stream=None) -> None:
+    """One warp waits, with the pipelines' bounded wait, on an mbarrier that nothing arrives on;
+    gave_up (int32 [1], CUDA) receives 0 when the wait gave up."""
+    _check(get_lib().sage_debug_wait_timeout(_ptr(gave_up), _stream(stream)), "sage_debug_wait_timeout")
 
 
 # ------------------------------------------------------------------ conveniences

@@ -789,6 +789,29 @@ cudaError_t launch_qk_debug(const CUtensorMap& tq, const CUtensorMap& tk, int32_
   return D == 128 ? launch_qk_debug_d<128>(tq, tk, s, BH, N, st) : launch_qk_debug_d<64>(tq, tk, s, BH, N, st);
 }
 
+// Failure detection check: one warp initialises an mbarrier that nothing ever arrives on and
+// waits on its first phase with the bounded wait every pipeline role uses.  The wait gives up
+// after kWaitLimitCycles, records kDevTimeoutBarrier in the status word and the kernel returns
+// normally, so the context stays usable.  out[0] = 1 if the wait completed (it cannot), 0 if
+// it gave up.
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(int* __restrict__ out) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar, 0, &abort_flag);
+  if (threadIdx.x == 0) out[0] = ok ? 1 : 0;
+}
+
+cudaError_t launch_wait_timeout(int* out, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 32, 0, st>>>(out);
+  return cudaGetLastError();
+}
+
 int read_and_clear_device_error(cudaStream_t st, cudaError_t* err) {
   *err = cudaStreamSynchronize(st);
   if (*err != cudaSuccess) return -1;

@@ -25,6 +25,8 @@ struct AttnArgs {
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_qk_debug(const CUtensorMap& tq, const CUtensorMap& tk, int32_t* s, int BH, int N, int D,
                             cudaStream_t st);
+// One warp waits on an mbarrier that nothing arrives on, with the pipelines' bounded wait.
+cudaError_t launch_wait_timeout(int* out, cudaStream_t st);
 // Synchronizes st, returns the device status word (and clears it); -1 if a CUDA call failed.
 int read_and_clear_device_error(cudaStream_t st, cudaError_t* err);
 

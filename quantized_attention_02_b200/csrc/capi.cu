@@ -289,6 +289,11 @@ int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, c
                              static_cast<cudaStream_t>(stream), trace, trace_ctas);
 }
 
+int sage_debug_wait_timeout(int* gave_up, void* stream) {
+  if (!gave_up) return SAGE_ERR_INVALID;
+  return cuda_status(sage::launch_wait_timeout(gave_up, static_cast<cudaStream_t>(stream)));
+}
+
 int sage_last_device_error(void* stream) {
   cudaError_t e;
   const int code = sage::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);

@@ -91,6 +91,7 @@ def test_null_pointers_and_bad_scalars(sa):
     misaligned = ctypes.c_void_p(0x1008)
     assert L.sage_smooth_k(misaligned, FAKE, 1, 1, 128, 64, s) == -1
     assert L.sage_debug_qk_int32(FAKE, FAKE, None, 1, 1, 128, 64, s) == -1
+    assert L.sage_debug_wait_timeout(None, s) == -1
 
 
 def test_host_pipeline_validation(sa):
