@@ -85,7 +85,11 @@ PROFILE = Workload("profile_b1h16_n16384_d128", 1, 16, 16384, 128, False, True, 
 # the video-DiT shape with a sixth of its heads: small enough for a full profiler capture
 PROFILE64 = Workload("profile_b1h16_n16384_d64", 1, 16, 16384, 64, False, True, bias_std=4.0)
 
-ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64)}
+# the headline sweep point with per-token scales (one per query / key token) instead of per-block
+TOKEN128 = Workload("token_n16384_d128_full", 1, 64, 16384, 128, False, False, n_out=4, out_mag=20.0)
+TOKEN64 = Workload("token_n16384_d64_full", 1, 64, 16384, 64, False, False, n_out=4, out_mag=20.0)
+
+ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
