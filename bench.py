@@ -145,10 +145,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_sample(w: W.Workload, budget_s: float = 12.0):
+def oracle_sample(w: W.Workload, budget_s: float = 12.0, keep: bool = False):
     """Time the CPU oracle (smooth K, quantize, attention) on a bounded sample of the
     workload: one head, R query rows; the rate is scaled to TOPS by the rows' share of
-    the attention work.  Returns (tops, cores, description)."""
+    the attention work.  Returns (tops, cores, description), plus (q, k, v, rows, o_rows)
+    of the sample when keep is set."""
     import numpy as np
 
     import oracle
@@ -169,7 +170,7 @@ def oracle_sample(w: W.Workload, budget_s: float = 12.0):
     n = int(min(w.N, max(rows.size, rows.size * max(1.0, (budget_s - t_prep) / max(t_probe, 1e-3)))))
     rows = np.sort(rng.choice(w.N, size=n, replace=False)).astype(np.int64)
     t2 = time.perf_counter()
-    oracle.attn_rows(q8[0, 0], k8[0, 0], sq[0, 0], sk[0, 0], v[0, 0], rows, w.causal, w.sm_scale, (gq, gk))
+    o_rows, _ = oracle.attn_rows(q8[0, 0], k8[0, 0], sq[0, 0], sk[0, 0], v[0, 0], rows, w.causal, w.sm_scale, (gq, gk))
     t_rows = time.perf_counter() - t2
     # attention ops of the sampled rows (causal rows see i+1 keys)
     keys = (rows + 1).sum() if w.causal else rows.size * w.N
@@ -179,7 +180,43 @@ def oracle_sample(w: W.Workload, budget_s: float = 12.0):
     t = t_rows + t_prep * (ops / head_ops)
     desc = (f"oracle (plain C, OpenMP) on 1 head of {w.name}: smooth+quantize the head, then attention for "
             f"{rows.size} of {w.N} query rows; {t:.1f} s")
+    if keep:
+        return ops / t / 1e12, cores, desc, (q, k, v, rows, o_rows)
     return ops / t / 1e12, cores, desc
+
+
+def sample_accuracy(sa, w: W.Workload, sample, dev) -> dict:
+    """The GPU forward pass on the oracle sample's head (outside the timed region), compared on
+    the sampled rows with the oracle's rows and, on up to 256 of them, with unquantized fp64
+    attention.  Never raises: a failure is reported in the returned object."""
+    try:
+        import numpy as np
+        q, k, v, rows, o_ref = sample
+        gran = sa.SAGE_PER_BLOCK if w.per_block else sa.SAGE_PER_TOKEN
+        o = sa.sageattn(q.to(dev), k.to(dev), v.to(dev), w.causal, w.sm_scale, gran)
+        if dev.type == "cuda":
+            torch.cuda.synchronize(dev)
+        og = o[0, 0].float().cpu().numpy().astype(np.float64)[rows]
+        o_ref = np.asarray(o_ref, dtype=np.float64)
+
+        def cos(a, b):
+            return float(np.dot(a.ravel(), b.ravel()) / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+        sub = np.linspace(0, rows.size - 1, min(rows.size, 256)).astype(np.int64)
+        qf = q[0, 0].double().numpy()[rows[sub]]
+        kf, vf = k[0, 0].double().numpy(), v[0, 0].double().numpy()
+        s = (qf @ kf.T) * w.sm_scale
+        if w.causal:
+            s = np.where(np.arange(w.N)[None, :] <= rows[sub][:, None], s, -np.inf)
+        s -= s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        exact = (e / e.sum(axis=1, keepdims=True)) @ vf
+        return {"rows": int(rows.size), "max_abs_err_over_max_v": round(float(np.abs(og - o_ref).max()) / float(v.abs().max()), 7),
+                "cos_vs_oracle": round(cos(og, o_ref), 8), "cos_vs_fp64_exact": round(cos(og[sub], exact), 6),
+                "bar": "max_abs_err_over_max_v <= 2e-3 and cos_vs_oracle >= 0.9999 (cos_vs_fp64_exact >= 0.995 on K-outlier inputs)",
+                "sample": "the cpu_baseline sample's head, GPU output of the same call path"}
+    except Exception as exc:  # noqa: BLE001  (reported, never fatal to the bench line)
+        return {"error": f"{type(exc).__name__}: {exc}"}
 
 
 # ------------------------------------------------------------------ multi-rank helpers
@@ -321,7 +358,12 @@ def run_ours(args, w: W.Workload):
         peak = mixed_peak_tops(p_sus)
         achieved = ops / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
-        cpu_tops, cores, desc = (None, None, "skipped") if args.no_cpu_baseline else oracle_sample(w)
+        accuracy = None
+        if args.no_cpu_baseline:
+            cpu_tops, cores, desc = None, None, "skipped"
+        else:
+            cpu_tops, cores, desc, sample = oracle_sample(w, keep=True)
+            accuracy = sample_accuracy(sa, w, sample, dev)
         elem_bytes = w.BH * w.N * w.d * 2
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -344,6 +386,7 @@ def run_ours(args, w: W.Workload):
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
+            "accuracy": accuracy,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks.summary(),
         }

@@ -5,6 +5,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>  // header-only NVTX3: ranges cost a pointer check unless a profiler is attached
+
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -254,9 +256,16 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   float* sq = reinterpret_cast<float*>(w + off_sq);
   float* sk = reinterpret_cast<float*>(w + off_sk);
   float* km = reinterpret_cast<float*>(w + off_km);
+  // NVTX ranges mark the host-side enqueue of each step in a profiler's timeline
+  nvtxRangePushA("sage_smooth_k");
   rc = cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, BH, N, d, st));
+  nvtxRangePop();
+  nvtxRangePushA("sage_quant_qk");
   if (!rc) rc = sage_quant_qk(q, k, km, q8, k8, sq, sk, B, H, N, d, granularity, stream);
+  nvtxRangePop();
+  nvtxRangePushA("sage_attn_fused");
   if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity, st);
+  nvtxRangePop();
   const cudaError_t fe = cudaFreeAsync(ws, st);
   if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
   return rc;
