@@ -83,10 +83,11 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
 //   0   TMA producer: Q tiles once, then V tiles through their ring
 //   1 / 3  MMA warps: O^T_t += V^T . P~_t^T for query tile 0 / 1 (warp 1 also allocates TMEM)
 //   2   MMA warp: S_t = Q_t . K^T for both query tiles; also loads the K ring (TMA)
-//   4-7 / 8-11  softmax of query tile 0 / 1 (thread = query row = TMEM lane of S)
-//   12-15       correction and epilogue (thread = head dimension d = TMEM lane of O^T):
-//               rescales the O^T columns of rows whose offset moved, then normalizes by 1/l,
-//               stages O in shared memory and TMA-stores it.
+//   4-7 / 8-11  softmax of query tile 0 / 1 (thread = query row = TMEM lane of S), then that
+//               tile's epilogue (thread = head dimension = TMEM lane of O^T): normalizes by 1/l,
+//               stages O in shared memory and TMA-stores it, both tiles in parallel
+//   12-15       correction (thread = head dimension d = TMEM lane of O^T): rescales the O^T
+//               columns of rows whose offset moved, between two P.V products
 template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED>
 __global__ void __launch_bounds__(512, 1)
     sage_attn_v3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
