@@ -359,8 +359,8 @@ def run_ours(args, w: W.Workload):
         achieved = ops / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
         accuracy = None
-        if args.no_cpu_baseline:
-            cpu_tops, cores, desc = None, None, "skipped"
+        if args.no_cpu_baseline or world > 1:  # the CPU baseline belongs to the N=1 line only
+            cpu_tops, cores, desc = None, None, ("skipped" if world == 1 else "rank 0 at N=1 only")
         else:
             cpu_tops, cores, desc, sample = oracle_sample(w, keep=True)
             accuracy = sample_accuracy(sa, w, sample, dev)
