@@ -113,3 +113,32 @@ def test_binding_rejects_cpu_tensors(sa):
     q = torch.zeros(1, 1, 128, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         sa.sageattn(q, q, q)
+
+
+def _declared_arity():
+    """Parameter count of every function declared in include/sage_attn.h (comments stripped)."""
+    import re
+    from pathlib import Path
+    root = Path(__file__).resolve().parents[1]
+    text = (root / "include" / "sage_attn.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for m in re.finditer(r"\b(sage_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header(sa):
+    """Every function the binding declares ctypes argument types for takes exactly as many
+    arguments as its declaration in the header."""
+    arity = _declared_arity()
+    lib = sa.get_lib()
+    checked = 0
+    for name, n in arity.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is not None:
+            assert len(argtypes) == n, (name, len(argtypes), n)
+            checked += 1
+    assert checked >= 12
