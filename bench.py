@@ -413,8 +413,10 @@ def run_reference(args, w: W.Workload):
     if rank != 0:
         return None
     samples = []
+    # each step a bounded sample; the whole run stays near two and a half minutes
+    budget = min(4.0, max(0.5, 150.0 / (args.warmup + args.steps)))
     for i in range(args.warmup + args.steps):
-        tops, cores, desc = oracle_sample(w, budget_s=4.0)
+        tops, cores, desc = oracle_sample(w, budget_s=budget)
         if i >= args.warmup:
             samples.append(tops)
     value = statistics.median(samples)
