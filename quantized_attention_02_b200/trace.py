@@ -11,6 +11,8 @@ where a softmax warpgroup spends its cycles:
   mma_wait  P~ signalled -> next S ready      (P.V + next Q.K^T on the tensor core, plus
                                                the signalling latency both ways)
   period    S ready -> next S ready           (one key tile for one query tile)
+  prologue  CTA start -> first S ready       (set-up, first loads, first Q.K^T)
+  epilogue  last event -> CTA end            (last P.V, normalisation and store, final barrier)
 
 and the kernel-wide rate: cycles per (query tile x key tile) per SM.
 """
@@ -75,6 +77,14 @@ def summarize(tr: np.ndarray, T: int, causal: bool) -> dict:
     out["p1_minus_p0"] = float(np.median((p1 - p0)[both])) if both.any() else None
     dur = tr[:, 1] - tr[:, 0]
     n_tiles = 2 * (T if not causal else (T + 1) // 2)
+    # per CTA: start -> first S ready (set-up, first loads, first Q.K^T) and last recorded event
+    # -> end (last P.V, epilogue, final barrier); the end stamp is taken after the CTA barrier
+    big = np.iinfo(np.int64).max
+    s0, s1 = ev(0, 0)[:, 0], ev(1, 0)[:, 0]
+    first_s = np.minimum(np.where(s0 > 0, s0, big), np.where(s1 > 0, s1, big))
+    last = np.where(tr[:, 2:] > 0, tr[:, 2:], 0).max(axis=1)
+    out["prologue"] = float(np.median(first_s - tr[:, 0]))
+    out["epilogue"] = float(np.median(tr[:, 1] - last))
     out["cta_cycles"] = float(np.median(dur))
     out["cycles_per_tile_pair"] = float(np.median(dur)) / max(1, (T if not causal else T // 2))
     out["note"] = "cycles are SM clocks; 'cycles_per_tile_pair' = CTA cycles / key tiles (2 query tiles each)"
