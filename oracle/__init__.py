@@ -14,12 +14,19 @@ ideas.
 Parity status (which functions are pinned by checks other than themselves):
   smooth_k ........ pinned (exact fp64 mean for power-of-two N; shift of K by a
                     constant; numpy mean within 1 ulp)
-  quant ........... pinned (integer grid identity, round-trip bound, +-127 at the
-                    absmax, all-zero group, numpy-free brute force on tiny cases)
+  quant ........... pinned (scale fl32(a/127) and inverse fl32(127/a) against exact
+                    rationals over every positive fp16 absmax; codes = rne(fl32(x*inv));
+                    integer grid identity, round-trip bound, +-127 at the absmax,
+                    all-zero group)
   qk_int .......... pinned (brute-force Python loops; int64 numpy matmul)
-  attn ............ pinned (identity-quantizer special case vs exact fp64
-                    attention within the fp16 error bound; causal row 0 equals
-                    V[0]; causal rows ignore later keys; rows of P sum to 1)
+  attn ............ pinned (P~ rounded once fp64 -> fp16: hand-derived two-key
+                    case next to an fp16 midpoint in tests/golden; identity-quantizer
+                    special case vs exact fp64 attention within the fp16 error bound;
+                    causal row 0 equals V[0]; causal rows ignore later keys; rows of P
+                    sum to 1)
+Every pin is itself checked by tests/test_oracle_mutations.py: twenty planted slips
+(dropped or re-routed roundings, signs, indices, group sizes, operands), each of which
+makes the pins fail.
   attn_fp64 ....... pinned (softmax shift invariance; hand-derived closed forms
                     in tests/golden)
 """
@@ -59,7 +66,9 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # SAGE_ORACLE_LIB: a deliberately broken build of this file, loaded by the
+            # mutation tests (tests/test_oracle_mutations.py) to show that the pins fail on it
+            lib = ctypes.CDLL(os.environ.get("SAGE_ORACLE_LIB") or build())
             i64, i32, f64, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
             lib.oracle_smooth_k.argtypes = [vp, i64, i64, i64, vp]
             lib.oracle_quant.argtypes = [vp, vp, i64, i64, i64, i64, vp, vp]
@@ -72,6 +81,8 @@ def _load():
             lib.oracle_attn_fp64.argtypes = [vp, vp, vp, i64, i64, i64, i32, f64, vp]
             lib.oracle_round_fp16.argtypes = [vp, i64, vp]
             lib.oracle_round_fp16.restype = None
+            lib.oracle_quant_scale.argtypes = [vp, i64, vp, vp]
+            lib.oracle_quant_scale.restype = None
             for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_qk_int_rows", "oracle_attn",
                          "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
                 getattr(lib, name).restype = i32
@@ -122,6 +133,16 @@ def smooth_k(k) -> np.ndarray:
 
 def scale_count(N: int, g: int) -> int:
     return (N + g - 1) // g
+
+
+def quant_scale(a) -> tuple[np.ndarray, np.ndarray]:
+    """(scale, inverse) = (fl32(a/127), fl32(127/a)) for group absmax values a (fp32);
+    both 0 where a = 0.  The two roundings the INT8 reading fixes (Summary bullet 1)."""
+    a = np.ascontiguousarray(a, np.float32)
+    s = np.empty_like(a)
+    inv = np.empty_like(a)
+    _load().oracle_quant_scale(_ptr(a), a.size, _ptr(s), _ptr(inv))
+    return s, inv
 
 
 def quant(x, g: int, mu=None):

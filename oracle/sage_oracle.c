@@ -90,6 +90,21 @@ int oracle_smooth_k(const uint16_t* k, int64_t BH, int64_t N, int64_t d, float* 
  *     inv = fl32(127 / a)                    (a = 0: s = inv = 0, all codes 0)
  *     q   = clamp(round_half_even(fl32(x * inv)), -127, 127)
  * ------------------------------------------------------------------------- */
+static void quant_scale(float a, float* s, float* inv) {
+    *s = 0.0f;
+    *inv = 0.0f;
+    if (a > 0.0f) {
+        *s = a / 127.0f;   /* one fp32 division: the correctly rounded a/127 */
+        *inv = 127.0f / a; /* one fp32 division: the correctly rounded 127/a */
+    }
+}
+
+/* The scale and inverse of groups with the given absmax values a[i] (exported so
+ * that the tests can pin the two roundings against exact rational arithmetic). */
+void oracle_quant_scale(const float* a, int64_t n, float* s, float* inv) {
+    for (int64_t i = 0; i < n; ++i) quant_scale(a[i], s + i, inv + i);
+}
+
 int oracle_quant(const uint16_t* x16, const float* mu, int64_t BH, int64_t N, int64_t d,
                  int64_t g, int8_t* q, float* scale) {
     if (!x16 || !q || !scale || BH < 0 || N <= 0 || d <= 0 || g <= 0) return ORACLE_ERR_ARG;
@@ -108,11 +123,8 @@ int oracle_quant(const uint16_t* x16, const float* mu, int64_t BH, int64_t N, in
                     if (ax > a) a = ax;
                 }
             }
-            float s = 0.0f, inv = 0.0f;
-            if (a > 0.0f) {
-                s = a / 127.0f;
-                inv = 127.0f / a;
-            }
+            float s, inv;
+            quant_scale(a, &s, &inv);
             scale[bh * ngroups + gi] = s;
             for (int64_t t = t0; t < t1; ++t) {
                 for (int64_t c = 0; c < d; ++c) {

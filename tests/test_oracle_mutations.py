@@ -1,0 +1,88 @@
+"""Mutation tests of the oracle's pins.
+
+Each case plants one plausible slip in a copy of oracle/sage_oracle.c (a dropped
+rounding, a rounding taken another way, a wrong sign, index, group size or
+operand), builds the copy with the oracle's own compiler flags, and runs
+tests/test_oracle_pins.py against it in a fresh process (the oracle package loads
+the library named by SAGE_ORACLE_LIB).  The pins must fail on every mutant, and
+pass on an unmodified copy built the same way (the control case), so a pin that
+cannot tell a slip from the reading it pins shows up here.
+
+The readings pinned are those of the SageAttention summary page (Summary bullets
+1-2: INT8 Q.K^T after smoothing K, P.V in fp16; idea I1: the K shift).
+"""
+import concurrent.futures
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "sage_oracle.c")
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+
+# (name, text in sage_oracle.c, replacement, expected number of occurrences)
+MUTATIONS = [
+    ("p_unrounded", "const double pt = h2d(d2h(e));", "const double pt = e;", 1),
+    ("p_rounded_via_fp32", "const double pt = h2d(d2h(e));", "const double pt = h2d(d2h((double)(float)e));", 1),
+    ("row_sum_of_rounded_p", "l += e;\n        const double pt = h2d(d2h(e));",
+     "const double pt = h2d(d2h(e));\n        l += pt;", 1),
+    ("scale_by_reciprocal", "*s = a / 127.0f;", "*s = a * (1.0f / 127.0f);", 1),
+    ("inverse_of_scale", "*inv = 127.0f / a;", "*inv = 1.0f / (a / 127.0f);", 1),
+    ("codes_ties_away", "float r = nearbyintf(y);", "float r = roundf(y);", 1),
+    ("codes_truncated", "float r = nearbyintf(y);", "float r = truncf(y);", 1),
+    ("smoothing_sign", "if (mu) x = x - mu[bh * d + c];", "if (mu) x = x + mu[bh * d + c];", 2),
+    ("k_mean_over_n_minus_1", "float mean32 = sum32 / (float)N;", "float mean32 = sum32 / (float)(N - 1);", 1),
+    ("k_mean_fp32_accumulator", "int64_t s = 0;", "float s = 0;", 1),
+    ("causal_off_by_one", "causal ? i + 1 : N;\n    const int8_t* qi", "causal ? i : N;\n    const int8_t* qi", 1),
+    ("sm_scale_dropped", "s[j] = (double)dot * sqi * (double)skh[j / gk] * sm_scale;",
+     "s[j] = (double)dot * sqi * (double)skh[j / gk];", 1),
+    ("key_scale_group_of_q", "(double)skh[j / gk]", "(double)skh[j / gq]", 1),
+    ("query_scale_per_key", "const double sqi = (double)sqh[i / gq];", "const double sqi = (double)sqh[0];", 1),
+    ("no_max_subtraction", "const double e = exp(s[j] - m);", "const double e = exp(s[j]);", 1),
+    ("qk_uses_q_twice", "const int8_t* kj = k8 + (bh * N + j) * d;", "const int8_t* kj = q8 + (bh * N + j) * d;", 1),
+    ("qk_int_transposed", "S[(bh * N + i) * N + j] = acc;", "S[(bh * N + j) * N + i] = acc;", 1),
+    ("output_via_fp32", "if (o16) o16[i * d + c] = d2h(o);", "if (o16) o16[i * d + c] = d2h((double)(float)o);", 1),
+    ("fp64_attention_no_scale", "s[j] = dot * sm_scale;", "s[j] = dot;", 1),
+    ("fp64_attention_causal_off_by_one", "const int64_t jend = causal ? i + 1 : N;\n                    double m",
+     "const int64_t jend = causal ? i + 2 : N;\n                    double m", 1),
+]
+
+CFLAGS = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
+
+
+def _build_and_run_pins(name, old, new, count, tmpdir):
+    src = open(SRC).read()
+    if old:  # the control case builds the unmodified text
+        assert src.count(old) == count, f"{name}: expected {count} occurrence(s) of the mutated text"
+    mutated = src.replace(old, new) if old else src
+    c_path = os.path.join(tmpdir, f"{name}.c")
+    so_path = os.path.join(tmpdir, f"lib_{name}.so")
+    with open(c_path, "w") as f:
+        f.write(mutated)
+    subprocess.run(CFLAGS + ["-o", so_path, c_path, "-lm"], check=True, capture_output=True)
+    env = dict(os.environ, SAGE_ORACLE_LIB=so_path, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", PINS, "-x", "-q", "-p", "no:cacheprovider"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode, r.stdout[-2000:] + r.stderr[-2000:]
+
+
+def test_pins_fail_on_every_mutant_and_pass_on_the_control(tmp_path):
+    jobs = [("control", "", "", 0)] + MUTATIONS
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(2, min(8, os.cpu_count() or 2))) as ex:
+        futs = {name: ex.submit(_build_and_run_pins, name, old, new, cnt, str(tmp_path))
+                for name, old, new, cnt in jobs}
+        results = {name: f.result() for name, f in futs.items()}
+    rc, out = results.pop("control")
+    assert rc == 0, f"the unmodified oracle must pass its pins:\n{out}"
+    survivors = {name: out for name, (rc, out) in results.items() if rc != 1}
+    # pytest exits 1 when a test failed; anything else (0 = all passed, a crash) is a survivor
+    assert not survivors, "mutants the pins did not catch: " + ", ".join(
+        f"{n} (exit {results[n][0]})" for n in survivors)
+
+
+@pytest.mark.parametrize("name,old,new,count", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_mutation_targets_exist(name, old, new, count):
+    # the planted slips refer to the oracle's current text (a refactor must update them)
+    assert open(SRC).read().count(old) == count

@@ -7,9 +7,9 @@ component shared by all tokens of K leaves the softmax unchanged), a special
 case that reduces to textbook attention / exact integer arithmetic, an error
 bound, or brute force on tiny inputs.  Each is chosen so that a plausible slip
 in the oracle (dropped term, wrong sign, swapped index, transposed operand,
-wrong group boundary, wrong rounding) fails at least one test; the mutation
-tests at the end plant such slips in a copy of the oracle and check that the
-pins catch them.
+wrong group boundary, wrong rounding) fails at least one test;
+tests/test_oracle_mutations.py plants such slips in copies of the oracle and
+checks that this file fails on every one of them.
 """
 import math
 from fractions import Fraction
@@ -130,6 +130,45 @@ def test_quant_group_properties(g):
             # of magnitude <= 127, i.e. below 2^-15 of a step)
             err = np.abs(xf[h, blk] - qs * float(s[h, gi]))
             assert err.max() <= float(s[h, gi]) * (0.5 + 2**-15)
+
+
+def test_quant_scale_and_inverse_are_single_fp32_roundings():
+    # The reading of "quantized to INT8" (Summary bullet 1): s = fl32(a / 127) and
+    # inv = fl32(127 / a), each ONE correctly rounded fp32 division.  Checked against exact
+    # rational arithmetic over every positive finite fp16 absmax (Q groups) and a spread of
+    # fp32 absmax values (smoothed K groups); the set includes values where the tempting
+    # shortcuts a * fl32(1/127) and 1 / fl32(a / 127) round differently, so they would fail.
+    a16 = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    a32 = (np.exp(RNG.uniform(-20, 12, 3000)) * RNG.uniform(1, 2, 3000)).astype(np.float32)
+    a = np.concatenate([a16, a32, np.array([0.0], np.float32)])
+    s, inv = oracle.quant_scale(a)
+    assert s[-1] == 0 and inv[-1] == 0
+    a, s, inv = a[:-1], s[:-1], inv[:-1]
+    with np.errstate(over="ignore"):
+        shortcut_s = a * np.float32(1 / 127)
+        shortcut_inv = np.float32(1) / (a / np.float32(127))
+    assert np.count_nonzero(shortcut_s != s) > 100 and np.count_nonzero(shortcut_inv != inv) > 100
+    for ai, si, ii in zip(a.tolist(), s.tolist(), inv.tolist()):
+        fa = Fraction(ai)
+        assert np.float32(si) == round_to_f32_exact(fa / 127), ai
+        assert np.float32(ii) == round_to_f32_exact(Fraction(127) / fa), ai
+
+
+@pytest.mark.parametrize("g", [1, 64])
+def test_quant_codes_are_rounded_products_with_the_inverse(g):
+    # code = round_half_even(fl32(x * inv)) with inv the group's fl32(127 / a)
+    BH, N, d = 2, 192, 16
+    x = fp16(RNG.standard_normal((BH, N, d)) * 3)
+    q, s = oracle.quant(x, g)
+    xf = x.astype(np.float32)
+    for h in range(BH):
+        for gi in range(s.shape[1]):
+            blk = slice(gi * g, min(N, (gi + 1) * g))
+            a = np.abs(xf[h, blk]).max()
+            s_ref, inv = oracle.quant_scale(np.array([a], np.float32))
+            assert s[h, gi] == s_ref[0]
+            y = xf[h, blk] * inv[0]  # fp32 product, rounded once
+            np.testing.assert_array_equal(q[h, blk], np.rint(y).astype(np.int8))
 
 
 def test_quant_integer_grid_is_identity_and_rounds_half_to_even():
@@ -316,6 +355,35 @@ def test_attn_fp64_matches_textbook_and_is_shift_invariant():
             ref = exact_attention(q[h].astype(np.float64), k[h].astype(np.float64),
                                   v[h].astype(np.float64), causal, 0.25)
             assert np.abs(o[h] - ref).max() < 1e-12
+
+
+def test_p_tilde_is_rounded_once_to_fp16():
+    # Summary bullet 2: P.V runs on 16-bit floating-point operands, so the unnormalized
+    # probabilities are rounded to fp16 -- once, from the exact value (no detour via fp32), and
+    # the row sum uses the unrounded weights.  Two keys with scores 0 and -sm_scale: the case
+    # file derives O = (fp16(e) * 1) / (1 + e) by hand, with fp16(e) given as a multiple of
+    # 2^-12; 'tie_plus' sits 2^-40 above an fp16 midpoint, so an unrounded weight or a rounding
+    # via fp32 lands on a different value.
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "p_rounding_two_keys.json")
+    with open(path) as f:
+        cases = json.load(f)["cases"]
+    q8 = np.array([[[1], [1]]], np.int8)
+    k8 = np.array([[[0], [-1]]], np.int8)
+    ones = np.ones((1, 2), np.float32)
+    v = fp16(np.array([[[0.0], [1.0]]]))
+    for c in cases:
+        e_target = c["e_target"][0] / c["e_target"][1]  # exact rational, to the nearest fp64
+        sm_scale = -math.log(e_target)
+        e = math.exp(-sm_scale)  # the weight the oracle computes, exp(s1 - m) with m = s0 = 0
+        expect = (c["fp16_e_times_4096"] / 4096) / (1 + e)
+        o64, o16 = oracle.attn(q8, k8, ones, ones, v, False, sm_scale)
+        for i in range(2):
+            assert abs(o64[0, i, 0] - expect) <= 1e-16, (c["name"], o64[0, i, 0], expect)
+        if c["fp32_detour_times_4096"] != c["fp16_e_times_4096"]:
+            detour = (c["fp32_detour_times_4096"] / 4096) / (1 + e)
+            assert abs(expect - detour) > 1e-5 and abs(expect - e / (1 + e)) > 1e-5
 
 
 def test_closed_form_two_keys():
