@@ -13,6 +13,7 @@
 // address with cudaGetSymbolAddress, with that device current, and caches it.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -64,12 +65,13 @@ size_t sage_noalloc_scratch_bytes(int B, int H, int N, int d, int granularity) {
 
 int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                           int causal, float sm_scale, int granularity, void* stream) {
+  // the checks of sage_attn_fwd, in its order (same status for the same arguments)
   if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SAGE_ERR_INVALID;
-  if (granularity != SAGE_PER_TOKEN && granularity != SAGE_PER_BLOCK) return SAGE_ERR_INVALID;
-  if (!(sm_scale > 0.f) || sm_scale > 3.4e38f) return SAGE_ERR_INVALID;  // also rejects NaN and inf
   if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N * d >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+  if (!std::isfinite(sm_scale) || !(sm_scale > 0.f)) return SAGE_ERR_INVALID;
+  if (granularity != SAGE_PER_TOKEN && granularity != SAGE_PER_BLOCK) return SAGE_ERR_INVALID;
   for (const void* p : {q, k, static_cast<const void*>(v), static_cast<const void*>(o)})
     if (reinterpret_cast<uintptr_t>(p) & 15u) return SAGE_ERR_INVALID;
   const size_t need = sage_noalloc_scratch_bytes(B, H, N, d, granularity);

@@ -142,3 +142,28 @@ def test_binding_argtypes_match_the_header(sa):
             assert len(argtypes) == n, (name, len(argtypes), n)
             checked += 1
     assert checked >= 12
+
+
+def test_noalloc_validates_like_sage_attn_fwd(sa):
+    # the allocation-free entry point returns the status sage_attn_fwd returns for the same
+    # invalid arguments (both decide before any CUDA call)
+    L = sa.get_lib()
+    s = ctypes.c_void_p(0)
+    mis = ctypes.c_void_p(0x1008)
+    cases = [
+        ((None, FAKE, FAKE, FAKE), (1, 1, 128, 64, 0, 0.1, 1)),
+        ((FAKE,) * 4, (0, 1, 128, 64, 0, 0.1, 1)),
+        ((FAKE,) * 4, (1, 1, 128, 96, 0, 0.1, 1)),
+        ((FAKE,) * 4, (1, 1, 128, 96, 0, 0.1, 7)),          # bad d and granularity: d decides
+        ((FAKE,) * 4, (4096, 4096, 1024, 128, 0, 0.1, 1)),
+        ((FAKE,) * 4, (1, 1, 128, 64, 0, float("inf"), 1)),
+        ((FAKE,) * 4, (1, 1, 128, 64, 0, float("nan"), 1)),
+        ((FAKE,) * 4, (1, 1, 128, 64, 0, -0.5, 1)),
+        ((FAKE,) * 4, (1, 1, 128, 64, 0, 0.0, 1)),
+        ((FAKE,) * 4, (1, 1, 128, 64, 0, 0.1, 3)),
+        ((FAKE, FAKE, mis, FAKE), (1, 1, 128, 64, 0, 0.1, 1)),
+    ]
+    for ptrs, args in cases:
+        a = L.sage_attn_fwd(*ptrs, *args, s)
+        b = L.sage_attn_fwd_noalloc(*ptrs, *args, s)
+        assert a == b and a < 0, (args, a, b)

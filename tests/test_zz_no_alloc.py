@@ -23,9 +23,9 @@ ATOL_FRAC = 2e-3
 COS_MIN = 0.9999
 
 
-def _close(a: torch.Tensor, b: torch.Tensor, vmax: float):
-    a = a.float().cpu().numpy().astype(np.float64).ravel()
-    b = b.float().cpu().numpy().astype(np.float64).ravel()
+def _close(a: np.ndarray, b: np.ndarray, vmax: float):
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
     err = float(np.abs(a - b).max())
     cos = float(np.dot(a, b) / (np.linalg.norm(a) * np.linalg.norm(b)))
     assert err <= ATOL_FRAC * vmax, err
@@ -59,7 +59,14 @@ def test_noalloc_matches_sage_attn_fwd_on_two_calls_in_a_row():
             assert rc == sa.SAGE_OK, sa.sage_status_string(rc)
             torch.cuda.synchronize()
             assert sa.sage_last_device_error() == 0
-            _close(o, o_ref, float(v.abs().max()))
+            # the same kernels on the same inputs: bit-identical to sage_attn_fwd
+            assert torch.equal(o, o_ref), w.name
+            if w.name == "noalloc_b" and seed == 1:
+                # and within the method's bar of the oracle (the second call, on a scratch
+                # array that still holds the first call's codes and scales)
+                import oracle
+                ref = oracle.sage_attn(q.cpu(), k.cpu(), v.cpu(), w.causal, w.sm_scale, per_block=w.per_block)
+                _close(o.float().cpu().numpy(), ref["o64"], float(v.abs().max()))
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
