@@ -603,7 +603,7 @@ __global__ void __launch_bounds__(384, 1)
 #include "attn_v3.cuh"
 
 // ---------------------------------------------------------------- debug: INT32 S = q8 k8^T
-// One CTA per (128-row query tile, head).  Thread 0 issues the TMA loads and the same
+// One CTA per (128-row query tile, head), all along grid x.  Thread 0 issues the TMA loads and the same
 // kind::i8 MMA as the fused kernel; warps 4-7 copy S from TMEM to global memory.
 template <int D>
 __global__ void __launch_bounds__(256, 1)
@@ -624,7 +624,8 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q_tile = blockIdx.x, bh = blockIdx.y;
+  const int n_qt = N / BM;  // grid x = B*H heads x n_qt query tiles (no 65535 cap on heads)
+  const int q_tile = static_cast<int>(blockIdx.x) % n_qt, bh = static_cast<int>(blockIdx.x) / n_qt;
   const int row_base = bh * N;
   const int n_kv = N / BN;
 
@@ -779,7 +780,7 @@ static cudaError_t launch_qk_debug_d(const CUtensorMap& tq, const CUtensorMap& t
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid(N / 128, BH);
+  dim3 grid(static_cast<unsigned>(N / 128) * static_cast<unsigned>(BH));
   kern<<<grid, 256, SMEM, st>>>(tq, tk, s, N);
   return cudaGetLastError();
 }

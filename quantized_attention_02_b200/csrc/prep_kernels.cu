@@ -44,7 +44,7 @@ __device__ __forceinline__ void split_acc(uint32_t word, int& h0, int& h1, float
 }
 
 // One thread-block cluster of C CTAs per head (C = 1, 2, 4 or 8, chosen from N at launch so
-// that every CTA gets at least 2048 tokens).  CTA r of the cluster sums the contiguous
+// that every CTA gets at least 2048 tokens), the clusters side by side along grid x.  CTA r of the cluster sums the contiguous
 // token slice [r*S, min(N, (r+1)*S)), S = ceil(N / C), reading whole rows: a team of T = D/8
 // threads covers one token row with one 16-byte load each (coalesced), a 512-thread CTA covers
 // 512/T rows per pass and keeps four passes of loads in flight.  The per-CTA channel sums
@@ -64,8 +64,8 @@ __global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* 
   constexpr int WARPS = kSmoothThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int n_ctas = static_cast<int>(cluster.num_blocks());  // the cluster spans grid x
-  const int bh = blockIdx.y;
+  const int n_ctas = static_cast<int>(cluster.num_blocks());  // consecutive CTAs of grid x
+  const int bh = static_cast<int>(blockIdx.x) / n_ctas;      // (grid x holds B*H clusters: no 65535 cap)
   const int piece = threadIdx.x % T;       // channels piece*8 .. piece*8+7
   const int row = threadIdx.x / T;
   const int slice = (N + n_ctas - 1) / n_ctas;
@@ -281,7 +281,7 @@ static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cu
   int ctas = 1;  // a power of two, at most kSmoothMaxCtas, with >= kSmoothTokensPerCta tokens per CTA
   while (ctas < kSmoothMaxCtas && N / (2 * ctas) >= kSmoothTokensPerCta) ctas *= 2;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas), static_cast<unsigned>(BH));  // one cluster (grid x) per head
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas) * static_cast<unsigned>(BH));  // one cluster of `ctas` CTAs per head
   cfg.blockDim = dim3(kSmoothThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
