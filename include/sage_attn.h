@@ -118,19 +118,16 @@ int sage_debug_attn_trace(const int8_t* q8, const int8_t* k8, const float* sq, c
                           float sm_scale, int granularity, long long* trace, int trace_ctas,
                           void* stream);
 
-/* Debug: tensor-core issue probe for the MMA shapes of the fused kernel (the loop computes the
- * destination and accumulate flag per instruction; its rate is a lower bound on the tensor rate,
- * not the peak).  Launches
- * `ctas` CTAs (use the SM count; one per SM); in each, `issuers` warps (1 or 2) issue back-to-back
- * MMAs, iters/issuers each (iters a multiple of 4*issuers, <= 2^24), each warp rotating over its
- * own `chains` accumulators, on zero-filled operands; issuer 0 writes the CTA's SM-clock cycles
- * to cycles[cta] (int64 [ctas], device memory).  status (device int, caller-zeroed) is set to 1
- * if a final wait gave up.  Modes: 0 = kind::i8 M128 K32 (both operands in shared memory),
- * 1 = kind::f16 M128 K16 (A in tensor memory, B MN-major in shared memory, n <= 128), 2 =
- * kind::f16 M128 K16 (both in shared memory); n in {64, 128, 256}; chains in {1, 2, 4};
- * issuers*chains*n <= 256.  Multiply-accumulates per MMA: 128*n*K. */
-int sage_debug_mma_rate(int mode, int n, int chains, int issuers, int iters, int ctas, long long* cycles,
-                        int* status, void* stream);
+/* Debug / measurement: the dense tensor-core rate of this GPU per MMA kind, for the roofline's
+ * denominators (not an operation of the pages).  Launches `ctas` CTAs (use the SM count: one per
+ * SM); in each, two warps issue `iters` (a multiple of 8, 8 .. 2^24) back-to-back tcgen05 MMAs of
+ * shape M=128, N=256 with loop-invariant operands (zero-filled shared memory) into their own
+ * accumulators.  kind 0 = kind::i8 (K = 32), 1 = kind::f16 (K = 16), 2 = kind::f8f6f4 with E4M3
+ * operands (K = 32); every instruction is 128*256*K multiply-accumulates.  cycles: int64 [ctas]
+ * device memory, receives each CTA's SM cycles from its first issue to the completion of both
+ * warps' products.  status: device int (caller-zeroed), set to 1 if a bounded wait gave up.
+ * SAGE_ERR_INVALID for a bad kind, iters or pointer; SAGE_ERR_CUDA if the launch failed. */
+int sage_debug_mma_peak(int kind, int iters, int ctas, long long* cycles, int* status, void* stream);
 
 /* Debug / failure detection: launches one warp that waits on an mbarrier nothing ever arrives
  * on, with the same bounded wait (about 0.5 s of SM clocks) that every pipeline role of the

@@ -58,12 +58,12 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_noalloc_scratch_bytes.argtypes = [_i, _i, _i, _i, _i]
         lib.sage_noalloc_scratch_bytes.restype = _sz
         lib.sage_debug_attn_trace.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _i, _p]
-        lib.sage_debug_mma_rate.argtypes = [_i, _i, _i, _i, _i, _i, _p, _p, _p]
+        lib.sage_debug_mma_peak.argtypes = [_i, _i, _i, _p, _p, _p]
         lib.sage_debug_wait_timeout.argtypes = [_p, _p]
         lib.sage_attn_fwd_host.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p]
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
-                  "sage_debug_attn_trace", "sage_debug_mma_rate", "sage_attn_fwd_host",
+                  "sage_debug_attn_trace", "sage_debug_mma_peak", "sage_attn_fwd_host",
                   "sage_debug_wait_timeout"):
             getattr(lib, n).restype = _i
         _lib = lib
@@ -160,32 +160,32 @@ def sage_debug_attn_trace(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float, g
                                            int(trace_ctas), _stream(stream)), "sage_debug_attn_trace")
 
 
-MMA_PROBE_KINDS = {0: ("i8", 32), 1: ("f16 A-from-TMEM", 16), 2: ("f16", 16)}
+MMA_PEAK_KINDS = {0: ("kind::i8", 32), 1: ("kind::f16", 16), 2: ("kind::f8f6f4 e4m3", 32)}
 
 
-def mma_rate(mode: int, n: int = 128, chains: int = 1, issuers: int = 1, iters: int = 20000) -> dict:
-    """Run the tensor-core probe on every SM; return MACs per SM clock and the whole-GPU
-    rate in TOPS (2 ops per multiply-accumulate) timed with CUDA events."""
+def mma_peak(kind: int, iters: int = 4096) -> dict:
+    """Dense tensor-core rate of this GPU for one MMA kind (0 = INT8, 1 = FP16, 2 = FP8 E4M3):
+    one CTA per SM, two warps issuing M=128 N=256 MMAs back to back.  Returns multiply-
+    accumulates per SM clock and the whole-GPU rate in TOPS (2 ops per multiply-accumulate,
+    CUDA events on the current stream, at whatever clock the GPU runs)."""
     dev = torch.cuda.current_device()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     cycles = torch.zeros(sms, dtype=torch.int64, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    kind, K = MMA_PROBE_KINDS[mode]
+    name, K = MMA_PEAK_KINDS[kind]
     st = torch.cuda.current_stream()
     lib = get_lib()
-    _check(lib.sage_debug_mma_rate(mode, n, chains, issuers, 64, sms, _ptr(cycles), _ptr(status), _stream(st)), "mma_rate")
+    _check(lib.sage_debug_mma_peak(kind, 64, sms, _ptr(cycles), _ptr(status), _stream(st)), "mma_peak")  # warm-up
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
-    _check(lib.sage_debug_mma_rate(mode, n, chains, issuers, iters, sms, _ptr(cycles), _ptr(status), _stream(st)),
-           "mma_rate")
+    _check(lib.sage_debug_mma_peak(kind, iters, sms, _ptr(cycles), _ptr(status), _stream(st)), "mma_peak")
     e1.record(st)
     torch.cuda.synchronize()
     if int(status.item()) != 0:
-        raise RuntimeError("mma_rate wait gave up")
-    macs = 128 * n * K * iters
+        raise RuntimeError("mma_peak wait gave up")
+    macs = 2 * iters * 128 * 256 * K  # per CTA: two warps
     cyc = float(cycles.double().median())
-    return {"mode": mode, "kind": kind, "shape": [128, n, K], "chains": chains, "issuers": issuers,
-            "macs_per_clk_per_sm": macs / cyc,
+    return {"kind": name, "shape": [128, 256, K], "macs_per_clk_per_sm": macs / cyc,
             "tops": 2.0 * macs * sms / (e0.elapsed_time(e1) * 1e-3) / 1e12}
 
 
