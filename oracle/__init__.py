@@ -24,7 +24,12 @@ Parity status (which functions are pinned by checks other than themselves):
                     special case vs exact fp64 attention within the fp16 error bound;
                     causal row 0 equals V[0]; causal rows ignore later keys; rows of P
                     sum to 1)
-Every pin is itself checked by tests/test_oracle_mutations.py: twenty planted slips
+  e4m3_encode/decode, quant_v_fp8, attn_fp8pv (FP8 P.V variant, SageAttention2 abstract;
+                    sage_oracle_sa2.c) ... pinned (PyTorch's float8_e4m3fn values and
+                    brute-force nearest search; exact rational scales and mean; hand-
+                    derived two-key cases in tests/golden; the P~-rounding bound against
+                    textbook attention; V-shift invariance; causal row 0)
+Every pin is itself checked by tests/test_oracle_mutations.py: planted slips
 (dropped or re-routed roundings, signs, indices, group sizes, operands), each of which
 makes the pins fail.
   attn_fp64 ....... pinned (softmax shift invariance; hand-derived closed forms
@@ -40,7 +45,7 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "sage_oracle.c")
+_SRCS = [os.path.join(_HERE, f) for f in ("sage_oracle.c", "sage_oracle_sa2.c")]
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "libsage_oracle.so")
 _lock = threading.Lock()
@@ -53,10 +58,10 @@ GROUP_PER_BLOCK = (128, 64)  # (Q tokens, K tokens) per quantization group
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (-O2, no FMA contraction, OpenMP)."""
     os.makedirs(_LIB_DIR, exist_ok=True)
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(s) for s in _SRCS):
         tmp = _LIB + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
-               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, *_SRCS, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -83,6 +88,16 @@ def _load():
             lib.oracle_round_fp16.restype = None
             lib.oracle_quant_scale.argtypes = [vp, i64, vp, vp]
             lib.oracle_quant_scale.restype = None
+            lib.oracle_e4m3_encode_n.argtypes = [vp, i64, vp]
+            lib.oracle_e4m3_encode_n.restype = None
+            lib.oracle_e4m3_decode_n.argtypes = [vp, i64, vp]
+            lib.oracle_e4m3_decode_n.restype = None
+            lib.oracle_quant_v_fp8.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+            lib.oracle_attn_fp8pv.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f64, i64, i64, vp, vp]
+            lib.oracle_attn_fp8pv_rows.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp,
+                                                   i64, vp]
+            for name in ("oracle_quant_v_fp8", "oracle_attn_fp8pv", "oracle_attn_fp8pv_rows"):
+                getattr(lib, name).restype = i32
             for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_qk_int_rows", "oracle_attn",
                          "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
                 getattr(lib, name).restype = i32
@@ -264,6 +279,91 @@ def sage_attn(q, k, v, causal: bool, sm_scale: float, per_block: bool, smooth: b
     k8, sk = quant(k, gk, km)
     o64, o16 = attn(q8, k8, sq, sk, v, causal, sm_scale, (gq, gk))
     return dict(km=km, q8=q8, sq=sq, k8=k8, sk=sk, o64=o64, o16=o16)
+
+
+# ------------------------------------------------------------------ FP8 P.V variant
+# (SageAttention2 abstract: (P~, V) quantized to FP8, V smoothed, P~V in an FP32 buffer;
+# readings in sage_oracle_sa2.c)
+def e4m3_encode(x) -> np.ndarray:
+    """Round to the nearest E4M3 value (ties to even, saturating at +-448): uint8 codes."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e4m3_encode_n(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(b) -> np.ndarray:
+    """Value of E4M3 codes (fp64)."""
+    b = np.ascontiguousarray(b, np.uint8)
+    out = np.empty(b.shape, np.float64)
+    _load().oracle_e4m3_decode_n(_ptr(b), b.size, _ptr(out))
+    return out
+
+
+def quant_v_fp8(v, smooth: bool = True):
+    """V to E4M3 with one fp32 scale per (head, channel), after subtracting the channel mean
+    when smooth.  Returns (v8 uint8 codes, sv fp32 [*lead, d], vm fp32 [*lead, d] or None)."""
+    vb = _as_fp16_bits(v)
+    BH, N, d = _bhnd(vb)
+    v8 = np.empty(vb.shape, np.uint8)
+    sv = np.empty(vb.shape[:-2] + (d,), np.float32)
+    vm = np.empty(vb.shape[:-2] + (d,), np.float32) if smooth else None
+    _check(_load().oracle_quant_v_fp8(_ptr(vb), BH, N, d, _ptr(vm) if smooth else None, _ptr(sv), _ptr(v8)),
+           "oracle_quant_v_fp8")
+    return v8, sv, vm
+
+
+def attn_fp8pv(q8, k8, sq, sk, v8, sv, vm, causal: bool, sm_scale: float, groups=GROUP_PER_TOKEN):
+    """INT8 Q.K^T attention with P~ and V in E4M3 (readings in sage_oracle_sa2.c).
+    Returns (O fp64, O fp16)."""
+    q8 = np.ascontiguousarray(q8, np.int8)
+    k8 = np.ascontiguousarray(k8, np.int8)
+    sq = np.ascontiguousarray(sq, np.float32)
+    sk = np.ascontiguousarray(sk, np.float32)
+    v8 = np.ascontiguousarray(v8, np.uint8)
+    sv = np.ascontiguousarray(sv, np.float32)
+    vm_arr = None if vm is None else np.ascontiguousarray(vm, np.float32)
+    BH, N, d = _bhnd(v8)
+    o64 = np.empty(v8.shape, np.float64)
+    o16 = np.empty(v8.shape, np.uint16)
+    gq, gk = groups
+    _check(_load().oracle_attn_fp8pv(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v8), _ptr(sv),
+                                     _ptr(vm_arr) if vm_arr is not None else None, BH, N, d, int(bool(causal)),
+                                     float(sm_scale), gq, gk, _ptr(o64), _ptr(o16)), "oracle_attn_fp8pv")
+    return o64, o16.view(np.float16)
+
+
+def attn_fp8pv_rows(q8h, k8h, sqh, skh, v8h, svh, vmh, rows, causal: bool, sm_scale: float,
+                    groups=GROUP_PER_TOKEN) -> np.ndarray:
+    """Like attn_fp8pv() for one head [N,d], only the listed query rows (fp64)."""
+    q8h = np.ascontiguousarray(q8h, np.int8)
+    k8h = np.ascontiguousarray(k8h, np.int8)
+    sqh = np.ascontiguousarray(sqh, np.float32)
+    skh = np.ascontiguousarray(skh, np.float32)
+    v8h = np.ascontiguousarray(v8h, np.uint8)
+    svh = np.ascontiguousarray(svh, np.float32)
+    vmh = None if vmh is None else np.ascontiguousarray(vmh, np.float32)
+    N, d = v8h.shape
+    rows = np.ascontiguousarray(rows, np.int64)
+    o64 = np.empty((rows.size, d), np.float64)
+    gq, gk = groups
+    _check(_load().oracle_attn_fp8pv_rows(_ptr(q8h), _ptr(k8h), _ptr(sqh), _ptr(skh), _ptr(v8h), _ptr(svh),
+                                          _ptr(vmh) if vmh is not None else None, N, d, int(bool(causal)),
+                                          float(sm_scale), gq, gk, _ptr(rows), rows.size, _ptr(o64)),
+           "oracle_attn_fp8pv_rows")
+    return o64
+
+
+def sage_attn_fp8pv(q, k, v, causal: bool, sm_scale: float, per_block: bool, smooth_v: bool = True):
+    """The FP8 P.V variant in order: smooth K, quantize Q and K to INT8, quantize V to E4M3
+    (smoothed), attention with P~ in E4M3.  Returns every intermediate."""
+    gq, gk = GROUP_PER_BLOCK if per_block else GROUP_PER_TOKEN
+    km = smooth_k(k)
+    q8, sq = quant(q, gq)
+    k8, sk = quant(k, gk, km)
+    v8, sv, vm = quant_v_fp8(v, smooth_v)
+    o64, o16 = attn_fp8pv(q8, k8, sq, sk, v8, sv, vm, causal, sm_scale, (gq, gk))
+    return dict(km=km, q8=q8, sq=sq, k8=k8, sk=sk, v8=v8, sv=sv, vm=vm, o64=o64, o16=o16)
 
 
 def metrics(a: np.ndarray, b: np.ndarray) -> dict:

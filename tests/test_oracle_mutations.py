@@ -1,15 +1,17 @@
 """Mutation tests of the oracle's pins.
 
-Each case plants one plausible slip in a copy of oracle/sage_oracle.c (a dropped
-rounding, a rounding taken another way, a wrong sign, index, group size or
-operand), builds the copy with the oracle's own compiler flags, and runs
-tests/test_oracle_pins.py against it in a fresh process (the oracle package loads
+Each case plants one plausible slip in a copy of the oracle's C sources (a dropped
+rounding, a rounding taken another way, a wrong sign, index, group size, offset or
+operand), builds the copy with the oracle's own compiler flags, and runs the pin
+files (tests/test_oracle_pins.py, tests/test_oracle_pins_fp8.py) against it in a
+fresh process (the oracle package loads
 the library named by SAGE_ORACLE_LIB).  The pins must fail on every mutant, and
 pass on an unmodified copy built the same way (the control case), so a pin that
 cannot tell a slip from the reading it pins shows up here.
 
 The readings pinned are those of the SageAttention summary page (Summary bullets
-1-2: INT8 Q.K^T after smoothing K, P.V in fp16; idea I1: the K shift).
+1-2: INT8 Q.K^T after smoothing K, P.V in fp16; idea I1: the K shift) and of the
+SageAttention2 abstract for the FP8 P.V variant (E4M3 P~ and V, V smoothing).
 """
 import concurrent.futures
 import os
@@ -19,11 +21,11 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "oracle", "sage_oracle.c")
-PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+SRCS = {f: os.path.join(ROOT, "oracle", f) for f in ("sage_oracle.c", "sage_oracle_sa2.c")}
+PINS = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_pins_fp8.py")]
 
 # (name, text in sage_oracle.c, replacement, expected number of occurrences)
-MUTATIONS = [
+BASE_MUTATIONS = [
     ("p_unrounded", "const double pt = h2d(d2h(e));", "const double pt = e;", 1),
     ("p_rounded_via_fp32", "const double pt = h2d(d2h(e));", "const double pt = h2d(d2h((double)(float)e));", 1),
     ("row_sum_of_rounded_p", "l += e;\n        const double pt = h2d(d2h(e));",
@@ -49,31 +51,56 @@ MUTATIONS = [
      "const int64_t jend = causal ? i + 2 : N;\n                    double m", 1),
 ]
 
+# (name, text in sage_oracle_sa2.c, replacement, expected number of occurrences)
+FP8_MUTATIONS = [
+    ("fp8_p_unrounded", "const double pt = oracle_e4m3_decode(oracle_e4m3_encode(p));", "const double pt = p;", 1),
+    ("fp8_p_as_fp16", "const double pt = oracle_e4m3_decode(oracle_e4m3_encode(p));",
+     "const double pt = (double)(_Float16)p;", 1),
+    ("fp8_offset_exact_max", "const double M = ceil(umax);", "const double M = umax;", 1),
+    ("fp8_offset_floor", "const double M = ceil(umax);", "const double M = floor(umax);", 1),
+    ("fp8_row_sum_of_rounded", "l += p;\n        const double pt = oracle_e4m3_decode(oracle_e4m3_encode(p));",
+     "const double pt = oracle_e4m3_decode(oracle_e4m3_encode(p));\n        l += pt;", 1),
+    ("fp8_v_int8_range", "s = a / 448.0f;\n                inv = 448.0f / a;",
+     "s = a / 127.0f;\n                inv = 127.0f / a;", 1),
+    ("fp8_v_mean_not_added", "+ (vmh ? (double)vmh[c] : 0.0)", "", 1),
+    ("fp8_v_smoothing_sign", "(float)h2d_sa2(vh[t * d + c]) - mean;", "(float)h2d_sa2(vh[t * d + c]) + mean;", 2),
+    ("fp8_v_scale_not_applied", "acc[c] * (double)svh[c] / l", "acc[c] / l", 1),
+    ("e4m3_ties_away", "double m = nearbyint(ldexp(a, 3 - eb));", "double m = round(ldexp(a, 3 - eb));", 1),
+    ("e4m3_subnormal_step", "nearbyint(ldexp(a, 9))", "nearbyint(ldexp(a, 10))", 1),
+    ("e4m3_nan_not_saturated", "return sign | 0x7E; /* 448", "return sign | 0x7F; /* 448", 1),
+    ("e4m3_decode_bias", "ldexp(1.0 + F / 8.0, E - 7)", "ldexp(1.0 + F / 8.0, E - 8)", 1),
+]
+
+MUTATIONS = [("sage_oracle.c",) + m for m in BASE_MUTATIONS] + [("sage_oracle_sa2.c",) + m for m in FP8_MUTATIONS]
+
 CFLAGS = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
 
 
-def _build_and_run_pins(name, old, new, count, tmpdir):
-    src = open(SRC).read()
-    if old:  # the control case builds the unmodified text
-        assert src.count(old) == count, f"{name}: expected {count} occurrence(s) of the mutated text"
-    mutated = src.replace(old, new) if old else src
-    c_path = os.path.join(tmpdir, f"{name}.c")
-    so_path = os.path.join(tmpdir, f"lib_{name}.so")
-    with open(c_path, "w") as f:
-        f.write(mutated)
-    subprocess.run(CFLAGS + ["-o", so_path, c_path, "-lm"], check=True, capture_output=True)
+def _build_and_run_pins(fname, name, old, new, count, tmpdir):
+    os.makedirs(os.path.join(tmpdir, name), exist_ok=True)
+    c_paths = []
+    for f, path in SRCS.items():
+        src = open(path).read()
+        if f == fname and old:  # the control case builds the unmodified texts
+            assert src.count(old) == count, f"{name}: expected {count} occurrence(s) of the mutated text"
+            src = src.replace(old, new)
+        c_paths.append(os.path.join(tmpdir, name, f))
+        with open(c_paths[-1], "w") as fh:
+            fh.write(src)
+    so_path = os.path.join(tmpdir, name, "lib_oracle.so")
+    subprocess.run(CFLAGS + ["-o", so_path, *c_paths, "-lm"], check=True, capture_output=True)
     env = dict(os.environ, SAGE_ORACLE_LIB=so_path, OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", PINS, "-x", "-q", "-p", "no:cacheprovider"],
+    r = subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     return r.returncode, r.stdout[-2000:] + r.stderr[-2000:]
 
 
 def test_pins_fail_on_every_mutant_and_pass_on_the_control(tmp_path):
-    jobs = [("control", "", "", 0)] + MUTATIONS
+    jobs = [("sage_oracle.c", "control", "", "", 0)] + MUTATIONS
     with concurrent.futures.ThreadPoolExecutor(max_workers=max(2, min(8, os.cpu_count() or 2))) as ex:
-        futs = {name: ex.submit(_build_and_run_pins, name, old, new, cnt, str(tmp_path))
-                for name, old, new, cnt in jobs}
-        results = {name: f.result() for name, f in futs.items()}
+        futs = {name: ex.submit(_build_and_run_pins, f, name, old, new, cnt, str(tmp_path))
+                for f, name, old, new, cnt in jobs}
+        results = {name: fu.result() for name, fu in futs.items()}
     rc, out = results.pop("control")
     assert rc == 0, f"the unmodified oracle must pass its pins:\n{out}"
     survivors = {name: out for name, (rc, out) in results.items() if rc != 1}
@@ -82,7 +109,7 @@ def test_pins_fail_on_every_mutant_and_pass_on_the_control(tmp_path):
         f"{n} (exit {results[n][0]})" for n in survivors)
 
 
-@pytest.mark.parametrize("name,old,new,count", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_mutation_targets_exist(name, old, new, count):
+@pytest.mark.parametrize("fname,name,old,new,count", MUTATIONS, ids=[m[1] for m in MUTATIONS])
+def test_mutation_targets_exist(fname, name, old, new, count):
     # the planted slips refer to the oracle's current text (a refactor must update them)
-    assert open(SRC).read().count(old) == count
+    assert open(SRCS[fname]).read().count(old) == count
