@@ -280,8 +280,23 @@ def run_ours(args, w: W.Workload):
         if world > 1:
             dist.barrier()
 
+    fp8 = args.variant == "fp8pv"
+    if fp8:  # E4M3 V codes, per-channel scales and means for the FP8 P.V variant's kernel-only timing
+        v8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        sv = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+        vm = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+
     def step():
-        sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+        if fp8:
+            sa.sage_attn_fwd_fp8pv(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+        else:
+            sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+
+    def fused():
+        if fp8:
+            sa.sage_attn_fwd_fp8pv_quantized(q8, k8, sq, sk, v8, sv, vm, o, w.causal, w.sm_scale, gran, stream)
+        else:
+            sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
 
     # the tensor cores' dense per-SM rates for INT8 and FP16 (and FP8) on this GPU, measured
     # before the timed region: the roofline's INT8 : FP16 ratio as measured here
@@ -323,13 +338,15 @@ def run_ours(args, w: W.Workload):
     # ---- the fused kernel alone (already-quantized inputs), same stream, for the roofline
     sa.sage_smooth_k(k, km, stream)
     sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream)
+    if fp8:
+        sa.sage_quant_v_fp8(v, v8, sv, vm, stream)
     for _ in range(3):
-        sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
+        fused()
     torch.cuda.synchronize(dev)
     k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     k0.record(stream)
     for _ in range(args.steps):
-        sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
+        fused()
     k1.record(stream)
     torch.cuda.synchronize(dev)
     kernel_ms = k0.elapsed_time(k1) / args.steps
@@ -352,6 +369,8 @@ def run_ours(args, w: W.Workload):
         "attn_kernel_ms": kernel_ms,
         "step_ms": ms,
     }
+    if fp8:
+        breakdown["quant_v_fp8_ms"] = timed(lambda: sa.sage_quant_v_fp8(v, v8, sv, vm, stream), nb)
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, D2H output per step
     qp, kp, vp = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
@@ -359,6 +378,13 @@ def run_ours(args, w: W.Workload):
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
+        if fp8:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            step()
+            op.copy_(o, non_blocking=True)
+            return
         # the C-ABI call with host buffers: copies in, compute and copies out overlap across
         # chunks of heads inside the call
         sa.sage_attn_fwd_host(qp, kp, vp, op, w.causal, w.sm_scale, gran, 0, stream)
@@ -384,12 +410,14 @@ def run_ours(args, w: W.Workload):
         p_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
         p_burst = float(peaks["bf16_tflops"])
         # the kernel-only loop is short (steps x kernel_ms, well under a second), so the burst
-        # peak is its denominator; the sustained figure is kept in the note
-        peak = mixed_peak_tops(p_burst)
+        # peak is its denominator; the sustained figure is kept in the note.  The FP8 P.V variant's
+        # P.V runs at the FP8 rate (2 x FP16, as INT8): its roofline is the INT8 one.
+        peak_of = (lambda p: 2.0 * p) if fp8 else mixed_peak_tops
+        peak = peak_of(p_burst)
         achieved = ops / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
         accuracy = None
-        if args.no_cpu_baseline or world > 1:  # the CPU baseline belongs to the N=1 line only
+        if args.no_cpu_baseline or world > 1 or fp8:  # the CPU baseline belongs to the N=1 headline line only
             cpu_tops, cores, desc = None, None, ("skipped" if world == 1 else "rank 0 at N=1 only")
         else:
             cpu_tops, cores, desc, sample = oracle_sample(w, keep=True)
@@ -398,21 +426,23 @@ def run_ours(args, w: W.Workload):
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8+f16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3" if fp8 else "int8+f16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
+                       "variant": "fp8 P.V (E4M3 P~ and V, V smoothed)" if fp8 else "fp16 P.V",
                        "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default); no flush needed",
                        "parallelism": (f"heads sharded over {world} ranks ({w.BH} per rank, "
                                        f"global B*H = {world * w.BH}); no data-path collective")},
             "roofline": {"bound": "tensor", "kernel": ("sage_attn_v3_kernel" if w.d == 128 else "sage_attn_kernel"), "achieved": round(achieved, 2),
                          "peak": round(peak, 2), "unit": "TOPS", "frac": round(achieved / peak, 4),
                          "traffic": traffic,
-                         "peak_note": (f"mixed INT8+FP16 roofline 4/(2/P_i8 + 2/P_f16) of {src} peaks: P_f16 = "
+                         "peak_note": (f"{'INT8+FP8 roofline 4/(2/P_i8 + 2/P_f8), P_f8 = P_i8' if fp8 else 'mixed INT8+FP16 roofline 4/(2/P_i8 + 2/P_f16)'}"
+                                       f" of {src} peaks: P_f16 = "
                                        f"burst bf16 {p_burst} TFLOP/s (the kernel loop lasts "
                                        f"{kernel_ms * args.steps / 1e3:.2f} s), P_i8 = 2 x P_f16 (dense datasheet "
-                                       f"ratio) -> {peak:.1f} TOPS; against the sustained {p_sus}: "
-                                       f"{mixed_peak_tops(p_sus):.1f} TOPS, frac "
-                                       f"{achieved / mixed_peak_tops(p_sus):.4f}"),
+                                       f"ratio; the probe's measured ratio is in tensor_probe) -> {peak:.1f} TOPS; "
+                                       f"against the sustained {p_sus}: {peak_of(p_sus):.1f} TOPS, frac "
+                                       f"{achieved / peak_of(p_sus):.4f}"),
                          "kernel_ms": round(kernel_ms, 4), "tensor_probe": probe},
             "cpu_baseline": {"value": cpu_tops, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": round(job_tops(world, ops, e2e_ms), 2), "unit": UNIT,
@@ -420,7 +450,7 @@ def run_ours(args, w: W.Workload):
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
             "accuracy": accuracy,
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
     if world > 1:
@@ -468,6 +498,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
+    ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv"],
+                    help="fp16pv: the SageAttention method (P.V in fp16); fp8pv: its FP8 P.V variant (d=128)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiler runs)")
     args = ap.parse_args(argv)

@@ -97,6 +97,38 @@ int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq,
                             const void* v, void* o, int B, int H, int N, int d, int causal,
                             float sm_scale, int granularity, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * FP8 P.V variant, following the SageAttention2 abstract (author pages of Jia Wei and Haofeng
+ * Huang; arXiv 2411.10958): the matrices (P~, V) are quantized to FP8, V is smoothed, and P~V is
+ * accumulated in an FP32 buffer.  Q.K^T stays the INT8 product above (the abstract's INT4 Q.K^T
+ * is not part of this variant).  FP8 is E4M3 (bias 7, largest finite 448), round to nearest
+ * even, saturating.  Head dimension 128 only (d = 64 returns SAGE_ERR_UNSUPPORTED).
+ *
+ * V to FP8, per (b,h) and channel c: vm = channel mean over the N tokens (exact sum, as the K
+ * mean) when vm != NULL, else 0; x = fl32(V - vm); a = max_t |x|; sv = fl32(a/448);
+ * v8 = e4m3(fl32(x * fl32(448/a))) (a == 0: sv = 0, codes 0).  One scale per channel: it is
+ * constant along the P.V contraction (the tokens).
+ * v: fp16 [B,H,N,d] (in); v8: E4M3 codes [B,H,N,d] (out); sv: fp32 [B,H,d] (out);
+ * vm: fp32 [B,H,d] (out) or NULL (no smoothing). */
+int sage_quant_v_fp8(const void* v, uint8_t* v8, float* sv, float* vm, int B, int H, int N, int d, void* stream);
+
+/* The fused kernel of the FP8 P.V variant on quantized inputs: S and the online softmax as in
+ * sage_attn_fwd_quantized, except that the row offsets are integers in log2 units and
+ * P~ = e4m3(2^(s*log2(e) - offset + 8)) (the row's largest weight near 2^8, every weight rounded on
+ * the E4M3 grid of a power-of-two scaling of exp(s - max s)); O^T += V8^T . P~^T on tcgen05
+ * kind::f8f6f4 with fp32 accumulation in tensor memory; O = acc / l * sv + vm stored as fp16.
+ * The row sum l uses the unrounded weights.  q8, k8, sq, sk as for sage_attn_fwd_quantized;
+ * v8, sv, vm from sage_quant_v_fp8 (vm may be NULL); o: fp16 [B,H,N,d] (out). */
+int sage_attn_fwd_fp8pv_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
+                                  const uint8_t* v8, const float* sv, const float* vm, void* o, int B, int H, int N,
+                                  int d, int causal, float sm_scale, int granularity, void* stream);
+
+/* The whole FP8 P.V variant as a user calls it: smooth K, INT8 Q and K, V to FP8 with
+ * smoothing, the fused kernel above.  Arguments, validation and workspace as sage_attn_fwd (the
+ * workspace also holds the E4M3 V: 3*B*H*N*d bytes plus scales and means). */
+int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                        int causal, float sm_scale, int granularity, void* stream);
+
 /* Debug: the full integer product s[b,h,i,j] = sum_c q8[b,h,i,c] * k8[b,h,j,c] as int32
  * (exact: |s| <= 128*127*127 < 2^31), computed with the same tensor-core path as the fused
  * kernel.  s: int32 [B,H,N,N] (out); needs B*H*N*N < 2^31. */

@@ -53,6 +53,9 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_attn_fwd.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_attn_fwd_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_debug_qk_int32.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_quant_v_fp8.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_attn_fwd_fp8pv_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_attn_fwd_fp8pv.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_last_device_error.argtypes = [_p]
         lib.sage_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_noalloc_scratch_bytes.argtypes = [_i, _i, _i, _i, _i]
@@ -64,7 +67,8 @@ def get_lib() -> ctypes.CDLL:
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
                   "sage_debug_attn_trace", "sage_debug_mma_peak", "sage_attn_fwd_host",
-                  "sage_debug_wait_timeout"):
+                  "sage_debug_wait_timeout", "sage_quant_v_fp8", "sage_attn_fwd_fp8pv_quantized",
+                  "sage_attn_fwd_fp8pv"):
             getattr(lib, n).restype = _i
         _lib = lib
     return _lib
@@ -143,6 +147,29 @@ def sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float,
     _check(get_lib().sage_attn_fwd_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v), _ptr(o), B, H, N,
                                        d, int(bool(causal)), float(sm_scale), int(granularity),
                                        _stream(stream)), "sage_attn_fwd_quantized")
+
+
+def sage_quant_v_fp8(v, v8, sv, vm=None, stream=None) -> None:
+    """V to E4M3 codes (uint8 tensor) with per-(head, channel) scales sv; channel means into vm
+    (V smoothed) unless vm is None (FP8 P.V variant, SageAttention2 abstract)."""
+    B, H, N, d = _shape(v)
+    _check(get_lib().sage_quant_v_fp8(_ptr(v), _ptr(v8), _ptr(sv), _ptr(vm), B, H, N, d, _stream(stream)),
+           "sage_quant_v_fp8")
+
+
+def sage_attn_fwd_fp8pv_quantized(q8, k8, sq, sk, v8, sv, vm, o, causal: bool, sm_scale: float, granularity: int,
+                                  stream=None) -> None:
+    B, H, N, d = _shape(o)
+    _check(get_lib().sage_attn_fwd_fp8pv_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v8), _ptr(sv),
+                                                   _ptr(vm), _ptr(o), B, H, N, d, int(bool(causal)), float(sm_scale),
+                                                   int(granularity), _stream(stream)),
+           "sage_attn_fwd_fp8pv_quantized")
+
+
+def sage_attn_fwd_fp8pv(q, k, v, o, causal: bool, sm_scale: float, granularity: int, stream=None) -> None:
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_attn_fwd_fp8pv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+                                         float(sm_scale), int(granularity), _stream(stream)), "sage_attn_fwd_fp8pv")
 
 
 def sage_debug_qk_int32(q8, k8, s, stream=None) -> None:

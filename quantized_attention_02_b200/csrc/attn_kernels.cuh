@@ -20,6 +20,11 @@ struct AttnArgs {
   float sm_scale_log2;      // sm_scale * log2(e)
   long long* trace = nullptr;  // non-null: traced build, stamps of the first trace_ctas CTAs
   int trace_ctas = 0;
+  // FP8 P.V variant (D = 128): tm_v maps E4M3 codes [BH][N][128] (box {128, 128, 1}, 128 B
+  // swizzle); sv: per-(head, channel) scales [BH][128]; vm: channel means [BH][128] or null
+  bool fp8 = false;
+  const float* sv = nullptr;
+  const float* vm = nullptr;
 };
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);

@@ -13,7 +13,10 @@
 // Included by attn_kernels.cu inside namespace sage (one translation unit with the PTX helpers).
 #pragma once
 
-struct V3Layout {
+// FP8: the P.V variant with E4M3 P~ and V (kind::f8f6f4): one 128-byte TMA box per V tile and
+// one byte per P~ element; the P~ region keeps its fp16 size because the epilogue stages O there.
+template <bool FP8>
+struct V3LayoutT {
   static constexpr int D = 128;
   static constexpr int BM = 128, BN = 128;
   static constexpr int SK = 3;                // K stages
@@ -21,7 +24,7 @@ struct V3Layout {
   static constexpr int Q_BYTES = BM * D;      // int8 tile
   static constexpr int K_BYTES = BN * D;      // int8 tile
   static constexpr int V_BOX = BN * 128;      // one 64-column fp16 box (128-byte rows)
-  static constexpr int V_BYTES = BN * D * 2;  // two boxes
+  static constexpr int V_BYTES = FP8 ? BN * D : BN * D * 2;  // fp16: two boxes; e4m3: one
   static constexpr int P_ATOM = 256 * 128;    // 64 keys x 256 query rows of fp16 P~
   static constexpr int P_BYTES = 2 * P_ATOM;  // 128 keys
   static constexpr int OFF_Q = 0;
@@ -40,7 +43,27 @@ struct V3Layout {
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 512;
 };
-static_assert(V3Layout::SMEM <= 227 * 1024, "shared memory budget");
+using V3Layout = V3LayoutT<false>;
+static_assert(V3LayoutT<false>::SMEM <= 227 * 1024 && V3LayoutT<true>::SMEM <= 227 * 1024, "shared memory budget");
+
+// Exact 2^k for an integer k <= 0 (0 below the normal range): the FP8 variant's offsets are
+// integers, so its rescale factors are powers of two and rescaling O and l is exact.
+__device__ __forceinline__ float exp2_int(float k) {
+  const int e = 127 + static_cast<int>(k);
+  return e > 0 ? __int_as_float(e << 23) : 0.f;
+}
+
+// Four fp32 values to E4M3 (round to nearest even, saturating), packed little-endian.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;  // cvt packs its first source into the upper byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
 
 // exp2 on the FMA pipe for a pair of arguments (Cody-Waite style range reduction plus a
 // polynomial), to take part of the exp2 work off the MUFU unit:
@@ -88,13 +111,22 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
 //               stages O in shared memory and TMA-stores it, both tiles in parallel
 //   12-15       correction (thread = head dimension d = TMEM lane of O^T): rescales the O^T
 //               columns of rows whose offset moved, between two P.V products
-template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED>
+//
+// FP8 = true is the P.V variant of the SageAttention2 abstract ((P~, V) in FP8, P~V accumulated in
+// an FP32 buffer -- here the tensor memory accumulator): V arrives as E4M3 codes with per-channel
+// scales sv and channel means vm (vm may be null), P~ is rounded to E4M3 and P.V runs as
+// tcgen05 kind::f8f6f4 with fp32 accumulation.  The row offsets are integers (quantum >= 1) and
+// P~ = 2^(s - m_use + 8), so P~ is rounded on the E4M3 grid of a power-of-two scaling of
+// exp(s - max s), as the oracle rounds it, and the offset moves as soon as the row maximum passes
+// it by half a unit (P~ <= 2^8.5 < 448); the epilogue applies sv and adds vm.
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED, bool FP8 = false>
 __global__ void __launch_bounds__(512, 1)
     sage_attn_v3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                         const float* __restrict__ sq, const float* __restrict__ sk, int BH, int N,
-                        float sm_scale_log2, long long* __restrict__ trace, int trace_ctas) {
-  using L = V3Layout;
+                        float sm_scale_log2, long long* __restrict__ trace, int trace_ctas,
+                        const float* __restrict__ sv = nullptr, const float* __restrict__ vm = nullptr) {
+  using L = V3LayoutT<FP8>;
   constexpr int D = L::D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -225,7 +257,7 @@ __global__ void __launch_bounds__(512, 1)
         if (j >= L::SV && !mbar_wait(bar_v_empty + sv_, (j / L::SV - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar_v_full + sv_, L::V_BYTES);
         tma_load_3d(sV + sv_ * L::V_BYTES, &tm_v, bar_v_full + sv_, 0, key_row, bh);
-        tma_load_3d(sV + sv_ * L::V_BYTES + L::V_BOX, &tm_v, bar_v_full + sv_, 64, key_row, bh);
+        if constexpr (!FP8) tma_load_3d(sV + sv_ * L::V_BYTES + L::V_BOX, &tm_v, bar_v_full + sv_, 64, key_row, bh);
         v_issued[sv_] = j / L::SV + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
@@ -241,8 +273,11 @@ __global__ void __launch_bounds__(512, 1)
     // tensor core.  The whole warp runs the loop; elect.sync lets one lane issue.
     const int t = warp == 1 ? 0 : 1;
     if (t < n_tiles) {
+      // tile t's P~ rows: fp16, 128 rows of each 64-key atom; e4m3, 128 rows of 128 bytes
       const uint32_t v_base = smem_u32(sV), p_base = smem_u32(sP) + t * 128 * 128;
       constexpr uint32_t IDESC_PV = make_idesc(1 /*f32*/, 0, 0, 1 /*A = V^T MN-major*/, 0, 128, 128);
+      // kind::f8f6f4: format 0 = E4M3 for A and B, A = V^T MN-major (allowed for 8-bit E4M3)
+      constexpr uint32_t IDESC_PV8 = make_idesc(1 /*f32*/, 0 /*e4m3*/, 0 /*e4m3*/, 1, 0, 128, 128);
       const uint32_t d_tmem = tmem + 256 + 128 * t;
       bool ok = true;
       for (int j = 0; ok && j < n_iter[t]; ++j) {
@@ -253,6 +288,17 @@ __global__ void __launch_bounds__(512, 1)
         for (int half = 0; half < 2; ++half) {
           if (!wait_warp(half == 0 ? bar_p_lo + t : bar_p_hi + t, j & 1)) { ok = false; break; }
           tc_fence_after();
+          if constexpr (FP8) {
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = half * 2 + k2;  // 32 keys per MMA
+              // A = V^T in E4M3: keys kk*32.. of the V tile (32 rows of 128 B: all 128 head dims)
+              const uint64_t a = make_smem_desc(v_base + s * L::V_BYTES + kk * 32 * 128, L::V_BYTES, 1024, kSwizzle128B);
+              // B = P~_t^T in E4M3: 32-byte step kk inside the tile's 128-byte swizzled rows
+              const uint64_t b = make_smem_desc(p_base + kk * 32, 16, 1024, kSwizzle128B);
+              mma_f8_ss_warp(d_tmem, a, b, IDESC_PV8, (j == 0 && kk == 0) ? 0u : 1u);
+            }
+          } else {
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
             const int kk = half * 4 + k4;  // 16 keys per MMA
@@ -261,6 +307,7 @@ __global__ void __launch_bounds__(512, 1)
             // B = P~_t^T: 64-key atom `half`, 32-byte step k4 inside the 128-byte swizzled rows
             const uint64_t b = make_smem_desc(p_base + half * L::P_ATOM + k4 * 32, 16, 1024, kSwizzle128B);
             mma_f16_ss_warp(d_tmem, a, b, IDESC_PV, (j == 0 && kk == 0) ? 0u : 1u);
+          }
           }
           if (half == 1) mma_commit_warp(bar_o_done + t);
         }
@@ -328,7 +375,8 @@ __global__ void __launch_bounds__(512, 1)
       const int qi = t * 128 + r;  // the CTA's query index (row of P~, column of O^T)
       const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
       const uint32_t tS = tmem + lane_addr + 128 * t;
-      const uint32_t p_row = smem_u32(sP) + qi * 128;
+      const uint32_t p_row = smem_u32(sP) + qi * 128;   // fp16 P~: this row in each 64-key atom
+      const uint32_t p_row8 = smem_u32(sP) + qi * 128;  // e4m3 P~: all 128 keys in one 128-byte row
       // rows past N (a partial last tile) compute on zeros and are never stored
       const float sq_r = PER_TOKEN ? (q_row < N ? __ldg(sq + row_base + q_row) : 0.f) : __ldg(sq + bh * n_qtiles + q_tile);
       const float a_r = sq_r * sm_scale_log2;
@@ -342,6 +390,16 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) skmax = fmaxf(skmax, __shfl_xor_sync(0xffffffffu, skmax, off));
         qm = offset_quantum(kMagicF * trim_scale(a_r * skmax));
+      }
+      // FP8: integer offsets (a power-of-two quantum of at least 1), P~ = 2^(s - m_use + p_shift)
+      // with the row maximum near 2^8; the offset moves once the maximum passes it by half a unit.
+      // (A quantum above 8 -- scores so coarse that one integer step of S moves them by more than
+      // 2^21 -- keeps the shift 0.)
+      float p_shift = 0.f, lazy = 8.f;
+      if constexpr (FP8) {
+        qm = fmaxf(qm, 1.f);
+        p_shift = qm <= 8.f ? 8.f : 0.f;
+        lazy = qm <= 8.f ? 0.5f : 8.f;
       }
 
       // per-token key scales: thread r fetches scale r of a key tile (zero past N) and the group
@@ -418,9 +476,9 @@ __global__ void __launch_bounds__(512, 1)
         bool rescale = false;
         if (j == 0) {
           m_use = round_up_to(mx, qm);
-        } else if (mx > m_use + 8.f) {
+        } else if (mx > m_use + lazy) {
           const float m_new = round_up_to(mx, qm);
-          alpha = fast_exp2(m_use - m_new);
+          alpha = FP8 ? exp2_int(m_use - m_new) : fast_exp2(m_use - m_new);
           m_use = m_new;
           rescale = true;
         }
@@ -439,8 +497,9 @@ __global__ void __launch_bounds__(512, 1)
             for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
           }
         }
-        const float nb0 = -fmaf(kMagicF, cb0, m_use);  // exact: see offset_quantum
-        const float nb1 = -fmaf(kMagicF, cb1, m_use);
+        const float m_exp = m_use - p_shift;  // exponent offset of P~ (= m_use for fp16 P~)
+        const float nb0 = -fmaf(kMagicF, cb0, m_exp);  // exact: see offset_quantum
+        const float nb1 = -fmaf(kMagicF, cb1, m_exp);
         if (r == 0) stamp((3 * t + 1) * n_kv_total + j);
 
         // ---- P~ = exp2(s - m_use) in fp16, 32 keys at a time from TMEM (the next chunk's load in
@@ -466,6 +525,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_arrive(bar_s_free + t);  // S_t fully read: the next Q.K^T may overwrite it
           }
           uint32_t pk[16];
+          float pf[FP8 ? 32 : 1];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const int c = cb + i;
@@ -474,7 +534,7 @@ __global__ void __launch_bounds__(512, 1)
               // fl(fl(S * sk) * a_r - m_use)
               const float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(x[i])), static_cast<float>(static_cast<int>(x[i + 1]))),
                                           *reinterpret_cast<const float2*>(skj + c));
-              tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
+              tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_exp, -m_exp));
             } else {
               const float cs = c < 64 ? cb0 : cb1;
               const float nb = c < 64 ? nb0 : nb1;
@@ -485,14 +545,31 @@ __global__ void __launch_bounds__(512, 1)
             // one pair in four on the FMA pipe (exp2_poly2), the rest on the MUFU unit
             const float2 p = ((i >> 1) & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
             lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
-            pk[i >> 1] = pack_half2(p.x, p.y);
+            if constexpr (FP8) {
+              pf[i] = p.x;
+              pf[i + 1] = p.y;
+            } else {
+              pk[i >> 1] = pack_half2(p.x, p.y);
+            }
           }
+          if constexpr (FP8) {
+            // keys cb..cb+31 = two 16-byte chunks of 16 keys in the query's 128-byte row
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int chunk = (cb >> 4) + g;
+              const float* f = pf + 16 * g;
+              st_shared_v4(p_row8 + ((chunk ^ (qi & 7)) << 4), pack_e4m3x4(f[0], f[1], f[2], f[3]),
+                           pack_e4m3x4(f[4], f[5], f[6], f[7]), pack_e4m3x4(f[8], f[9], f[10], f[11]),
+                           pack_e4m3x4(f[12], f[13], f[14], f[15]));
+            }
+          } else {
           // keys cb..cb+31 = four 16-byte chunks of 8 keys in 64-key atom cb/64
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const int chunk = ((cb & 63) >> 3) + g;
             st_shared_v4(p_row + (cb >> 6) * L::P_ATOM + ((chunk ^ (qi & 7)) << 4), pk[4 * g], pk[4 * g + 1],
                          pk[4 * g + 2], pk[4 * g + 3]);
+          }
           }
           if (cb == 32 || cb == 96) {
             fence_proxy_async_shared();
@@ -517,6 +594,7 @@ __global__ void __launch_bounds__(512, 1)
               if (!wait_warp(bar_o_done + t, (j - 1) & 1)) return false;
             }
             uint32_t pk[4];
+            float pf[FP8 ? 8 : 1];
 #pragma unroll
             for (int i = 0; i < 8; i += 2) {
               const int c = 8 * c8 + i;
@@ -524,7 +602,7 @@ __global__ void __launch_bounds__(512, 1)
               if constexpr (PER_TOKEN) {
                 const float2 v = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(x[i])), static_cast<float>(static_cast<int>(x[i + 1]))),
                                             *reinterpret_cast<const float2*>(skj + c));
-                tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_use, -m_use));
+                tt = __ffma2_rn(v, make_float2(a_r, a_r), make_float2(-m_exp, -m_exp));
               } else {
                 const float cs = c < 64 ? cb0 : cb1;
                 const float nb = c < 64 ? nb0 : nb1;
@@ -533,10 +611,21 @@ __global__ void __launch_bounds__(512, 1)
               }
               const float2 p = make_float2(c > cmax ? 0.f : fast_exp2(tt.x), c + 1 > cmax ? 0.f : fast_exp2(tt.y));
               lsum[(i >> 1) & 3] = __fadd2_rn(lsum[(i >> 1) & 3], p);
-              pk[i >> 1] = pack_half2(p.x, p.y);
+              if constexpr (FP8) {
+                pf[i] = p.x;
+                pf[i + 1] = p.y;
+              } else {
+                pk[i >> 1] = pack_half2(p.x, p.y);
+              }
             }
+            if constexpr (FP8) {
+              // keys 8*c8 .. 8*c8+7 = half (c8 mod 2) of 16-byte chunk c8/2 of the 128-byte row
+              st_shared_v2(p_row8 + (((c8 >> 1) ^ (qi & 7)) << 4) + (c8 & 1) * 8, pack_e4m3x4(pf[0], pf[1], pf[2], pf[3]),
+                           pack_e4m3x4(pf[4], pf[5], pf[6], pf[7]));
+            } else {
             // keys 8*c8 .. 8*c8+7 = 16-byte chunk (c8 mod 8) of 64-key atom c8/8
             st_shared_v4(p_row + (c8 >> 3) * L::P_ATOM + (((c8 & 7) ^ (qi & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            }
             if (c8 == 7 || c8 == 15) {
               fence_proxy_async_shared();
               mbar_arrive(c8 == 7 ? bar_p_lo + t : bar_p_hi + t);
@@ -567,6 +656,14 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t tOT = tmem + lane_addr + 256 + 128 * t;
         const uint32_t stage = smem_u32(sP) + (r >> 6) * L::P_ATOM + t * 128 * 128 + (r & 63) * 2;
         const float* inv_l = sL + t * 128;
+        // FP8: head dimension r's scale and mean (O = O^T acc / l * sv + vm)
+        float2 sv2 = make_float2(1.f, 1.f), vm2 = make_float2(0.f, 0.f);
+        if constexpr (FP8) {
+          const float s_ = __ldg(sv + static_cast<size_t>(bh) * D + r);
+          const float m_ = vm ? __ldg(vm + static_cast<size_t>(bh) * D + r) : 0.f;
+          sv2 = make_float2(s_, s_);
+          vm2 = make_float2(m_, m_);
+        }
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 64) {
           uint32_t ov[64];
@@ -577,8 +674,12 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int i = 0; i < 64; i += 4) {
             const float4 il = *reinterpret_cast<const float4*>(inv_l + cb + i);
-            const float2 a = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(il.x, il.y));
-            const float2 b = __fmul2_rn(make_float2(__uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3])), make_float2(il.z, il.w));
+            float2 a = __fmul2_rn(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(il.x, il.y));
+            float2 b = __fmul2_rn(make_float2(__uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3])), make_float2(il.z, il.w));
+            if constexpr (FP8) {
+              a = __ffma2_rn(a, sv2, vm2);
+              b = __ffma2_rn(b, sv2, vm2);
+            }
             const uint32_t ha = pack_half2(a.x, a.y), hb = pack_half2(b.x, b.y);
             st_shared_u16(stage + (cb + i) * 128, static_cast<uint16_t>(ha));
             st_shared_u16(stage + (cb + i + 1) * 128, static_cast<uint16_t>(ha >> 16));

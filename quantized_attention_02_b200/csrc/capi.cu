@@ -75,6 +75,11 @@ bool make_v_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
   return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// E4M3 V codes of the FP8 P.V variant: [BH][N][128] bytes, one box of 128 columns x 128 tokens.
+bool make_v8_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
+  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, BH, D, D, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // O written by TMA stores of [128 rows x 64 columns] fp16 boxes from unswizzled shared memory.
 bool make_o_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
   return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -104,12 +109,16 @@ int check_gran(int g) { return (g == SAGE_PER_TOKEN || g == SAGE_PER_BLOCK) ? SA
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
 
+// v: fp16 V, or (fp8_sv != nullptr) the E4M3 codes of the FP8 P.V variant with their
+// per-channel scales fp8_sv and means fp8_vm (may be null).
 int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v, void* o,
                         int B, int H, int N, int d, int causal, float sm_scale, int granularity,
-                        cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0) {
+                        cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0,
+                        const float* fp8_sv = nullptr, const float* fp8_vm = nullptr) {
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
-  if (!make_qk_map3(&tq, q8, N, BH, d) || !make_qk_map3(&tk, k8, N, BH, d) || !make_v_map3(&tv, v, N, BH, d) ||
+  const bool vmap_ok = fp8_sv ? make_v8_map3(&tv, v, N, BH, d) : make_v_map3(&tv, v, N, BH, d);
+  if (!make_qk_map3(&tq, q8, N, BH, d) || !make_qk_map3(&tk, k8, N, BH, d) || !vmap_ok ||
       !make_o_map3(&to, o, N, BH, d))
     return SAGE_ERR_CUDA;
   sage::AttnArgs a{};
@@ -128,6 +137,9 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
   a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
   a.trace = trace;
   a.trace_ctas = trace_ctas;
+  a.fp8 = fp8_sv != nullptr;
+  a.sv = fp8_sv;
+  a.vm = fp8_vm;
   const cudaError_t e = sage::launch_attn(a, st);
   return e == cudaErrorNotSupported ? SAGE_ERR_UNSUPPORTED : cuda_status(e);
 }
@@ -265,6 +277,79 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   nvtxRangePop();
   nvtxRangePushA("sage_attn_fused");
   if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity, st);
+  nvtxRangePop();
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
+}
+
+int sage_quant_v_fp8(const void* v, uint8_t* v8, float* sv, float* vm, int B, int H, int N, int d, void* stream) {
+  if (!v || !v8 || !sv) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (!aligned16(v) || !aligned16(v8)) return SAGE_ERR_INVALID;
+  return cuda_status(sage::launch_quant_v_fp8(static_cast<const __half*>(v), v8, sv, vm, B * H, N, d,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int sage_attn_fwd_fp8pv_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
+                                  const uint8_t* v8, const float* sv, const float* vm, void* o, int B, int H, int N,
+                                  int d, int causal, float sm_scale, int granularity, void* stream) {
+  if (!q8 || !k8 || !sq || !sk || !v8 || !sv || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(sk)) return SAGE_ERR_INVALID;
+  return attn_quantized_impl(q8, k8, sq, sk, v8, o, B, H, N, d, causal, sm_scale, granularity,
+                             static_cast<cudaStream_t>(stream), nullptr, 0, sv, vm);
+}
+
+int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                        float sm_scale, int granularity, void* stream) {
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const size_t elems = static_cast<size_t>(BH) * N * d;
+  const size_t nsq = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 1);
+  const size_t nsk = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 0);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t chan = up(static_cast<size_t>(BH) * d * 4);
+  const size_t off_k8 = up(elems);
+  const size_t off_v8 = off_k8 + up(elems);
+  const size_t off_sq = off_v8 + up(elems);
+  const size_t off_sk = off_sq + up(nsq * 4);
+  const size_t off_km = off_sk + up(nsk * 4);
+  const size_t off_sv = off_km + chan;
+  const size_t off_vm = off_sv + chan;
+  const size_t total = off_vm + chan;
+  void* ws = nullptr;
+  if (sage::workspace_alloc(&ws, total, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int8_t* q8 = reinterpret_cast<int8_t*>(w);
+  int8_t* k8 = reinterpret_cast<int8_t*>(w + off_k8);
+  uint8_t* v8 = w + off_v8;
+  float* sq = reinterpret_cast<float*>(w + off_sq);
+  float* sk = reinterpret_cast<float*>(w + off_sk);
+  float* km = reinterpret_cast<float*>(w + off_km);
+  float* sv = reinterpret_cast<float*>(w + off_sv);
+  float* vm = reinterpret_cast<float*>(w + off_vm);
+  nvtxRangePushA("sage_fp8pv_prep");
+  rc = cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, BH, N, d, st));
+  if (!rc) rc = sage_quant_qk(q, k, km, q8, k8, sq, sk, B, H, N, d, granularity, stream);
+  if (!rc) rc = cuda_status(sage::launch_quant_v_fp8(static_cast<const __half*>(v), v8, sv, vm, BH, N, d, st));
+  nvtxRangePop();
+  nvtxRangePushA("sage_fp8pv_fused");
+  if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v8, o, B, H, N, d, causal, sm_scale, granularity, st, nullptr, 0,
+                                    sv, vm);
   nvtxRangePop();
   const cudaError_t fe = cudaFreeAsync(ws, st);
   if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;

@@ -275,6 +275,189 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
   quant_block<D, G, SMOOTH>(x, km, q, scale, N, rows, blockIdx.x);
 }
 
+// ---------------------------------------------------------------- V to FP8 (E4M3)
+// The FP8 P.V variant (SageAttention2 abstract: (P~, V) quantized to FP8, V smoothed): per
+// (b,h) and channel c,
+//   vm = fl32(fl32(S_c) / N) * 2^-24 from the exact sum S_c of V[t][c] * 2^24 (SMOOTH; else 0),
+//   a  = max_t |fl32(V[t][c] - vm)|,  sv = fl32(a / 448),  inv = fl32(448 / a)  (a = 0: 0, 0),
+//   v8 = e4m3(fl32(fl32(V - vm) * inv)), round to nearest even, saturating at +-448.
+// One cluster of C CTAs per head (as smooth_k_kernel) in two passes over the head's tokens:
+// pass 1 sums (the exact split of split_acc) and takes the channel maximum and minimum of V; the
+// CTAs exchange their partials through distributed shared memory and each derives vm, a, sv and
+// inv itself; pass 2 re-reads its token slice (now mostly from L2) and writes the codes.  The
+// absmax needs no third pass: fl32(x - vm) is monotonic in x, so
+// a = max(fl32(max V - vm), fl32(vm - min V)).
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;  // cvt packs its first source into the upper byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+template <int D, bool SMOOTH>
+__global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __half* __restrict__ v,
+                                                                     uint8_t* __restrict__ v8, float* __restrict__ sv,
+                                                                     float* __restrict__ vm, int N) {
+  constexpr int T = D / 8;                 // threads per token row (one 16-byte piece each)
+  constexpr int R = kSmoothThreads / T;    // rows per pass
+  constexpr int U = 4;                     // passes in flight
+  constexpr int WARPS = kSmoothThreads / 32;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int n_ctas = static_cast<int>(cluster.num_blocks());
+  const int bh = static_cast<int>(blockIdx.x) / n_ctas;
+  const int piece = threadIdx.x % T;
+  const int row = threadIdx.x / T;
+  const int slice = (N + n_ctas - 1) / n_ctas;
+  const int t0 = rank * slice;
+  const int t1 = min(N, t0 + slice);
+  const __half* base = v + (static_cast<size_t>(bh) * N) * D + piece * 8;
+
+  // ---- pass 1: exact sums, maxima and minima of this thread's 8 channels over its rows
+  long long acc[8];
+  float mx[8], mn[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    acc[i] = 0;
+    mx[i] = -INFINITY;
+    mn[i] = INFINITY;
+  }
+  constexpr int ITERS = kSplitFlushTokens / U;
+  for (int t = t0 + row; t < t1;) {
+    int hs[8];
+    float2 ls[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hs[i] = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
+    for (int it = 0; it < ITERS && t < t1; ++it, t += U * R) {
+      uint4 w[U];
+      bool live[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        live[u] = t + u * R < t1;
+        w[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D))
+                       : make_uint4(0u, 0u, 0u, 0u);  // +0.0 adds nothing; kept out of max / min below
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if constexpr (SMOOTH) split_acc(words[i], hs[2 * i], hs[2 * i + 1], ls[i]);
+          if (live[u]) {
+            const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&words[i]));
+            mx[2 * i] = fmaxf(mx[2 * i], x.x);
+            mx[2 * i + 1] = fmaxf(mx[2 * i + 1], x.y);
+            mn[2 * i] = fminf(mn[2 * i], x.x);
+            mn[2 * i + 1] = fminf(mn[2 * i + 1], x.y);
+          }
+        }
+      }
+    }
+    if constexpr (SMOOTH) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += (static_cast<long long>(hs[2 * i]) << 18) + __float2int_rn(__fmul_rn(ls[i].x, 16777216.0f));
+        acc[2 * i + 1] += (static_cast<long long>(hs[2 * i + 1]) << 18) + __float2int_rn(__fmul_rn(ls[i].y, 16777216.0f));
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int off = T; off < 32; off <<= 1) {
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], off));
+      mn[i] = fminf(mn[i], __shfl_xor_sync(0xffffffffu, mn[i], off));
+    }
+  }
+  __shared__ long long part[WARPS][T][8];
+  __shared__ float pmax[WARPS][T][8], pmin[WARPS][T][8];
+  __shared__ long long csum[D];  // this CTA's channel partials, read by every CTA of the cluster
+  __shared__ float cmax[D], cmin[D];
+  __shared__ float s_vm[D], s_inv[D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < T) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      part[warp][lane][i] = acc[i];
+      pmax[warp][lane][i] = mx[i];
+      pmin[warp][lane][i] = mn[i];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int p = threadIdx.x >> 3, i = threadIdx.x & 7;  // channel = p*8 + i = threadIdx.x
+    long long s = 0;
+    float a = -INFINITY, b = INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      s += part[w][p][i];
+      a = fmaxf(a, pmax[w][p][i]);
+      b = fminf(b, pmin[w][p][i]);
+    }
+    csum[threadIdx.x] = s;
+    cmax[threadIdx.x] = a;
+    cmin[threadIdx.x] = b;
+  }
+  cluster.sync();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    long long s = 0;
+    float hi = -INFINITY, lo = INFINITY;
+    for (int r = 0; r < n_ctas; ++r) {
+      s += *cluster.map_shared_rank(csum + c, r);
+      hi = fmaxf(hi, *cluster.map_shared_rank(cmax + c, r));
+      lo = fminf(lo, *cluster.map_shared_rank(cmin + c, r));
+    }
+    float mean = 0.f;
+    if constexpr (SMOOTH) mean = __fmul_rn(__fdiv_rn(__ll2float_rn(s), static_cast<float>(N)), 5.9604644775390625e-08f);
+    const float a = fmaxf(0.f, fmaxf(__fsub_rn(hi, mean), __fsub_rn(mean, lo)));
+    float scale = 0.f, inv = 0.f;
+    if (a > 0.f) {
+      scale = __fdiv_rn(a, 448.0f);
+      inv = __fdiv_rn(448.0f, a);
+    }
+    s_vm[c] = mean;
+    s_inv[c] = inv;
+    if (rank == 0) {
+      sv[static_cast<size_t>(bh) * D + c] = scale;
+      if constexpr (SMOOTH) vm[static_cast<size_t>(bh) * D + c] = mean;
+    }
+  }
+  cluster.sync();  // every CTA keeps its partials in place until all have read them
+
+  // ---- pass 2: codes of this CTA's token slice
+  float m8[8], i8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    m8[i] = s_vm[piece * 8 + i];
+    i8[i] = s_inv[piece * 8 + i];
+  }
+  uint8_t* out = v8 + (static_cast<size_t>(bh) * N) * D + piece * 8;
+  for (int t = t0 + row; t < t1; t += U * R) {
+    uint4 w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      w[u] = (t + u * R < t1) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D))
+                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (t + u * R >= t1) continue;
+      float x[8];
+      unpack8(w[u], x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if constexpr (SMOOTH) x[i] = __fsub_rn(x[i], m8[i]);
+        x[i] = __fmul_rn(x[i], i8[i]);
+      }
+      *reinterpret_cast<uint2*>(out + static_cast<size_t>(t + u * R) * D) =
+          make_uint2(e4m3x4(x[0], x[1], x[2], x[3]), e4m3x4(x[4], x[5], x[6], x[7]));
+    }
+  }
+}
+
 // ---------------------------------------------------------------- launchers
 template <int D>
 static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cudaStream_t st) {
@@ -293,6 +476,32 @@ static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cu
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, smooth_k_kernel<D>, k, km, N);
+}
+
+template <int D>
+static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N,
+                                        cudaStream_t st) {
+  int ctas = 1;  // the cluster size of smooth_k: >= kSmoothTokensPerCta tokens per CTA, at most 8
+  while (ctas < kSmoothMaxCtas && N / (2 * ctas) >= kSmoothTokensPerCta) ctas *= 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas) * static_cast<unsigned>(BH));
+  cfg.blockDim = dim3(kSmoothThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (vm) return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, true>, v, v8, sv, vm, N);
+  return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, false>, v, v8, sv, vm, N);
+}
+
+cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N, int D,
+                               cudaStream_t st) {
+  return D == 128 ? launch_quant_v_fp8_d<128>(v, v8, sv, vm, BH, N, st) : launch_quant_v_fp8_d<64>(v, v8, sv, vm, BH, N, st);
 }
 
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st) {

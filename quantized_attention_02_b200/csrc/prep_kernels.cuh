@@ -8,6 +8,9 @@ namespace sage {
 
 // km[bh, c] = mean over N tokens of k[bh, :, c]; k fp16 [BH, N, D], km fp32 [BH, D].
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st);
+// V to E4M3 with per-(head, channel) scales sv; vm: channel means (V smoothed) or nullptr (not smoothed).
+cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N, int D,
+                               cudaStream_t st);
 
 // Quantize q and k fp16 [BH, N, D] to int8 q8 / k8 with fp32 scales sq / sk (one launch per
 // tensor): per token (per_token), else in groups of 128 Q tokens and 64 K tokens.  km (fp32 [BH, D])
