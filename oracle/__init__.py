@@ -29,6 +29,11 @@ Parity status (which functions are pinned by checks other than themselves):
                     brute-force nearest search; exact rational scales and mean; hand-
                     derived two-key cases in tests/golden; the P~-rounding bound against
                     textbook attention; V-shift invariance; causal row 0)
+  sparse_predict, attn_sparse, attn_sparse_tiles (block-sparse variant, SpargeAttn
+                    abstract; sage_oracle_sparse.c) ... pinned (the dense oracle when every
+                    block is kept; textbook attention over the kept keys; a numpy re-
+                    derivation of the predicted map; closed forms of the self-similarity;
+                    hand-built second-stage cases; limits of tau and theta)
 Every pin is itself checked by tests/test_oracle_mutations.py: planted slips
 (dropped or re-routed roundings, signs, indices, group sizes, operands), each of which
 makes the pins fail.
@@ -45,7 +50,7 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, f) for f in ("sage_oracle.c", "sage_oracle_sa2.c")]
+_SRCS = [os.path.join(_HERE, f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c")]
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "libsage_oracle.so")
 _lock = threading.Lock()
@@ -98,6 +103,14 @@ def _load():
                                                    i64, vp]
             for name in ("oracle_quant_v_fp8", "oracle_attn_fp8pv", "oracle_attn_fp8pv_rows"):
                 getattr(lib, name).restype = i32
+            lib.oracle_sparse_predict.argtypes = [vp, vp, i64, i64, i64, i32, f64, f64, f64, f64, vp, vp, vp, vp]
+            lib.oracle_sparse_predict.restype = i32
+            lib.oracle_attn_sparse.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f64, i64, i64, vp, f64, vp,
+                                               vp, vp]
+            lib.oracle_attn_sparse.restype = i32
+            lib.oracle_attn_sparse_tiles.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp, f64, vp,
+                                                     i64, vp, vp]
+            lib.oracle_attn_sparse_tiles.restype = i32
             for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_qk_int_rows", "oracle_attn",
                          "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
                 getattr(lib, name).restype = i32
@@ -364,6 +377,75 @@ def sage_attn_fp8pv(q, k, v, causal: bool, sm_scale: float, per_block: bool, smo
     v8, sv, vm = quant_v_fp8(v, smooth_v)
     o64, o16 = attn_fp8pv(q8, k8, sq, sk, v8, sv, vm, causal, sm_scale, (gq, gk))
     return dict(km=km, q8=q8, sq=sq, k8=k8, sk=sk, v8=v8, sv=sv, vm=vm, o64=o64, o16=o16)
+
+
+# ------------------------------------------------------------------ block-sparse variant
+# (SpargeAttn abstract: a first stage that predicts the attention map and skips matrix
+# products, a second softmax-aware stage that skips more; readings in sage_oracle_sparse.c)
+SPARSE_BQ, SPARSE_BK = 256, 128
+
+
+def sparse_predict(q, k, causal: bool, sm_scale: float, tau: float, theta: float, eps: float = 1e-4):
+    """Stage 1: the kept (query block of 256, key block of 128) pairs.  Returns (mask uint8
+    [*lead, NQB, NKB], unsure uint8 (decisions within eps of flipping), qsim [*lead, NQB],
+    ksim [*lead, NKB])."""
+    qb, kb = _as_fp16_bits(q), _as_fp16_bits(k)
+    BH, N, d = _bhnd(qb)
+    nqb, nkb = -(-N // SPARSE_BQ), -(-N // SPARSE_BK)
+    lead = qb.shape[:-2]
+    mask = np.empty(lead + (nqb, nkb), np.uint8)
+    unsure = np.empty(lead + (nqb, nkb), np.uint8)
+    qsim = np.empty(lead + (nqb,), np.float64)
+    ksim = np.empty(lead + (nkb,), np.float64)
+    _check(_load().oracle_sparse_predict(_ptr(qb), _ptr(kb), BH, N, d, int(bool(causal)), float(sm_scale),
+                                         float(tau), float(theta), float(eps), _ptr(mask), _ptr(unsure), _ptr(qsim),
+                                         _ptr(ksim)), "oracle_sparse_predict")
+    return mask, unsure, qsim, ksim
+
+
+def attn_sparse(q8, k8, sq, sk, v, mask, causal: bool, sm_scale: float, lam: float, groups=GROUP_PER_TOKEN):
+    """Block-sparse quantized attention over the kept blocks of `mask`, with the stage-2 filter
+    lam (log2 units; inf = none).  Returns (O fp64, O fp16, skipped uint8 [*lead, NQT, NKB])."""
+    q8 = np.ascontiguousarray(q8, np.int8)
+    k8 = np.ascontiguousarray(k8, np.int8)
+    sq = np.ascontiguousarray(sq, np.float32)
+    sk = np.ascontiguousarray(sk, np.float32)
+    vb = _as_fp16_bits(v)
+    BH, N, d = _bhnd(vb)
+    mask = np.ascontiguousarray(mask, np.uint8)
+    if mask.size != BH * (-(-N // SPARSE_BQ)) * (-(-N // SPARSE_BK)):
+        raise ValueError("mask must be [BH, ceil(N/256), ceil(N/128)]")
+    nqt = -(-N // 128)
+    o64 = np.empty(vb.shape, np.float64)
+    o16 = np.empty(vb.shape, np.uint16)
+    skipped = np.empty(vb.shape[:-2] + (nqt, -(-N // SPARSE_BK)), np.uint8)
+    gq, gk = groups
+    _check(_load().oracle_attn_sparse(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(vb), BH, N, d, int(bool(causal)),
+                                      float(sm_scale), gq, gk, _ptr(mask), float(lam), _ptr(o64), _ptr(o16),
+                                      _ptr(skipped)), "oracle_attn_sparse")
+    return o64, o16.view(np.float16), skipped
+
+
+def attn_sparse_tiles(q8h, k8h, sqh, skh, vh, maskh, tiles, causal: bool, sm_scale: float, lam: float,
+                      groups=GROUP_PER_TOKEN):
+    """attn_sparse() for the listed 128-row query tiles of one head [N, d] only.  Returns
+    (O fp64 [len(tiles), 128, d] -- rows past N are NaN --, skipped uint8 [len(tiles), NKB])."""
+    q8h = np.ascontiguousarray(q8h, np.int8)
+    k8h = np.ascontiguousarray(k8h, np.int8)
+    sqh = np.ascontiguousarray(sqh, np.float32)
+    skh = np.ascontiguousarray(skh, np.float32)
+    vb = _as_fp16_bits(vh)
+    N, d = vb.shape
+    maskh = np.ascontiguousarray(maskh, np.uint8)
+    tiles = np.ascontiguousarray(tiles, np.int64)
+    o64 = np.full((tiles.size, 128, d), np.nan, np.float64)
+    skipped = np.empty((tiles.size, -(-N // SPARSE_BK)), np.uint8)
+    gq, gk = groups
+    _check(_load().oracle_attn_sparse_tiles(_ptr(q8h), _ptr(k8h), _ptr(sqh), _ptr(skh), _ptr(vb), N, d,
+                                            int(bool(causal)), float(sm_scale), gq, gk, _ptr(maskh), float(lam),
+                                            _ptr(tiles), tiles.size, _ptr(o64), _ptr(skipped)),
+           "oracle_attn_sparse_tiles")
+    return o64, skipped
 
 
 def metrics(a: np.ndarray, b: np.ndarray) -> dict:

@@ -3,7 +3,7 @@
 Each case plants one plausible slip in a copy of the oracle's C sources (a dropped
 rounding, a rounding taken another way, a wrong sign, index, group size, offset or
 operand), builds the copy with the oracle's own compiler flags, and runs the pin
-files (tests/test_oracle_pins.py, tests/test_oracle_pins_fp8.py) against it in a
+files (tests/test_oracle_pins*.py) against it in a
 fresh process (the oracle package loads
 the library named by SAGE_ORACLE_LIB).  The pins must fail on every mutant, and
 pass on an unmodified copy built the same way (the control case), so a pin that
@@ -11,7 +11,8 @@ cannot tell a slip from the reading it pins shows up here.
 
 The readings pinned are those of the SageAttention summary page (Summary bullets
 1-2: INT8 Q.K^T after smoothing K, P.V in fp16; idea I1: the K shift) and of the
-SageAttention2 abstract for the FP8 P.V variant (E4M3 P~ and V, V smoothing).
+SageAttention2 abstract for the FP8 P.V variant (E4M3 P~ and V, V smoothing) and of
+the SpargeAttn abstract for the block-sparse variant (predicted map, softmax-aware skip).
 """
 import concurrent.futures
 import os
@@ -21,8 +22,9 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRCS = {f: os.path.join(ROOT, "oracle", f) for f in ("sage_oracle.c", "sage_oracle_sa2.c")}
-PINS = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_pins_fp8.py")]
+SRCS = {f: os.path.join(ROOT, "oracle", f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c")}
+PINS = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_pins_fp8.py",
+                                                 "test_oracle_pins_sparse.py")]
 
 # (name, text in sage_oracle.c, replacement, expected number of occurrences)
 BASE_MUTATIONS = [
@@ -71,7 +73,26 @@ FP8_MUTATIONS = [
     ("e4m3_decode_bias", "ldexp(1.0 + F / 8.0, E - 7)", "ldexp(1.0 + F / 8.0, E - 8)", 1),
 ]
 
-MUTATIONS = [("sage_oracle.c",) + m for m in BASE_MUTATIONS] + [("sage_oracle_sa2.c",) + m for m in FP8_MUTATIONS]
+# (name, text in sage_oracle_sparse.c, replacement, expected number of occurrences)
+SPARSE_MUTATIONS = [
+    ("sparse_sort_ascending", "(p[order[b - 1]] < p[a] ||", "(p[order[b - 1]] > p[a] ||", 1),
+    ("sparse_no_causal_diagonal", "if (causal && (j + 1) * BK > i * BQ) mrow[j] = 1;", "", 1),
+    ("sparse_similarity_override_inverted", "if (!q_alike || ks[j] < theta) mrow[j] = 1;",
+     "if (!q_alike || ks[j] > theta) mrow[j] = 1;", 1),
+    ("sparse_similarity_over_n", "return s2 / ((double)n * (double)n);", "return s2 / (double)n;", 1),
+    ("sparse_sum_not_mean", "mean[c] /= (double)n;", "", 1),
+    ("sparse_cut_one_short", "while (cut < nvis && cum < tau)", "while (cut < nvis && cum + p[order[cut]] < tau)", 1),
+    ("sparse_last_visible_block_dropped", "const int64_t nvis = causal ? last_q / BK + 1 : NKB;",
+     "const int64_t nvis = causal ? last_q / BK : NKB;", 1),
+    ("stage2_lambda_sign", "if (!(m < mrun[i - r0] - lambda)) skip = 0;", "if (!(m < mrun[i - r0] + lambda)) skip = 0;", 1),
+    ("stage2_running_max_starts_at_zero", "mrun[i - r0] = -INFINITY;", "mrun[i - r0] = 0.0;", 1),
+    ("stage2_running_max_frozen", "if (bmax[i - r0] > mrun[i - r0]) mrun[i - r0] = bmax[i - r0];", ";", 1),
+    ("stage2_skipped_keys_still_used", "            continue;\n        }\n        used[b] = 1;",
+     "        }\n        used[b] = 1;", 1),
+]
+
+MUTATIONS = ([("sage_oracle.c",) + m for m in BASE_MUTATIONS] + [("sage_oracle_sa2.c",) + m for m in FP8_MUTATIONS]
+             + [("sage_oracle_sparse.c",) + m for m in SPARSE_MUTATIONS])
 
 CFLAGS = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
 

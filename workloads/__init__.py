@@ -18,6 +18,11 @@ this order, all in fp32, then rounded to fp16):
   5. outlier signs: +-1 uniformly per (b,h, outlier)
   6. V      ~ N(0, 1)                            shape [B,H,N,d]
   K = noise + bias, where the outlier channels' bias is replaced by sign * mag.
+Windowed (block-sparse) workloads, window > 0, draw one more tensor after V:
+  7. u      ~ N(0, 1), each row scaled to unit length, shape [B,H,ceil(N/window),d]
+  and add align * u[t // window] to both Q and K: tokens of one window share a direction, so the
+  attention concentrates inside windows -- the locality of the video-DiT inputs the sparse
+  attention pages evaluate on (SpargeAttn abstract: attention maps are often sparse).
 """
 from __future__ import annotations
 
@@ -40,6 +45,8 @@ class Workload:
     bias_std: float = 1.0
     n_out: int = 0
     out_mag: float = 0.0
+    window: int = 0        # > 0: tokens in windows of this many share a direction of length align
+    align: float = 0.0
 
     @property
     def BH(self) -> int:
@@ -58,7 +65,9 @@ class Workload:
         g = "per-block 128Q/64K" if self.per_block else "per-token"
         return (f"B={self.B},H={self.H},N={self.N},d={self.d} {'causal' if self.causal else 'non-causal'}, "
                 f"{g}, Q~N(0,{self.q_std}^2), K~N(0,1)+bias(N(0,{self.bias_std}^2)"
-                + (f", {self.n_out} ch +-{self.out_mag:g}" if self.n_out else "") + "), V~N(0,1)")
+                + (f", {self.n_out} ch +-{self.out_mag:g}" if self.n_out else "") + "), V~N(0,1)"
+                + (f", Q and K + {self.align:g} x a unit direction shared by each window of {self.window} tokens"
+                   if self.window else ""))
 
 
 # The five workload families: a tiny per-token case, a small causal per-block
@@ -89,7 +98,13 @@ PROFILE64 = Workload("profile_b1h16_n16384_d64", 1, 16, 16384, 64, False, True, 
 TOKEN128 = Workload("token_n16384_d128_full", 1, 64, 16384, 128, False, False, n_out=4, out_mag=20.0)
 TOKEN64 = Workload("token_n16384_d64_full", 1, 64, 16384, 64, False, False, n_out=4, out_mag=20.0)
 
-ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64)}
+# block-sparse stand-in for the video-DiT attention maps (SpargeAttn abstract): the headline
+# shape with windows of 2048 tokens (16 key tiles) whose Q and K share a direction of length 14
+# (in-window scores about 17 above the rest, natural log units, at d^-1/2 = 0.088)
+SPARSE = Workload("sparse_n16384_d128_win2048", 1, 64, 16384, 128, False, True, window=2048, align=14.0)
+SPARSE_CAUSAL = Workload("sparse_n16384_d128_win2048_causal", 1, 64, 16384, 128, True, True, window=2048, align=14.0)
+
+ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64, SPARSE, SPARSE_CAUSAL)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
@@ -111,6 +126,13 @@ def make_qkv(w: Workload, seed: int = 0):
         bias.view(w.B, w.H, w.d).scatter_(-1, perm, signs * w.out_mag)
     k += bias
     v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if w.window:
+        n_win = -(-w.N // w.window)
+        u = torch.randn((w.B, w.H, n_win, w.d), generator=g, dtype=torch.float32)
+        u = u / u.norm(dim=-1, keepdim=True)
+        shared = u[:, :, torch.arange(w.N) // w.window] * w.align
+        q += shared
+        k += shared
     return q.half().contiguous(), k.half().contiguous(), v.half().contiguous()
 
 
