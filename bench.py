@@ -281,6 +281,11 @@ def run_ours(args, w: W.Workload):
             dist.barrier()
 
     fp8 = args.variant == "fp8pv"
+    sparse = args.variant == "sparse"
+    if sparse:  # the block lists of stage 1 for the sparse variant's kernel-only timing
+        nqb, nkb = sa.sparse_blocks(w.N)
+        kv_cnt = torch.zeros((w.B, w.H, nqb), dtype=torch.int32, device=dev)
+        kv_idx = torch.zeros((w.B, w.H, nqb, nkb), dtype=torch.int16, device=dev)
     if fp8:  # E4M3 V codes, per-channel scales and means for the FP8 P.V variant's kernel-only timing
         v8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
         sv = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
@@ -289,12 +294,18 @@ def run_ours(args, w: W.Workload):
     def step():
         if fp8:
             sa.sage_attn_fwd_fp8pv(q, k, v, o, w.causal, w.sm_scale, gran, stream)
+        elif sparse:
+            sa.sage_attn_fwd_sparse(q, k, v, o, w.causal, w.sm_scale, gran, args.tau, args.theta, args.skip_lambda,
+                                    stream)
         else:
             sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
 
     def fused():
         if fp8:
             sa.sage_attn_fwd_fp8pv_quantized(q8, k8, sq, sk, v8, sv, vm, o, w.causal, w.sm_scale, gran, stream)
+        elif sparse:
+            sa.sage_attn_fwd_sparse_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, kv_cnt, kv_idx,
+                                              args.skip_lambda, stream)
         else:
             sa.sage_attn_fwd_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, stream)
 
@@ -340,6 +351,8 @@ def run_ours(args, w: W.Workload):
     sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream)
     if fp8:
         sa.sage_quant_v_fp8(v, v8, sv, vm, stream)
+    if sparse:
+        sa.sage_sparse_predict(q, k, w.causal, w.sm_scale, args.tau, args.theta, kv_cnt, kv_idx, stream)
     for _ in range(3):
         fused()
     torch.cuda.synchronize(dev)
@@ -371,6 +384,15 @@ def run_ours(args, w: W.Workload):
     }
     if fp8:
         breakdown["quant_v_fp8_ms"] = timed(lambda: sa.sage_quant_v_fp8(v, v8, sv, vm, stream), nb)
+    density = None
+    if sparse:
+        breakdown["sparse_predict_ms"] = timed(
+            lambda: sa.sage_sparse_predict(q, k, w.causal, w.sm_scale, args.tau, args.theta, kv_cnt, kv_idx, stream), nb)
+        # share of the dense Q.K^T work stage 1 keeps: kept (256-query, 128-key) block pairs over
+        # the visible ones (the causal diagonal blocks counted as whole blocks on both sides)
+        nqb_, nkb_ = sa.sparse_blocks(w.N)
+        vis = [(min(w.N, (i + 1) * 256) - 1) // 128 + 1 if w.causal else nkb_ for i in range(nqb_)]
+        density = float(kv_cnt.sum().item()) / (w.BH * sum(vis))
 
     # ---- end to end through the C ABI with host buffers: H2D inputs, D2H output per step
     qp, kp, vp = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
@@ -378,7 +400,7 @@ def run_ours(args, w: W.Workload):
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
-        if fp8:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
+        if fp8 or sparse:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
             q.copy_(qp, non_blocking=True)
             k.copy_(kp, non_blocking=True)
             v.copy_(vp, non_blocking=True)
@@ -414,10 +436,12 @@ def run_ours(args, w: W.Workload):
         # P.V runs at the FP8 rate (2 x FP16, as INT8): its roofline is the INT8 one.
         peak_of = (lambda p: 2.0 * p) if fp8 else mixed_peak_tops
         peak = peak_of(p_burst)
-        achieved = ops / (kernel_ms * 1e-3) / 1e12
+        # executed work: the sparse variant runs the kept share of the blocks (value stays the
+        # dense-equivalent rate, the way block-sparse attention speedups are quoted)
+        achieved = ops * (density if sparse else 1.0) / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
         accuracy = None
-        if args.no_cpu_baseline or world > 1 or fp8:  # the CPU baseline belongs to the N=1 headline line only
+        if args.no_cpu_baseline or world > 1 or fp8 or sparse:  # the CPU baseline belongs to the N=1 headline line only
             cpu_tops, cores, desc = None, None, ("skipped" if world == 1 else "rank 0 at N=1 only")
         else:
             cpu_tops, cores, desc, sample = oracle_sample(w, keep=True)
@@ -429,7 +453,10 @@ def run_ours(args, w: W.Workload):
             "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3" if fp8 else "int8+f16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
-                       "variant": "fp8 P.V (E4M3 P~ and V, V smoothed)" if fp8 else "fp16 P.V",
+                       "variant": ("fp8 P.V (E4M3 P~ and V, V smoothed)" if fp8 else
+                                   (f"block-sparse (tau {args.tau}, theta {args.theta}, lambda {args.skip_lambda}); "
+                                    f"stage-1 kept share {density:.4f}; value = dense-equivalent TOPS" if sparse
+                                    else "fp16 P.V")),
                        "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default); no flush needed",
                        "parallelism": (f"heads sharded over {world} ranks ({w.BH} per rank, "
                                        f"global B*H = {world * w.BH}); no data-path collective")},
@@ -450,7 +477,7 @@ def run_ours(args, w: W.Workload):
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
             "accuracy": accuracy,
-            "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0)) * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0) + (2 if sparse else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
     if world > 1:
@@ -498,8 +525,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
-    ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv"],
-                    help="fp16pv: the SageAttention method (P.V in fp16); fp8pv: its FP8 P.V variant (d=128)")
+    ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv", "sparse"],
+                    help="fp16pv: the SageAttention method (P.V in fp16); fp8pv: its FP8 P.V variant (d=128); "
+                         "sparse: the block-sparse variant (d=128; use a sparse_* workload)")
+    ap.add_argument("--tau", type=float, default=0.99, help="sparse: cumulative probability kept by stage 1")
+    ap.add_argument("--theta", type=float, default=0.3, help="sparse: self-similarity below which a block is kept")
+    ap.add_argument("--skip-lambda", type=float, default=20.0, help="sparse: stage-2 threshold (log2 units)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiler runs)")
     args = ap.parse_args(argv)

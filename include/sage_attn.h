@@ -129,6 +129,45 @@ int sage_attn_fwd_fp8pv_quantized(const int8_t* q8, const int8_t* k8, const floa
 int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                         int causal, float sm_scale, int granularity, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Block-sparse variant, following the SpargeAttn abstract (author pages of Jia Wei and Haofeng
+ * Huang; arXiv 2502.18137): a sparse and quantized attention with a two-stage online filter.
+ * Stage 1 predicts the attention map at block level and skips the products of the blocks it
+ * drops; stage 2, inside the online softmax, skips the P.V product (and the exp2 work) of a block
+ * whose scores all lie far below the running row maximum.  Head dimension 128 and N <= 65536
+ * (SAGE_ERR_UNSUPPORTED otherwise); P.V in fp16 as in sage_attn_fwd.
+ *
+ * Stage 1 (sage_sparse_predict): query blocks of 256 tokens (QB = ceil(N/256) per (b,h)) and key
+ * blocks of 128 tokens (KB = ceil(N/128)).  Each block is represented by the mean of its tokens;
+ * the predicted map of a query block is softmax_j(q_mean . k_mean_j * sm_scale) over the key
+ * blocks it may see (causal: those starting at or before its last query).  Kept: the fewest key
+ * blocks, in decreasing predicted probability (ties: lower index first), whose probabilities sum
+ * to at least tau (0 < tau <= 1); every visible key block when the query block's self-
+ * similarity (the mean cosine over ordered pairs of its tokens) is below theta; every key block
+ * whose self-similarity is below theta; causal: the blocks holding the query block's own keys.
+ * q, k: fp16 [B,H,N,d] (in); kv_count: int [B,H,QB] (out, the number of kept key blocks);
+ * kv_index: int16 [B,H,QB,KB] (out, the kept key blocks in increasing order, entries past the
+ * count left unchanged).  Allocates a small stream-ordered workspace (block means). */
+int sage_sparse_predict(const void* q, const void* k, int B, int H, int N, int d, int causal, float sm_scale,
+                        float tau, float theta, int* kv_count, int16_t* kv_index, void* stream);
+
+/* The fused kernel of the block-sparse variant on quantized inputs: as sage_attn_fwd_quantized
+ * over the kept key blocks of kv_count / kv_index (any ascending lists; causal lists must hold
+ * the blocks with each query's own key), plus stage 2: a query tile of 128 rows drops key block
+ * j when, for each of its rows below N, the block's largest score (log2 units) lies more than
+ * skip_lambda below the row's largest score over the blocks it visited before (its first block
+ * is never dropped).  skip_lambda > 0; +INFINITY turns stage 2 off. */
+int sage_attn_fwd_sparse_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
+                                   const void* v, void* o, int B, int H, int N, int d, int causal, float sm_scale,
+                                   int granularity, const int* kv_count, const int16_t* kv_index, float skip_lambda,
+                                   void* stream);
+
+/* The whole block-sparse variant as a user calls it: stage-1 prediction, smooth K, INT8 Q and K,
+ * the fused kernel with stage 2.  Workspace as sage_attn_fwd plus the block lists. */
+int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                         int causal, float sm_scale, int granularity, float tau, float theta, float skip_lambda,
+                         void* stream);
+
 /* Debug: the full integer product s[b,h,i,j] = sum_c q8[b,h,i,c] * k8[b,h,j,c] as int32
  * (exact: |s| <= 128*127*127 < 2^31), computed with the same tensor-core path as the fused
  * kernel.  s: int32 [B,H,N,N] (out); needs B*H*N*N < 2^31. */

@@ -56,6 +56,10 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_quant_v_fp8.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
         lib.sage_attn_fwd_fp8pv_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_attn_fwd_fp8pv.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_sparse_predict.argtypes = [_p, _p, _i, _i, _i, _i, _i, _f, _f, _f, _p, _p, _p]
+        lib.sage_attn_fwd_sparse_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _p, _f,
+                                                       _p]
+        lib.sage_attn_fwd_sparse.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _f, _f, _f, _p]
         lib.sage_last_device_error.argtypes = [_p]
         lib.sage_attn_fwd_noalloc.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_noalloc_scratch_bytes.argtypes = [_i, _i, _i, _i, _i]
@@ -68,7 +72,8 @@ def get_lib() -> ctypes.CDLL:
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
                   "sage_debug_attn_trace", "sage_debug_mma_peak", "sage_attn_fwd_host",
                   "sage_debug_wait_timeout", "sage_quant_v_fp8", "sage_attn_fwd_fp8pv_quantized",
-                  "sage_attn_fwd_fp8pv"):
+                  "sage_attn_fwd_fp8pv", "sage_sparse_predict", "sage_attn_fwd_sparse_quantized",
+                  "sage_attn_fwd_sparse"):
             getattr(lib, n).restype = _i
         _lib = lib
     return _lib
@@ -170,6 +175,38 @@ def sage_attn_fwd_fp8pv(q, k, v, o, causal: bool, sm_scale: float, granularity: 
     B, H, N, d = _shape(q)
     _check(get_lib().sage_attn_fwd_fp8pv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
                                          float(sm_scale), int(granularity), _stream(stream)), "sage_attn_fwd_fp8pv")
+
+
+def sparse_blocks(N: int) -> tuple[int, int]:
+    """(query blocks, key blocks) of the block-sparse variant: ceil(N/256), ceil(N/128)."""
+    return (N + 255) // 256, (N + 127) // 128
+
+
+def sage_sparse_predict(q, k, causal: bool, sm_scale: float, tau: float, theta: float, kv_count, kv_index,
+                        stream=None) -> None:
+    """Stage 1 of the block-sparse variant (SpargeAttn abstract): kv_count int32 [B,H,QB] and
+    kv_index int16 [B,H,QB,KB] receive each query block's kept key blocks."""
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_sparse_predict(_ptr(q), _ptr(k), B, H, N, d, int(bool(causal)), float(sm_scale), float(tau),
+                                         float(theta), _ptr(kv_count), _ptr(kv_index), _stream(stream)),
+           "sage_sparse_predict")
+
+
+def sage_attn_fwd_sparse_quantized(q8, k8, sq, sk, v, o, causal: bool, sm_scale: float, granularity: int, kv_count,
+                                   kv_index, skip_lambda: float, stream=None) -> None:
+    B, H, N, d = _shape(v)
+    _check(get_lib().sage_attn_fwd_sparse_quantized(_ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(v), _ptr(o), B, H, N,
+                                                    d, int(bool(causal)), float(sm_scale), int(granularity),
+                                                    _ptr(kv_count), _ptr(kv_index), float(skip_lambda),
+                                                    _stream(stream)), "sage_attn_fwd_sparse_quantized")
+
+
+def sage_attn_fwd_sparse(q, k, v, o, causal: bool, sm_scale: float, granularity: int, tau: float, theta: float,
+                         skip_lambda: float, stream=None) -> None:
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_attn_fwd_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+                                          float(sm_scale), int(granularity), float(tau), float(theta),
+                                          float(skip_lambda), _stream(stream)), "sage_attn_fwd_sparse")
 
 
 def sage_debug_qk_int32(q8, k8, s, stream=None) -> None:

@@ -31,8 +31,10 @@ SOURCES = {
     "noalloc.cu": [],
     "host_pipeline.cu": [],
     "mma_rate.cu": [],
+    "sparse_kernels.cu": [],
 }
-HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh", "workspace.cuh"]
+HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh", "workspace.cuh",
+           "sparse_kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

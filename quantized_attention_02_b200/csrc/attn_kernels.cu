@@ -724,10 +724,10 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false, bool FP8 = false>
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false, bool FP8 = false, bool SPARSE = false>
 static cudaError_t launch_attn_v3(const AttnArgs& a, cudaStream_t st) {
   using L = V3LayoutT<FP8>;
-  auto kern = sage_attn_v3_kernel<CAUSAL, PER_TOKEN, TRACE, RAGGED, FP8>;
+  auto kern = sage_attn_v3_kernel<CAUSAL, PER_TOKEN, TRACE, RAGGED, FP8, SPARSE>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
@@ -737,7 +737,7 @@ static cudaError_t launch_attn_v3(const AttnArgs& a, cudaStream_t st) {
   const int n_pairs = ((a.N + L::BM - 1) / L::BM + 1) / 2;
   dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
   kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.sq, a.sk, a.BH, a.N, a.sm_scale_log2,
-                                          a.trace, a.trace_ctas, a.sv, a.vm);
+                                          a.trace, a.trace_ctas, a.sv, a.vm, a.kv_count, a.kv_index, a.skip_lambda);
   return cudaGetLastError();
 }
 
@@ -750,20 +750,24 @@ static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
   return a.per_token ? launch_attn_t<D, false, true, false, RAGGED>(a, st) : launch_attn_t<D, false, false, false, RAGGED>(a, st);
 }
 
-template <bool RAGGED, bool FP8 = false>
+template <bool RAGGED, bool FP8 = false, bool SPARSE = false>
 static cudaError_t launch_attn_128(const AttnArgs& a, cudaStream_t st) {
   if (a.causal)
-    return a.per_token ? launch_attn_v3<true, true, false, RAGGED, FP8>(a, st)
-                       : launch_attn_v3<true, false, false, RAGGED, FP8>(a, st);
-  return a.per_token ? launch_attn_v3<false, true, false, RAGGED, FP8>(a, st)
-                     : launch_attn_v3<false, false, false, RAGGED, FP8>(a, st);
+    return a.per_token ? launch_attn_v3<true, true, false, RAGGED, FP8, SPARSE>(a, st)
+                       : launch_attn_v3<true, false, false, RAGGED, FP8, SPARSE>(a, st);
+  return a.per_token ? launch_attn_v3<false, true, false, RAGGED, FP8, SPARSE>(a, st)
+                     : launch_attn_v3<false, false, false, RAGGED, FP8, SPARSE>(a, st);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   const bool ragged = a.N % 128 != 0;
   if (a.fp8) {  // the FP8 P.V variant: head dimension 128, untraced
-    if (a.D != 128 || a.trace) return cudaErrorNotSupported;
+    if (a.D != 128 || a.trace || a.kv_count) return cudaErrorNotSupported;
     return ragged ? launch_attn_128<true, true>(a, st) : launch_attn_128<false, true>(a, st);
+  }
+  if (a.kv_count) {  // the block-sparse variant: head dimension 128, untraced, up to 512 key tiles
+    if (a.D != 128 || a.trace || (a.N + 127) / 128 > V3Layout::MAX_LIST) return cudaErrorNotSupported;
+    return ragged ? launch_attn_128<true, false, true>(a, st) : launch_attn_128<false, false, true>(a, st);
   }
   if (a.trace) {  // traced builds exist for per-block granularity and whole tiles only
     if (a.per_token || ragged) return cudaErrorNotSupported;

@@ -25,6 +25,12 @@ struct AttnArgs {
   bool fp8 = false;
   const float* sv = nullptr;
   const float* vm = nullptr;
+  // block-sparse variant (D = 128, fp16 P.V): per CTA (head, pair of query tiles) the number of
+  // kept key tiles and their ascending list ([BH][ceil(N/256)][ceil(N/128)] int16); the stage-2
+  // threshold in log2 units (+inf: no stage 2)
+  const int* kv_count = nullptr;
+  const int16_t* kv_index = nullptr;
+  float skip_lambda = 0.f;
 };
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);

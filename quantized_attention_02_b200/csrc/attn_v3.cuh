@@ -40,7 +40,11 @@ struct V3LayoutT {
   // corr_done, drain, key scales staged, plus the Q.K^T warp's drain
   static constexpr int NUM_BARS = 1 + 2 * SK + 2 * SV + 10 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  // block-sparse variant: the CTA's key-tile list (int16, up to 512 tiles) and the skip votes
+  static constexpr int MAX_LIST = 512;
+  static constexpr int OFF_LIST = OFF_MISC + 16;
+  static constexpr int OFF_SKIP = OFF_LIST + MAX_LIST * 2;  // [2 tiles][3] group votes, [2 tiles][2] P.V flags
+  static constexpr int SMEM = OFF_SKIP + 64 + 1024;
   static constexpr int THREADS = 512;
 };
 using V3Layout = V3LayoutT<false>;
@@ -119,13 +123,24 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
 // P~ = 2^(s - m_use + 8), so P~ is rounded on the E4M3 grid of a power-of-two scaling of
 // exp(s - max s), as the oracle rounds it, and the offset moves as soon as the row maximum passes
 // it by half a unit (P~ <= 2^8.5 < 448); the epilogue applies sv and adds vm.
-template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED, bool FP8 = false>
+//
+// SPARSE = true is the block-sparse variant of the SpargeAttn abstract (a predicted map skips
+// products; a softmax-aware filter skips more).  kv_count[bh * n_pairs + pair] and the ascending
+// key-tile list kv_index[(bh * n_pairs + pair) * ceil(N/128) + i] say which key tiles the CTA
+// visits (stage 1); every role walks the list instead of 0 .. n_kv-1.  Stage 2: a softmax group
+// drops key tile j of its query tile when, for each of its rows below N, the tile's largest score
+// lies more than skip_lambda (log2 units) under the row's running maximum; the group agrees
+// through a vote and a named barrier, skips its exp2 pass, and its P.V warp issues nothing for
+// that tile (the tile adds to neither O nor l).
+template <bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED, bool FP8 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(512, 1)
     sage_attn_v3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                         const float* __restrict__ sq, const float* __restrict__ sk, int BH, int N,
                         float sm_scale_log2, long long* __restrict__ trace, int trace_ctas,
-                        const float* __restrict__ sv = nullptr, const float* __restrict__ vm = nullptr) {
+                        const float* __restrict__ sv = nullptr, const float* __restrict__ vm = nullptr,
+                        const int* __restrict__ kv_count = nullptr, const int16_t* __restrict__ kv_index = nullptr,
+                        float skip_lambda = 0.f) {
   using L = V3LayoutT<FP8>;
   constexpr int D = L::D;
   extern __shared__ uint8_t smem_raw[];
@@ -172,7 +187,28 @@ __global__ void __launch_bounds__(512, 1)
   int n_iter[2];
   n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
   n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
+  int16_t* sList = reinterpret_cast<int16_t*>(smem + L::OFF_LIST);
+  int* sSkipVote = reinterpret_cast<int*>(smem + L::OFF_SKIP);       // [2 tiles][3]: a row keeps the tile
+  int* sPvKeep = reinterpret_cast<int*>(smem + L::OFF_SKIP + 32);    // [2 tiles][2]: P.V of key tile j issued
+  if constexpr (SPARSE) {
+    // the list is ascending; causal lists end with the diagonal tiles, so tile 0 stops one key
+    // tile before tile 1 when the list holds tile0 + 1 (only tile 1 sees it)
+    // a malformed list (count or entries out of range) gives unspecified output, never an access
+    // outside the tensors: both are clamped into range
+    const int count = min(max(kv_count[static_cast<size_t>(bh) * n_pairs + pair], 0), min(n_kv_total, L::MAX_LIST));
+    const int16_t* lst = kv_index + (static_cast<size_t>(bh) * n_pairs + pair) * n_kv_total;
+    for (int i = threadIdx.x; i < count; i += L::THREADS)
+      sList[i] = static_cast<int16_t>(min(max(static_cast<int>(lst[i]), 0), n_kv_total - 1));
+    const int last = count > 0 ? min(max(static_cast<int>(lst[count - 1]), 0), n_kv_total - 1) : -1;
+    n_iter[1] = n_tiles > 1 ? count : 0;
+    n_iter[0] = (CAUSAL && n_tiles > 1 && last == tile0 + 1) ? count - 1 : count;
+  }
   const int n_kv = max(n_iter[0], n_iter[1]);
+  // key tile visited in step j
+  auto key_tile = [&](int j) -> int {
+    if constexpr (SPARSE) return sList[j];
+    return j;
+  };
   const int row_base = bh * N;
 
   long long* trace_row = nullptr;
@@ -215,6 +251,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar_sks, 128);
     mbar_init(bar_sks + 1, 128);
     for (int i = 0; i < 6; ++i) sFlag[i] = 0;
+    for (int i = 0; i < 6; ++i) sSkipVote[i] = 0;
     *abort_flag = 0;
     *arrived = 0;
     fence_barrier_init();
@@ -252,7 +289,7 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; t < n_tiles; ++t)
         tma_load_3d(sQ + t * L::Q_BYTES, &tm_q, bar_q, 0, (tile0 + t) * L::BM, bh);
       for (int j = 0; j < n_kv; ++j) {
-        const int key_row = j * L::BN;  // token row within the head
+        const int key_row = key_tile(j) * L::BN;  // token row within the head
         const int sv_ = j % L::SV;
         if (j >= L::SV && !mbar_wait(bar_v_empty + sv_, (j / L::SV - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar_v_full + sv_, L::V_BYTES);
@@ -288,7 +325,10 @@ __global__ void __launch_bounds__(512, 1)
         for (int half = 0; half < 2; ++half) {
           if (!wait_warp(half == 0 ? bar_p_lo + t : bar_p_hi + t, j & 1)) { ok = false; break; }
           tc_fence_after();
-          if constexpr (FP8) {
+          bool issue = true;  // block-sparse variant: the softmax group may have dropped key tile j
+          if constexpr (SPARSE) issue = *reinterpret_cast<volatile int*>(sPvKeep + t * 2 + (j & 1)) != 0;
+          if (!issue) {
+          } else if constexpr (FP8) {
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
               const int kk = half * 2 + k2;  // 32 keys per MMA
@@ -328,7 +368,7 @@ __global__ void __launch_bounds__(512, 1)
     auto load_k = [&](int jj) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar_k_full + jj % L::SK, L::K_BYTES);
-        tma_load_3d(sK + (jj % L::SK) * L::K_BYTES, &tm_k, bar_k_full + jj % L::SK, 0, jj * L::BN, bh);
+        tma_load_3d(sK + (jj % L::SK) * L::K_BYTES, &tm_k, bar_k_full + jj % L::SK, 0, key_tile(jj) * L::BN, bh);
       }
       k_loaded = jj + 1;
     };
@@ -407,7 +447,7 @@ __global__ void __launch_bounds__(512, 1)
       // for key tile j+1 is issued early in iteration j and stored at its end
       float* sks_t = sSKs + t * 256;
       auto key_scale = [&](int jj) -> float {
-        const int key = jj * L::BN + r;
+        const int key = key_tile(jj) * L::BN + r;
         return key < N ? __ldg(sk_head + key) : 0.f;
       };
       if constexpr (PER_TOKEN) {
@@ -416,6 +456,7 @@ __global__ void __launch_bounds__(512, 1)
       }
 
       float m_use = 0.f;
+      float m_run = -INFINITY;  // block-sparse variant: the row's largest score so far (log2 units)
       float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       bool ok = true;
       for (int j = 0; j < n_iter[t]; ++j) {
@@ -430,16 +471,17 @@ __global__ void __launch_bounds__(512, 1)
         }
         // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
         // c > cmax of this tile are left out of the maximum and get P~ = 0
-        const int kvalid = N - j * L::BN;
-        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
-        const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
+        const int kt = key_tile(j);
+        const int kvalid = N - kt * L::BN;
+        const bool diag = (CAUSAL && kt == q_tile) || (RAGGED && kvalid < L::BN);
+        const int cmax = min((CAUSAL && kt == q_tile) ? r : L::BN - 1, kvalid - 1);
 
         // ---- row maximum of the dequantized scores (log2 units), S read in two halves
         float mx = -INFINITY;
         float cb0 = 0.f, cb1 = 0.f;
         if constexpr (!PER_TOKEN) {
-          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
-          cb1 = 2 * j + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * j + 1)) : 0.f;
+          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * kt));
+          cb1 = 2 * kt + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * kt + 1)) : 0.f;
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -471,12 +513,27 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
 
+        // ---- stage 2 (block-sparse variant): the group keeps key tile j when one of its rows
+        // below N scores within skip_lambda of its running maximum (always the first tile, whose
+        // running maximum is -inf).  Vote slots rotate over three steps: slot (j+1) % 3 was last
+        // read at step j-2, before every thread arrived at step j-1's barrier.
+        bool keep_tile = true;
+        if constexpr (SPARSE) {
+          const bool row_keeps = q_row < N && !(mx < m_run - skip_lambda);
+          int* vote = sSkipVote + t * 3;
+          if (r == 0) vote[(j + 1) % 3] = 0;
+          if (__any_sync(0xffffffffu, row_keeps) && lane == 0) atomicOr(vote + j % 3, 1);
+          group_sync(3 + t);
+          keep_tile = *reinterpret_cast<volatile int*>(vote + j % 3) != 0;
+          if (keep_tile && q_row < N) m_run = fmaxf(m_run, mx);
+        }
+
         // ---- offset update; the correction group rescales O^T columns of rows whose offset moved
         float alpha = 1.f;
         bool rescale = false;
         if (j == 0) {
           m_use = round_up_to(mx, qm);
-        } else if (mx > m_use + lazy) {
+        } else if (keep_tile && mx > m_use + lazy) {
           const float m_new = round_up_to(mx, qm);
           alpha = FP8 ? exp2_int(m_use - m_new) : fast_exp2(m_use - m_new);
           m_use = m_new;
@@ -572,6 +629,9 @@ __global__ void __launch_bounds__(512, 1)
           }
           }
           if (cb == 32 || cb == 96) {
+            if constexpr (SPARSE) {
+              if (cb == 32 && r == 0) sPvKeep[t * 2 + (j & 1)] = 1;  // read by the P.V warp after bar_p_lo
+            }
             fence_proxy_async_shared();
             mbar_arrive(cb == 32 ? bar_p_lo + t : bar_p_hi + t);
           }
@@ -627,13 +687,25 @@ __global__ void __launch_bounds__(512, 1)
             st_shared_v4(p_row + (c8 >> 3) * L::P_ATOM + (((c8 & 7) ^ (qi & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
             }
             if (c8 == 7 || c8 == 15) {
+              if constexpr (SPARSE) {
+                if (c8 == 7 && r == 0) sPvKeep[t * 2 + (j & 1)] = 1;
+              }
               fence_proxy_async_shared();
               mbar_arrive(c8 == 7 ? bar_p_lo + t : bar_p_hi + t);
             }
           }
           return true;
         };
-        if (!(diag ? exp_pass_masked() : exp_pass())) { ok = false; break; }
+        if (!keep_tile) {
+          // stage 2 dropped the tile: no exp2 pass and no P~.  The wait for the previous P.V keeps
+          // this group's bar_o_done waits one phase apart and orders the reuse of the flag slot.
+          if (j > 0 && !wait_warp(bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
+          tc_fence_before();
+          mbar_arrive(bar_s_free + t);  // S_t read (for the maximum)
+          if (r == 0) sPvKeep[t * 2 + (j & 1)] = 0;
+          mbar_arrive(bar_p_lo + t);
+          mbar_arrive(bar_p_hi + t);
+        } else if (!(diag ? exp_pass_masked() : exp_pass())) { ok = false; break; }
         if constexpr (PER_TOKEN) {  // key scales of tile j+1 into the other buffer
           if (j + 1 < n_iter[t]) {
             sks_t[((j + 1) & 1) * 128 + r] = sk_next;

@@ -14,6 +14,7 @@
 #include "attn_kernels.cuh"
 #include "prep_kernels.cuh"
 #include "sage_attn.h"
+#include "sparse_kernels.cuh"
 #include "workspace.cuh"
 
 namespace {
@@ -107,6 +108,11 @@ int check_scale(float sm_scale) {
 
 int check_gran(int g) { return (g == SAGE_PER_TOKEN || g == SAGE_PER_BLOCK) ? SAGE_OK : SAGE_ERR_INVALID; }
 
+// The block-sparse variant: head dimension 128 and at most 512 key tiles (N <= 65536).
+int check_sparse(int N, int d) {
+  return (d == 128 && (N + 127) / 128 <= sage::kSparseMaxKeyBlocks) ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
 
 // v: fp16 V, or (fp8_sv != nullptr) the E4M3 codes of the FP8 P.V variant with their
@@ -114,7 +120,8 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CU
 int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v, void* o,
                         int B, int H, int N, int d, int causal, float sm_scale, int granularity,
                         cudaStream_t st, long long* trace = nullptr, int trace_ctas = 0,
-                        const float* fp8_sv = nullptr, const float* fp8_vm = nullptr) {
+                        const float* fp8_sv = nullptr, const float* fp8_vm = nullptr,
+                        const int* kv_count = nullptr, const int16_t* kv_index = nullptr, float skip_lambda = 0.f) {
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
   const bool vmap_ok = fp8_sv ? make_v8_map3(&tv, v, N, BH, d) : make_v_map3(&tv, v, N, BH, d);
@@ -140,6 +147,9 @@ int attn_quantized_impl(const int8_t* q8, const int8_t* k8, const float* sq, con
   a.fp8 = fp8_sv != nullptr;
   a.sv = fp8_sv;
   a.vm = fp8_vm;
+  a.kv_count = kv_count;
+  a.kv_index = kv_index;
+  a.skip_lambda = skip_lambda;
   const cudaError_t e = sage::launch_attn(a, st);
   return e == cudaErrorNotSupported ? SAGE_ERR_UNSUPPORTED : cuda_status(e);
 }
@@ -350,6 +360,96 @@ int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, in
   nvtxRangePushA("sage_fp8pv_fused");
   if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v8, o, B, H, N, d, causal, sm_scale, granularity, st, nullptr, 0,
                                     sv, vm);
+  nvtxRangePop();
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
+}
+
+int sage_sparse_predict(const void* q, const void* k, int B, int H, int N, int d, int causal, float sm_scale, float tau,
+                        float theta, int* kv_count, int16_t* kv_index, void* stream) {
+  if (!q || !k || !kv_count || !kv_index) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_scale(sm_scale))) return rc;
+  if (!(tau > 0.f && tau <= 1.f) || !std::isfinite(theta)) return SAGE_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  void* ws = nullptr;
+  if (sage::workspace_alloc(&ws, sage::sparse_predict_workspace(BH, N, d), st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  rc = cuda_status(sage::launch_sparse_predict(static_cast<const __half*>(q), static_cast<const __half*>(k), ws, BH, N,
+                                               d, causal != 0, sm_scale, tau, theta, kv_count, kv_index, st));
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
+}
+
+int sage_attn_fwd_sparse_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk, const void* v,
+                                   void* o, int B, int H, int N, int d, int causal, float sm_scale, int granularity,
+                                   const int* kv_count, const int16_t* kv_index, float skip_lambda, void* stream) {
+  if (!q8 || !k8 || !sq || !sk || !v || !o || !kv_count || !kv_index) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!(skip_lambda > 0.f)) return SAGE_ERR_INVALID;  // +inf: no second stage; NaN rejected
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(sk)) return SAGE_ERR_INVALID;
+  return attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity,
+                             static_cast<cudaStream_t>(stream), nullptr, 0, nullptr, nullptr, kv_count, kv_index,
+                             skip_lambda);
+}
+
+int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                         float sm_scale, int granularity, float tau, float theta, float skip_lambda, void* stream) {
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
+  if (!(tau > 0.f && tau <= 1.f) || !std::isfinite(theta) || !(skip_lambda > 0.f)) return SAGE_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const size_t elems = static_cast<size_t>(BH) * N * d;
+  const size_t nsq = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 1);
+  const size_t nsk = static_cast<size_t>(BH) * sage_scale_count(N, granularity, 0);
+  const size_t nqb = static_cast<size_t>((N + 255) / 256), nkb = static_cast<size_t>((N + 127) / 128);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t off_k8 = up(elems);
+  const size_t off_sq = off_k8 + up(elems);
+  const size_t off_sk = off_sq + up(nsq * 4);
+  const size_t off_km = off_sk + up(nsk * 4);
+  const size_t off_cnt = off_km + up(static_cast<size_t>(BH) * d * 4);
+  const size_t off_idx = off_cnt + up(static_cast<size_t>(BH) * nqb * 4);
+  const size_t off_pred = off_idx + up(static_cast<size_t>(BH) * nqb * nkb * 2);
+  const size_t total = off_pred + up(sage::sparse_predict_workspace(BH, N, d));
+  void* ws = nullptr;
+  if (sage::workspace_alloc(&ws, total, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int8_t* q8 = reinterpret_cast<int8_t*>(w);
+  int8_t* k8 = reinterpret_cast<int8_t*>(w + off_k8);
+  float* sq = reinterpret_cast<float*>(w + off_sq);
+  float* sk = reinterpret_cast<float*>(w + off_sk);
+  float* km = reinterpret_cast<float*>(w + off_km);
+  int* cnt = reinterpret_cast<int*>(w + off_cnt);
+  int16_t* idx = reinterpret_cast<int16_t*>(w + off_idx);
+  nvtxRangePushA("sage_sparse_prep");
+  rc = cuda_status(sage::launch_sparse_predict(static_cast<const __half*>(q), static_cast<const __half*>(k),
+                                               w + off_pred, BH, N, d, causal != 0, sm_scale, tau, theta, cnt, idx, st));
+  if (!rc) rc = cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, BH, N, d, st));
+  if (!rc) rc = sage_quant_qk(q, k, km, q8, k8, sq, sk, B, H, N, d, granularity, stream);
+  nvtxRangePop();
+  nvtxRangePushA("sage_sparse_fused");
+  if (!rc) rc = attn_quantized_impl(q8, k8, sq, sk, v, o, B, H, N, d, causal, sm_scale, granularity, st, nullptr, 0,
+                                    nullptr, nullptr, cnt, idx, skip_lambda);
   nvtxRangePop();
   const cudaError_t fe = cudaFreeAsync(ws, st);
   if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
