@@ -379,6 +379,8 @@ def run_ours(args, w: W.Workload):
     breakdown = {
         "smooth_k_ms": timed(lambda: sa.sage_smooth_k(k, km, stream), nb),
         "quant_qk_ms": timed(lambda: sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream), nb),
+        # the same two steps in one launch (K mean, K and Q codes in one pass over each head's tokens)
+        "prep_one_launch_ms": timed(lambda: sa.sage_prep_qk(q, k, km, q8, k8, sq, sk, gran, stream), nb),
         "attn_kernel_ms": kernel_ms,
         "step_ms": ms,
     }

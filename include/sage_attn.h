@@ -79,6 +79,15 @@ int sage_smooth_k(const void* k, float* km, int B, int H, int N, int d, void* st
 int sage_quant_qk(const void* q, const void* k, const float* km, int8_t* q8, int8_t* k8, float* sq,
                   float* sk, int B, int H, int N, int d, int granularity, void* stream);
 
+/* sage_smooth_k followed by sage_quant_qk (with the mean) in ONE launch and one pass over the
+ * tokens of each head (K smoothing fused with the quantization): one cluster
+ * of CTAs per head sums K exactly over its token slices and shares the sums through distributed
+ * shared memory, then quantizes the slices' K groups (K minus the mean) and Q groups.  Outputs,
+ * bit for bit, those of the two calls: km fp32 [B,H,d]; q8, k8 int8 [B,H,N,d]; sq, sk fp32 scales
+ * of the granularity.  q, k: fp16 [B,H,N,d] (in). */
+int sage_prep_qk(const void* q, const void* k, float* km, int8_t* q8, int8_t* k8, float* sq, float* sk, int B, int H,
+                 int N, int d, int granularity, void* stream);
+
 /* The whole forward pass as a user calls it: smooth K, quantize Q and K, fused attention.
  * q, k, v: fp16 [B,H,N,d] (in); o: fp16 [B,H,N,d] (out).  causal: keys j > i masked
  * (top-left aligned).  Workspace (int8 Q/K, scales, km: 2*B*H*N*d bytes plus scales) is

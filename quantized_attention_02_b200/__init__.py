@@ -54,6 +54,7 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_attn_fwd_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_debug_qk_int32.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p]
         lib.sage_quant_v_fp8.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_prep_qk.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
         lib.sage_attn_fwd_fp8pv_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_attn_fwd_fp8pv.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_sparse_predict.argtypes = [_p, _p, _i, _i, _i, _i, _i, _f, _f, _f, _p, _p, _p]
@@ -71,7 +72,7 @@ def get_lib() -> ctypes.CDLL:
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
                   "sage_debug_attn_trace", "sage_debug_mma_peak", "sage_attn_fwd_host",
-                  "sage_debug_wait_timeout", "sage_quant_v_fp8", "sage_attn_fwd_fp8pv_quantized",
+                  "sage_debug_wait_timeout", "sage_quant_v_fp8", "sage_attn_fwd_fp8pv_quantized", "sage_prep_qk",
                   "sage_attn_fwd_fp8pv", "sage_sparse_predict", "sage_attn_fwd_sparse_quantized",
                   "sage_attn_fwd_sparse"):
             getattr(lib, n).restype = _i
@@ -138,6 +139,13 @@ def sage_quant_qk(q, k, km, q8, k8, sq, sk, granularity: int, stream=None) -> No
     B, H, N, d = _shape(q)
     _check(get_lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(km), _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk),
                              B, H, N, d, int(granularity), _stream(stream)), "sage_quant_qk")
+
+
+def sage_prep_qk(q, k, km, q8, k8, sq, sk, granularity: int, stream=None) -> None:
+    """K mean, K and Q codes and scales in one launch (the results of sage_smooth_k then sage_quant_qk)."""
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_prep_qk(_ptr(q), _ptr(k), _ptr(km), _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), B, H, N, d,
+                                  int(granularity), _stream(stream)), "sage_prep_qk")
 
 
 def sage_attn_fwd(q, k, v, o, causal: bool, sm_scale: float, granularity: int, stream=None) -> None:

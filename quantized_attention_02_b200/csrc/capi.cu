@@ -293,6 +293,18 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, i
   return rc;
 }
 
+int sage_prep_qk(const void* q, const void* k, float* km, int8_t* q8, int8_t* k8, float* sq, float* sk, int B, int H,
+                 int N, int d, int granularity, void* stream) {
+  if (!q || !k || !km || !q8 || !k8 || !sq || !sk) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if ((rc = check_gran(granularity))) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8)) return SAGE_ERR_INVALID;
+  return cuda_status(sage::launch_prep_fused(static_cast<const __half*>(q), static_cast<const __half*>(k), km, q8, k8,
+                                             sq, sk, B * H, N, d, granularity == SAGE_PER_TOKEN,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 int sage_quant_v_fp8(const void* v, uint8_t* v8, float* sv, float* vm, int B, int H, int N, int d, void* stream) {
   if (!v || !v8 || !sv) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);

@@ -55,24 +55,18 @@ constexpr int kSmoothMaxCtas = 8;
 constexpr int kSmoothThreads = 512;
 constexpr int kSmoothTokensPerCta = 2048;
 
+// Exact channel sums of the token rows [t0, t1) of one head's K (base points at channel piece*8 of
+// token 0), by the whole CTA: every thread accumulates its rows with split_acc, flushing into int64
+// every kSplitFlushTokens tokens; the CTA's sums land in csum[D].  Ends with the CTA's threads
+// synchronized (csum complete).
 template <int D>
-__global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* __restrict__ k,
-                                                                  float* __restrict__ km, int N) {
+__device__ __forceinline__ void cta_k_channel_sums(const __half* __restrict__ base, int t0, int t1,
+                                                   long long* __restrict__ csum) {
   constexpr int T = D / 8;                 // threads per token row
   constexpr int R = kSmoothThreads / T;    // rows per pass
   constexpr int U = 4;                     // passes in flight
   constexpr int WARPS = kSmoothThreads / 32;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int n_ctas = static_cast<int>(cluster.num_blocks());  // consecutive CTAs of grid x
-  const int bh = static_cast<int>(blockIdx.x) / n_ctas;      // (grid x holds B*H clusters: no 65535 cap)
-  const int piece = threadIdx.x % T;       // channels piece*8 .. piece*8+7
   const int row = threadIdx.x / T;
-  const int slice = (N + n_ctas - 1) / n_ctas;
-  const int t0 = rank * slice;
-  const int t1 = min(N, t0 + slice);
-  const __half* base = k + (static_cast<size_t>(bh) * N) * D + piece * 8;
-
   constexpr int ITERS = kSplitFlushTokens / U;  // loop iterations between flushes
   long long acc[8];
 #pragma unroll
@@ -111,7 +105,6 @@ __global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* 
     for (int off = T; off < 32; off <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
   }
   __shared__ long long part[WARPS][T][8];
-  __shared__ long long csum[D];  // this CTA's channel sums, read by rank 0 of the cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane < T) {
 #pragma unroll
@@ -125,14 +118,37 @@ __global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* 
     for (int w = 0; w < WARPS; ++w) s += part[w][p][i];
     csum[threadIdx.x] = s;
   }
+  __syncthreads();
+}
+
+// The K mean of channel c from the cluster's per-CTA sums (distributed shared memory):
+// fl32(fl32(S_c) / N) * 2^-24.
+__device__ __forceinline__ float cluster_k_mean(cg::cluster_group& cluster, long long* csum, int c, int n_ctas,
+                                                int N) {
+  long long s = 0;
+  for (int r = 0; r < n_ctas; ++r) s += *cluster.map_shared_rank(csum + c, r);
+  const float s32 = __ll2float_rn(s);
+  const float mean = __fdiv_rn(s32, static_cast<float>(N));
+  return __fmul_rn(mean, 5.9604644775390625e-08f);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSmoothThreads) smooth_k_kernel(const __half* __restrict__ k,
+                                                                  float* __restrict__ km, int N) {
+  constexpr int T = D / 8;                 // threads per token row
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int n_ctas = static_cast<int>(cluster.num_blocks());  // consecutive CTAs of grid x
+  const int bh = static_cast<int>(blockIdx.x) / n_ctas;      // (grid x holds B*H clusters: no 65535 cap)
+  const int piece = threadIdx.x % T;       // channels piece*8 .. piece*8+7
+  const int slice = (N + n_ctas - 1) / n_ctas;
+  const int t0 = rank * slice;
+  const int t1 = min(N, t0 + slice);
+  __shared__ long long csum[D];  // this CTA's channel sums, read by rank 0 of the cluster
+  cta_k_channel_sums<D>(k + (static_cast<size_t>(bh) * N) * D + piece * 8, t0, t1, csum);
   cluster.sync();
-  if (rank == 0 && threadIdx.x < D) {
-    long long s = 0;
-    for (int r = 0; r < n_ctas; ++r) s += *cluster.map_shared_rank(csum + threadIdx.x, r);
-    const float s32 = __ll2float_rn(s);
-    const float mean = __fdiv_rn(s32, static_cast<float>(N));
-    km[static_cast<size_t>(bh) * D + threadIdx.x] = __fmul_rn(mean, 5.9604644775390625e-08f);
-  }
+  if (rank == 0 && threadIdx.x < D)
+    km[static_cast<size_t>(bh) * D + threadIdx.x] = cluster_k_mean(cluster, csum, threadIdx.x, n_ctas, N);
   cluster.sync();  // every CTA keeps its csum in place until rank 0 has read it
 }
 
@@ -273,6 +289,160 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* __restrict__ x
                                                     int8_t* __restrict__ q, float* __restrict__ scale, int N,
                                                     long long rows) {
   quant_block<D, G, SMOOTH>(x, km, q, scale, N, rows, blockIdx.x);
+}
+
+// ---------------------------------------------------------------- the whole preparation in one launch
+// K mean, K codes and Q codes of a head in one launch: one cluster of C CTAs per head (C as for
+// smooth_k_kernel) splits the head's tokens into slices of whole 128-token blocks.  Phase 1 sums K
+// exactly over the slice (cta_k_channel_sums) and every CTA derives the mean from the cluster's
+// sums in distributed shared memory.  Phase 2 quantizes the slice's K groups (K minus the mean)
+// and Q groups.  Per-block groups go to teams of G*T/8 threads (eight 16-byte loads each; T = D/8
+// threads per token row): a team loads its whole group into registers (fp16, one read), takes the
+// absmax with shuffles and one named barrier, and writes the codes from registers.  Per-token groups go to T-lane
+// teams within a warp (no barrier).  Same arithmetic as smooth_k_kernel and quant_kernel, so the
+// same bits.  Rows past N read as zeros (and are neither smoothed nor stored).
+// BAR0: the first named-barrier id of this pass's teams (ids BAR0 .. BAR0 + TEAMS - 1).  Each
+// pass needs its own ids: a team that finishes its K groups early enters the Q pass while other
+// teams still synchronize on theirs, and one barrier id must never see two thread counts at once.
+template <int D, int G, bool SMOOTH, int BAR0>
+__device__ __forceinline__ void team_quant_groups(const __half* __restrict__ x, const float (&mu)[8],
+                                                  int8_t* __restrict__ out, float* __restrict__ scale, int N,
+                                                  int bh, int t0, int t1, float* red) {
+  constexpr int T = D / 8;       // threads per token row
+  const int piece = threadIdx.x % T;
+  const __half* head = x + (static_cast<size_t>(bh) * N) * D + piece * 8;
+  int8_t* ohead = out + (static_cast<size_t>(bh) * N) * D + piece * 8;
+  auto smooth = [&](float (&v)[8], bool live) {
+    if constexpr (SMOOTH) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = live ? __fsub_rn(v[i], mu[i]) : 0.f;
+    }
+  };
+  if constexpr (G == 1) {
+    // one token per T-lane team; all CTA rows, U passes at a time
+    constexpr int R = kSmoothThreads / T;
+    constexpr int U = 4;
+    const int row = threadIdx.x / T;
+    for (int t = t0 + row; t - row < t1; t += U * R) {  // t - row is CTA-uniform: whole warps iterate
+      uint4 w[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int tok = t + u * R;
+        w[u] = tok < t1 ? __ldg(reinterpret_cast<const uint4*>(head + static_cast<size_t>(tok) * D))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int tok = t + u * R;
+        float v[8];
+        unpack8(w[u], v);
+        smooth(v, tok < t1);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+#pragma unroll
+        for (int off = T / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        float s = 0.f, inv = 0.f;
+        if (a > 0.f) {
+          s = __fdiv_rn(a, 127.0f);
+          inv = __fdiv_rn(127.0f, a);
+        }
+        if (tok < t1) {
+          *reinterpret_cast<uint2*>(ohead + static_cast<size_t>(tok) * D) = pack8(v, inv);
+          if (piece == 0) scale[static_cast<size_t>(bh) * N + tok] = s;
+        }
+      }
+    }
+  } else {
+    constexpr int PASSES = 8;               // 16-byte loads per thread, all in flight
+    constexpr int TEAM = G * T / PASSES;    // threads per group team (64 .. 256)
+    constexpr int TEAMS = kSmoothThreads / TEAM;
+    constexpr int P = TEAM / T;             // rows per team pass
+    constexpr int TW = TEAM / 32;           // warps per team
+    static_assert(TEAM % 32 == 0 && TEAMS <= 8 && P * PASSES == G && BAR0 + TEAMS <= 16, "team shape");
+    const int team = threadIdx.x / TEAM, tt = threadIdx.x % TEAM;
+    const int row = tt / T;
+    const int n_groups = (N + G - 1) / G;
+    int parity = 0;
+    for (int g = t0 / G + team; g * G < t1; g += TEAMS, parity ^= 1) {
+      const int g0 = g * G;
+      uint4 w[PASSES];
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        const int tok = g0 + p * P + row;
+        w[p] = tok < t1 ? __ldg(reinterpret_cast<const uint4*>(head + static_cast<size_t>(tok) * D))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float a = 0.f;
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        float v[8];
+        unpack8(w[p], v);
+        smooth(v, g0 + p * P + row < t1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      // the team's warp maxima meet in shared memory (two slots, alternating by group, so a slot
+      // is only rewritten after every thread of the team has passed the next barrier)
+      float* slot = red + parity * (kSmoothThreads / 32) + team * TW;
+      if ((tt & 31) == 0) slot[tt >> 5] = a;
+      asm volatile("barrier.sync %0, %1;" ::"r"(BAR0 + team), "r"(TEAM) : "memory");
+      a = slot[0];
+#pragma unroll
+      for (int i = 1; i < TW; ++i) a = fmaxf(a, slot[i]);
+      float s = 0.f, inv = 0.f;
+      if (a > 0.f) {
+        s = __fdiv_rn(a, 127.0f);
+        inv = __fdiv_rn(127.0f, a);
+      }
+      if (tt == 0) scale[static_cast<size_t>(bh) * n_groups + g] = s;
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        const int tok = g0 + p * P + row;
+        float v[8];
+        unpack8(w[p], v);
+        smooth(v, tok < t1);
+        if (tok < t1) *reinterpret_cast<uint2*>(ohead + static_cast<size_t>(tok) * D) = pack8(v, inv);
+      }
+    }
+  }
+}
+
+template <int D, int GQ, int GK>
+__global__ void __launch_bounds__(kSmoothThreads) prep_fused_kernel(const __half* __restrict__ q,
+                                                                    const __half* __restrict__ k,
+                                                                    float* __restrict__ km, int8_t* __restrict__ q8,
+                                                                    int8_t* __restrict__ k8, float* __restrict__ sq,
+                                                                    float* __restrict__ sk, int N) {
+  constexpr int T = D / 8;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int n_ctas = static_cast<int>(cluster.num_blocks());
+  const int bh = static_cast<int>(blockIdx.x) / n_ctas;
+  const int piece = threadIdx.x % T;
+  const int slice = ((N + n_ctas - 1) / n_ctas + 127) / 128 * 128;  // whole 128-token blocks
+  const int t0 = min(N, rank * slice);
+  const int t1 = min(N, t0 + slice);
+  __shared__ long long csum[D];
+  __shared__ float s_mu[D];
+  cta_k_channel_sums<D>(k + (static_cast<size_t>(bh) * N) * D + piece * 8, t0, t1, csum);
+  cluster.sync();
+  if (threadIdx.x < D) {
+    const float m = cluster_k_mean(cluster, csum, threadIdx.x, n_ctas, N);
+    s_mu[threadIdx.x] = m;
+    if (rank == 0) km[static_cast<size_t>(bh) * D + threadIdx.x] = m;
+  }
+  cluster.sync();  // the cluster's sums have been read; s_mu is complete in every CTA
+  // group-team warp maxima [parity][warp], one array per pass: a warp moving on to the Q groups
+  // must not overwrite a slot another warp of its K team has yet to read
+  __shared__ float red_k[2 * (kSmoothThreads / 32)], red_q[2 * (kSmoothThreads / 32)];
+  float mu[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mu[i] = s_mu[piece * 8 + i];
+  team_quant_groups<D, GK, true, 1>(k, mu, k8, sk, N, bh, t0, t1, red_k);   // barrier ids 1 .. 8
+  team_quant_groups<D, GQ, false, 9>(q, mu, q8, sq, N, bh, t0, t1, red_q);  // barrier ids 9 .. 12
 }
 
 // ---------------------------------------------------------------- V to FP8 (E4M3)
@@ -502,6 +672,39 @@ static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8, float* sv,
 cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N, int D,
                                cudaStream_t st) {
   return D == 128 ? launch_quant_v_fp8_d<128>(v, v8, sv, vm, BH, N, st) : launch_quant_v_fp8_d<64>(v, v8, sv, vm, BH, N, st);
+}
+
+template <int D, int GQ, int GK>
+static cudaError_t launch_prep_fused_g(const __half* q, const __half* k, float* km, int8_t* q8, int8_t* k8, float* sq,
+                                       float* sk, int BH, int N, cudaStream_t st) {
+  int ctas = 1;  // the cluster size of smooth_k
+  while (ctas < kSmoothMaxCtas && N / (2 * ctas) >= kSmoothTokensPerCta) ctas *= 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas) * static_cast<unsigned>(BH));
+  cfg.blockDim = dim3(kSmoothThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prep_fused_kernel<D, GQ, GK>, q, k, km, q8, k8, sq, sk, N);
+}
+
+template <int D>
+static cudaError_t launch_prep_fused_d(const __half* q, const __half* k, float* km, int8_t* q8, int8_t* k8, float* sq,
+                                       float* sk, int BH, int N, bool per_token, cudaStream_t st) {
+  return per_token ? launch_prep_fused_g<D, 1, 1>(q, k, km, q8, k8, sq, sk, BH, N, st)
+                   : launch_prep_fused_g<D, 128, 64>(q, k, km, q8, k8, sq, sk, BH, N, st);
+}
+
+cudaError_t launch_prep_fused(const __half* q, const __half* k, float* km, int8_t* q8, int8_t* k8, float* sq,
+                              float* sk, int BH, int N, int D, bool per_token, cudaStream_t st) {
+  return D == 128 ? launch_prep_fused_d<128>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st)
+                  : launch_prep_fused_d<64>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st);
 }
 
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st) {

@@ -8,6 +8,10 @@ namespace sage {
 
 // km[bh, c] = mean over N tokens of k[bh, :, c]; k fp16 [BH, N, D], km fp32 [BH, D].
 cudaError_t launch_smooth_k(const __half* k, float* km, int BH, int N, int D, cudaStream_t st);
+// K mean, K codes and Q codes in one launch (one cluster per head, one pass over its tokens);
+// same results as launch_smooth_k followed by launch_quant_qk with the mean.
+cudaError_t launch_prep_fused(const __half* q, const __half* k, float* km, int8_t* q8, int8_t* k8, float* sq,
+                              float* sk, int BH, int N, int D, bool per_token, cudaStream_t st);
 // V to E4M3 with per-(head, channel) scales sv; vm: channel means (V smoothed) or nullptr (not smoothed).
 cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N, int D,
                                cudaStream_t st);

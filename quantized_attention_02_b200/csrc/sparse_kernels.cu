@@ -44,27 +44,37 @@ __global__ void __launch_bounds__(kPoolThreads) sparse_pool_kernel(const __half*
   float sum[8], usum[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) sum[i] = usum[i] = 0.f;
-  // whole passes, so that every lane takes part in the row's shuffles; rows past n read zeros
-  for (int t = row; t < size; t += R) {
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (t < n) w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t) * D + piece * 8));
-    const __half2* h = reinterpret_cast<const __half2*>(&w);
-    float x[8];
-    float ss = 0.f;
+  // whole passes, so that every lane takes part in the row's shuffles; rows past n read zeros.
+  // U passes' loads are issued together (a block is 8 to 32 passes), so the loop is not bound
+  // by one load's latency per pass.
+  constexpr int U = 4;
+  for (int t = row; t < size; t += U * R) {
+    uint4 w[U];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    for (int u = 0; u < U; ++u) {
+      w[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (t + u * R < n) w[u] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D + piece * 8));
     }
 #pragma unroll
-    for (int off = T / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;  // a zero token adds nothing to either sum
+    for (int u = 0; u < U; ++u) {
+      const __half2* h = reinterpret_cast<const __half2*>(&w[u]);
+      float x[8];
+      float ss = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      sum[i] += x[i];
-      usum[i] = fmaf(x[i], inv, usum[i]);
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+        ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+      }
+#pragma unroll
+      for (int off = T / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;  // a zero token adds nothing to either sum
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sum[i] += x[i];
+        usum[i] = fmaf(x[i], inv, usum[i]);
+      }
     }
   }
   // lanes of a warp with the same piece differ by multiples of T

@@ -67,3 +67,31 @@ def test_k_mean_of_large_values_is_exact(sa):
     torch.cuda.synchronize()
     assert sa.sage_last_device_error() == 0
     np.testing.assert_array_equal(km.cpu().numpy(), oracle.smooth_k(k))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 200, 1000, 4095, 6001, 12289, 16384, 20000])
+@pytest.mark.parametrize("gran", [0, 1])
+def test_one_launch_prep_equals_the_two_steps_and_the_oracle(sa, N, d, gran):
+    """sage_prep_qk (K mean, K codes, Q codes in one launch, one cluster per head) gives the bits
+    of sage_smooth_k + sage_quant_qk, and those of the oracle, at every cluster size, both
+    granularities and ragged lengths (slices of whole 128-token blocks, a short last one)."""
+    w = W.Workload(f"prep1_n{N}_d{d}", 1, 3, N, d, False, gran == 1, n_out=4, out_mag=20.0)
+    q, k, _ = W.make_qkv(w, seed=N + 1)
+    qd, kd = q.cuda(), k.cuda()
+    a = sa.empty_quantized(qd, gran)
+    b = sa.empty_quantized(qd, gran)
+    for t in b:
+        t.fill_(7)  # stale values the one-launch kernel must overwrite
+    sa.sage_smooth_k(kd, a[0])
+    sa.sage_quant_qk(qd, kd, a[0], *a[1:], gran)
+    sa.sage_prep_qk(qd, kd, *b, gran)
+    torch.cuda.synchronize()
+    assert sa.sage_last_device_error() == 0
+    for name, x, y in zip(("km", "q8", "k8", "sq", "sk"), a, b):
+        assert torch.equal(x, y), name
+    gq, gk = oracle.GROUP_PER_BLOCK if gran == 1 else oracle.GROUP_PER_TOKEN
+    km_ref = oracle.smooth_k(k)
+    np.testing.assert_array_equal(b[0].cpu().numpy(), km_ref)
+    np.testing.assert_array_equal(b[2].cpu().numpy(), oracle.quant(k, gk, km_ref)[0])
+    np.testing.assert_array_equal(b[1].cpu().numpy(), oracle.quant(q, gq)[0])

@@ -104,7 +104,12 @@ TOKEN64 = Workload("token_n16384_d64_full", 1, 64, 16384, 64, False, False, n_ou
 SPARSE = Workload("sparse_n16384_d128_win2048", 1, 64, 16384, 128, False, True, window=2048, align=14.0)
 SPARSE_CAUSAL = Workload("sparse_n16384_d128_win2048_causal", 1, 64, 16384, 128, True, True, window=2048, align=14.0)
 
-ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64, SPARSE, SPARSE_CAUSAL)}
+# a quarter of the block-sparse workload's heads, for profiler captures
+SPARSE_PROFILE = Workload("sparse_profile_b1h16_n16384_d128_win2048", 1, 16, 16384, 128, False, True, window=2048,
+                          align=14.0)
+
+ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64, SPARSE, SPARSE_CAUSAL,
+                           SPARSE_PROFILE)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
