@@ -143,8 +143,8 @@ int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, in
  * Huang; arXiv 2502.18137): a sparse and quantized attention with a two-stage online filter.
  * Stage 1 predicts the attention map at block level and skips the products of the blocks it
  * drops; stage 2, inside the online softmax, skips the P.V product (and the exp2 work) of a block
- * whose scores all lie far below the running row maximum.  Head dimension 128 and N <= 65536
- * (SAGE_ERR_UNSUPPORTED otherwise); P.V in fp16 as in sage_attn_fwd.
+ * whose scores all lie far below the running row maximum.  Head dimension 64 or 128 and
+ * N <= 65536 (SAGE_ERR_UNSUPPORTED otherwise); P.V in fp16 as in sage_attn_fwd.
  *
  * Stage 1 (sage_sparse_predict): query blocks of 256 tokens (QB = ceil(N/256) per (b,h)) and key
  * blocks of 128 tokens (KB = ceil(N/128)).  Each block is represented by the mean of its tokens;
@@ -165,7 +165,9 @@ int sage_sparse_predict(const void* q, const void* k, int B, int H, int N, int d
  * the blocks with each query's own key), plus stage 2: a query tile of 128 rows drops key block
  * j when, for each of its rows below N, the block's largest score (log2 units) lies more than
  * skip_lambda below the row's largest score over the blocks it visited before (its first block
- * is never dropped).  skip_lambda > 0; +INFINITY turns stage 2 off. */
+ * is never dropped).  skip_lambda > 0; +INFINITY turns stage 2 off.  A query block whose count
+ * is 0 (or whose list lacks the blocks its causal rows need) gets unspecified output; counts
+ * and entries out of range are clamped, so no access ever leaves the tensors. */
 int sage_attn_fwd_sparse_quantized(const int8_t* q8, const int8_t* k8, const float* sq, const float* sk,
                                    const void* v, void* o, int B, int H, int N, int d, int causal, float sm_scale,
                                    int granularity, const int* kv_count, const int16_t* kv_index, float skip_lambda,

@@ -49,7 +49,10 @@ struct AttnLayout {
   static constexpr int OFF_BAR = OFF_SK + STAGES * BN * 4;
   static constexpr int NUM_BARS = 1 + 3 * STAGES + 6 * NQT;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int USED = OFF_MISC + 16;
+  static constexpr int MAX_LIST = 512;                      // block-sparse variant: key tiles a CTA may visit
+  static constexpr int OFF_LIST = OFF_MISC + 16;            // int16 list of the key tiles visited
+  static constexpr int OFF_SKIP = OFF_LIST + MAX_LIST * 2;  // [2][3] stage-2 votes, [2][2] P.V keep flags
+  static constexpr int USED = OFF_SKIP + 64;
   // at least 116 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   static constexpr int SMEM = (USED + 1024 > 116 * 1024 ? USED + 1024 : 116 * 1024);
   __host__ __device__ static constexpr uint32_t s_col(int t) { return 128u * t; }
@@ -131,14 +134,24 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+__device__ __forceinline__ void group_bar(int id) { asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory"); }
+
 // TRACE builds record SM clock stamps of the pipeline events of the first trace_ctas CTAs
 // (layout documented at sage_debug_attn_trace in include/sage_attn.h).
-template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED>
+//
+// SPARSE = true is the block-sparse variant of the SpargeAttn abstract, as in the head-dimension
+// 128 kernel: kv_count[bh * n_pairs + pair] and the ascending key-tile list
+// kv_index[(bh * n_pairs + pair) * ceil(N/128) + i] give the key tiles this CTA visits (stage 1),
+// and a softmax group drops key tile j of its query tile when every row below N scores more than
+// skip_lambda (log2 units) under its running maximum there (stage 2): no exp2 pass, no P.V.
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE, bool RAGGED, bool SPARSE = false>
 __global__ void __launch_bounds__(384, 1)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ sq,
                      const float* __restrict__ sk, __half* __restrict__ o, int BH, int N,
-                     float sm_scale_log2, long long* __restrict__ trace, int trace_ctas) {
+                     float sm_scale_log2, long long* __restrict__ trace, int trace_ctas,
+                     const int* __restrict__ kv_count = nullptr, const int16_t* __restrict__ kv_index = nullptr,
+                     float skip_lambda = 0.f) {
   using L = AttnLayout<D>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -177,7 +190,28 @@ __global__ void __launch_bounds__(384, 1)
   int n_iter[2];
   n_iter[0] = CAUSAL ? tile0 + 1 : n_kv_total;
   n_iter[1] = (n_tiles > 1) ? (CAUSAL ? tile0 + 2 : n_kv_total) : 0;
+  int16_t* sList = reinterpret_cast<int16_t*>(smem + L::OFF_LIST);
+  int* sSkipVote = reinterpret_cast<int*>(smem + L::OFF_SKIP);     // [2 tiles][3]: bit 0 a row keeps the
+                                                                   // tile, bit 1 a warp gave up waiting
+  int* sPvKeep = reinterpret_cast<int*>(smem + L::OFF_SKIP + 32);  // [2 tiles][2]: P.V of key tile j issued
+  if constexpr (SPARSE) {
+    // causal lists end with the diagonal tiles: tile 0 stops one step before tile 1 when the
+    // list holds tile0 + 1.  Count and entries are clamped into range (a malformed list gives
+    // unspecified output, never an access outside the tensors); the cta_sync after the barrier
+    // set-up publishes the list.
+    const int count = min(max(kv_count[static_cast<size_t>(bh) * n_pairs + pair], 0), min(n_kv_total, L::MAX_LIST));
+    const int16_t* lst = kv_index + (static_cast<size_t>(bh) * n_pairs + pair) * n_kv_total;
+    for (int i = threadIdx.x; i < count; i += L::THREADS)
+      sList[i] = static_cast<int16_t>(min(max(static_cast<int>(lst[i]), 0), n_kv_total - 1));
+    const int last = count > 0 ? min(max(static_cast<int>(lst[count - 1]), 0), n_kv_total - 1) : -1;
+    n_iter[1] = n_tiles > 1 ? count : 0;
+    n_iter[0] = (CAUSAL && n_tiles > 1 && last == tile0 + 1) ? count - 1 : count;
+  }
   const int n_kv = max(n_iter[0], n_iter[1]);
+  auto key_tile = [&](int j) -> int {  // key tile visited in step j
+    if constexpr (SPARSE) return sList[j];
+    return j;
+  };
   const int row_base = bh * N;  // first row of this head in the [BH*N, D] arrays
   long long* trace_row = nullptr;
   if constexpr (TRACE) {
@@ -213,6 +247,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar_p_lo + 1, 128);
     mbar_init(bar_s_free, 128);
     mbar_init(bar_s_free + 1, 128);
+    for (int i = 0; i < 6; ++i) sSkipVote[i] = 0;
     *abort_flag = 0;
     *arrived = 0;
     fence_barrier_init();
@@ -246,7 +281,7 @@ __global__ void __launch_bounds__(384, 1)
         const int s = j % STAGES;
         const int it = j / STAGES;
         if (j >= STAGES && !mbar_wait(bar_kv_empty + s, (it - 1) & 1, abort_flag)) break;
-        const int key_row = j * L::BN;  // token row within the head
+        const int key_row = key_tile(j) * L::BN;  // token row within the head
         // per-token key scales: one bulk copy when the 128 scales exist and start on a 16-byte
         // boundary, else plain loads (zeros past N) stored before the arrival that publishes them
         const bool bulk_sk = PER_TOKEN && (N % 4 == 0) && key_row + L::BN <= N;
@@ -332,11 +367,16 @@ __global__ void __launch_bounds__(384, 1)
         // work on the second half
         if (!wait(bar_p_lo + t, j & 1)) break;
         tc_fence_after();
-        if (j == 0) issue_pv(s, true, 0, L::BN / 32);
-        else issue_pv(s, false, 0, L::BN / 32);
+        // block-sparse variant: the softmax group may have dropped key tile j (never the first)
+        bool issue = true;
+        if constexpr (SPARSE) issue = *reinterpret_cast<volatile int*>(sPvKeep + t * 2 + (j & 1)) != 0;
+        if (issue) {
+          if (j == 0) issue_pv(s, true, 0, L::BN / 32);
+          else issue_pv(s, false, 0, L::BN / 32);
+        }
         if (!wait(bar_p_full + t, j & 1)) break;
         tc_fence_after();
-        issue_pv(s, false, L::BN / 32, L::BN / 16);
+        if (issue) issue_pv(s, false, L::BN / 32, L::BN / 16);
         mma_commit_warp(bar_o_done + t);
         if (lane == 0) stamp((6 + 2 * t) * n_kv_total + j);
         mma_commit_warp(bar_kv_empty + s);  // this tile's products reading stage s are issued
@@ -380,17 +420,33 @@ __global__ void __launch_bounds__(384, 1)
       }
 
       float m_use = 0.f;  // exponent offset (log2 units) applied to this row so far
+      float m_run = -INFINITY;  // block-sparse variant: the row's largest score so far (log2 units)
       float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       bool ok = true;
+      // Block-sparse variant: the four warps of the group meet at one named barrier per key tile
+      // (the stage-2 vote).  A warp whose bounded wait gave up still takes that barrier once for
+      // the step it leaves in, with bit 1 in the vote, and the whole group leaves there: no warp
+      // is left waiting at a barrier that the others never reach.
+      int* vote = sSkipVote + t * 3;
+      auto leave_vote = [&](int jj) {
+        if constexpr (SPARSE) {
+          if (jj < n_iter[t]) {
+            if (r == 0) vote[(jj + 1) % 3] = 0;
+            if (lane == 0) atomicOr(vote + jj % 3, 2);
+            group_bar(1 + t);
+          }
+        }
+      };
       for (int j = 0; j < n_iter[t]; ++j) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag))) { leave_vote(j); ok = false; break; }
         tc_fence_after();
         if (r == 0) stamp((3 * t) * n_kv_total + j);
         // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
         // c > cmax of this tile are left out of the maximum and get P~ = 0.  Such a tile is
         // always the last key tile of its query tile.
-        const int kvalid = N - j * L::BN;
-        const bool diag = (CAUSAL && j == q_tile) || (RAGGED && kvalid < L::BN);
+        const int kt = key_tile(j);
+        const int kvalid = N - kt * L::BN;
+        const bool diag = (CAUSAL && kt == q_tile) || (RAGGED && kvalid < L::BN);
         uint32_t x[128];
         tmem_ld64_sync(tS + 0, *reinterpret_cast<uint32_t(*)[64]>(x + 0));
         tmem_ld64_sync(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(x + 64));
@@ -398,7 +454,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
           mbar_arrive(bar_s_free + t);
         }
-        const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, kvalid - 1);
+        const int cmax = min((CAUSAL && kt == q_tile) ? r : L::BN - 1, kvalid - 1);
         const int s = j % STAGES;
         float mx;            // row maximum of the dequantized scores (log2 units)
         float cb0 = 0.f, cb1 = 0.f, nb0 = 0.f, nb1 = 0.f;
@@ -412,7 +468,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int c = 0; c < 128; ++c) x[c] += kMagicBits;
           }
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_k_full + s, (j / STAGES) & 1, abort_flag))) { leave_vote(j); ok = false; break; }
           // max of S * sk over the row's keys (masked: -inf), then times a_r >= 0
           float m3 = -INFINITY;
 #pragma unroll
@@ -425,8 +481,8 @@ __global__ void __launch_bounds__(384, 1)
           mx = m3 == -INFINITY ? -INFINITY : a_r * m3;
         } else {
           // integer maxima of the two 64-key halves (one key scale each); masked keys INT_MIN
-          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * j));
-          cb1 = 2 * j + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * j + 1)) : 0.f;
+          cb0 = trim_scale(a_r * __ldg(sk_head + 2 * kt));
+          cb1 = 2 * kt + 1 < n_kgroups ? trim_scale(a_r * __ldg(sk_head + 2 * kt + 1)) : 0.f;
           if (diag) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -444,12 +500,28 @@ __global__ void __launch_bounds__(384, 1)
           mx = fmaxf(m0, m1);
         }
 
+        // ---- stage 2 (block-sparse variant): the group keeps key tile j when one of its rows
+        // below N scores within skip_lambda of its running maximum (always the first tile, whose
+        // running maximum is -inf).  Vote slots rotate over three steps: slot (j+1) % 3 was last
+        // read at step j-2, before every thread reached step j-1's barrier.
+        bool keep_tile = true;
+        if constexpr (SPARSE) {
+          const bool row_keeps = q_row < N && !(mx < m_run - skip_lambda);
+          if (r == 0) vote[(j + 1) % 3] = 0;
+          if (__any_sync(0xffffffffu, row_keeps) && lane == 0) atomicOr(vote + j % 3, 1);
+          group_bar(1 + t);
+          const int v = *reinterpret_cast<volatile int*>(vote + j % 3);
+          if (v & 2) { ok = false; break; }  // a warp of the group gave up waiting
+          keep_tile = (v & 1) != 0;
+          if (keep_tile && q_row < N) m_run = fmaxf(m_run, mx);
+        }
+
         // ---- rescale only when the maximum grew by more than 2^8 (bounds P~ by 256)
         float alpha = 1.f;
         bool rescale = false;
         if (j == 0) {
           m_use = round_up_to(mx, qm);
-        } else if (mx > m_use + 8.f) {
+        } else if (keep_tile && mx > m_use + 8.f) {
           const float m_new = round_up_to(mx, qm);
           alpha = fast_exp2(m_use - m_new);
           m_use = m_new;
@@ -457,9 +529,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         // P.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1)
         if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done + t, (j - 1) & 1, abort_flag))) { leave_vote(j + 1); ok = false; break; }
           tc_fence_after();
         }
+        // the P.V warp read this slot at step j-2, before P.V(j-1) (complete above) was issued;
+        // the flag is published by this thread's arrival on bar_p_lo below
+        if (SPARSE && r == 0) sPvKeep[t * 2 + (j & 1)] = keep_tile ? 1 : 0;
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
@@ -548,7 +623,14 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         };
-        if (diag) {
+        if (!keep_tile) {
+          // stage 2 dropped the tile: no P~, and the P.V warp issues nothing for it
+          if (diag) {
+            tc_fence_before();
+            mbar_arrive(bar_s_free + t);
+          }
+          mbar_arrive(bar_p_lo + t);
+        } else if (diag) {
           exp_pass_masked();
           tc_fence_before();
           mbar_arrive(bar_s_free + t);  // its re-reads of S_t are done
@@ -706,10 +788,10 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // ---------------------------------------------------------------- launchers
-template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false>
+template <int D, bool CAUSAL, bool PER_TOKEN, bool TRACE = false, bool RAGGED = false, bool SPARSE = false>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<D>;
-  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN, TRACE, RAGGED>;
+  auto kern = sage_attn_kernel<D, CAUSAL, PER_TOKEN, TRACE, RAGGED, SPARSE>;
   static bool configured = false;  // attribute set once per instantiation (idempotent)
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
@@ -720,7 +802,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   const int n_pairs = (n_qtiles + 1) / 2;
   dim3 grid(static_cast<unsigned>(n_pairs * a.BH));
   kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sq, a.sk, a.o, a.BH, a.N, a.sm_scale_log2,
-                                          a.trace, a.trace_ctas);
+                                          a.trace, a.trace_ctas, a.kv_count, a.kv_index, a.skip_lambda);
   return cudaGetLastError();
 }
 
@@ -743,11 +825,13 @@ static cudaError_t launch_attn_v3(const AttnArgs& a, cudaStream_t st) {
 
 // RAGGED instantiations carry the key masking of a partial last key tile; whole-tile problems
 // (N a multiple of 128) use the others, whose non-causal forms have no masking code at all.
-template <int D, bool RAGGED>
+template <int D, bool RAGGED, bool SPARSE = false>
 static cudaError_t launch_attn_d(const AttnArgs& a, cudaStream_t st) {
   if (a.causal)
-    return a.per_token ? launch_attn_t<D, true, true, false, RAGGED>(a, st) : launch_attn_t<D, true, false, false, RAGGED>(a, st);
-  return a.per_token ? launch_attn_t<D, false, true, false, RAGGED>(a, st) : launch_attn_t<D, false, false, false, RAGGED>(a, st);
+    return a.per_token ? launch_attn_t<D, true, true, false, RAGGED, SPARSE>(a, st)
+                       : launch_attn_t<D, true, false, false, RAGGED, SPARSE>(a, st);
+  return a.per_token ? launch_attn_t<D, false, true, false, RAGGED, SPARSE>(a, st)
+                     : launch_attn_t<D, false, false, false, RAGGED, SPARSE>(a, st);
 }
 
 template <bool RAGGED, bool FP8 = false, bool SPARSE = false>
@@ -765,9 +849,11 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
     if (a.D != 128 || a.trace || a.kv_count) return cudaErrorNotSupported;
     return ragged ? launch_attn_128<true, true>(a, st) : launch_attn_128<false, true>(a, st);
   }
-  if (a.kv_count) {  // the block-sparse variant: head dimension 128, untraced, up to 512 key tiles
-    if (a.D != 128 || a.trace || (a.N + 127) / 128 > V3Layout::MAX_LIST) return cudaErrorNotSupported;
-    return ragged ? launch_attn_128<true, false, true>(a, st) : launch_attn_128<false, false, true>(a, st);
+  if (a.kv_count) {  // the block-sparse variant: untraced, up to 512 key tiles
+    static_assert(AttnLayout<64>::MAX_LIST == V3Layout::MAX_LIST, "one list bound for both head dimensions");
+    if (a.trace || (a.N + 127) / 128 > V3Layout::MAX_LIST) return cudaErrorNotSupported;
+    if (a.D == 128) return ragged ? launch_attn_128<true, false, true>(a, st) : launch_attn_128<false, false, true>(a, st);
+    return ragged ? launch_attn_d<64, true, true>(a, st) : launch_attn_d<64, false, true>(a, st);
   }
   if (a.trace) {  // traced builds exist for per-block granularity and whole tiles only
     if (a.per_token || ragged) return cudaErrorNotSupported;

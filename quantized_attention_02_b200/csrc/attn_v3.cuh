@@ -459,15 +459,29 @@ __global__ void __launch_bounds__(512, 1)
       float m_run = -INFINITY;  // block-sparse variant: the row's largest score so far (log2 units)
       float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
       bool ok = true;
+      // Block-sparse variant: the group's four warps meet at one named barrier per key tile (the
+      // stage-2 vote).  A warp whose bounded wait gave up still takes that barrier once for the
+      // step it leaves in, with bit 1 in the vote, and the whole group leaves there: no warp is
+      // left waiting at a barrier that the others never reach.
+      int* vote = sSkipVote + t * 3;
+      auto leave_vote = [&](int jj) {
+        if constexpr (SPARSE) {
+          if (jj < n_iter[t]) {
+            if (r == 0) vote[(jj + 1) % 3] = 0;
+            if (lane == 0) atomicOr(vote + jj % 3, 2);
+            group_sync(3 + t);
+          }
+        }
+      };
       for (int j = 0; j < n_iter[t]; ++j) {
-        if (!wait_warp(bar_s_full + t, j & 1)) { ok = false; break; }
+        if (!wait_warp(bar_s_full + t, j & 1)) { leave_vote(j); ok = false; break; }
         tc_fence_after();
         if (r == 0) stamp((3 * t) * n_kv_total + j);
         const float* skj = sks_t + (j & 1) * 128;  // per-token key scales of key tile j (shared memory)
         float sk_next = 0.f;
         if constexpr (PER_TOKEN) {
           if (j + 1 < n_iter[t]) sk_next = key_scale(j + 1);
-          if (!wait_warp(bar_sks + t, j & 1)) { ok = false; break; }
+          if (!wait_warp(bar_sks + t, j & 1)) { leave_vote(j); ok = false; break; }
         }
         // masked keys: past the diagonal (causal) and past N (a partial last key tile); keys
         // c > cmax of this tile are left out of the maximum and get P~ = 0
@@ -520,11 +534,12 @@ __global__ void __launch_bounds__(512, 1)
         bool keep_tile = true;
         if constexpr (SPARSE) {
           const bool row_keeps = q_row < N && !(mx < m_run - skip_lambda);
-          int* vote = sSkipVote + t * 3;
           if (r == 0) vote[(j + 1) % 3] = 0;
           if (__any_sync(0xffffffffu, row_keeps) && lane == 0) atomicOr(vote + j % 3, 1);
           group_sync(3 + t);
-          keep_tile = *reinterpret_cast<volatile int*>(vote + j % 3) != 0;
+          const int v = *reinterpret_cast<volatile int*>(vote + j % 3);
+          if (v & 2) { ok = false; break; }  // a warp of the group gave up waiting
+          keep_tile = (v & 1) != 0;
           if (keep_tile && q_row < N) m_run = fmaxf(m_run, mx);
         }
 
@@ -699,13 +714,13 @@ __global__ void __launch_bounds__(512, 1)
         if (!keep_tile) {
           // stage 2 dropped the tile: no exp2 pass and no P~.  The wait for the previous P.V keeps
           // this group's bar_o_done waits one phase apart and orders the reuse of the flag slot.
-          if (j > 0 && !wait_warp(bar_o_done + t, (j - 1) & 1)) { ok = false; break; }
+          if (j > 0 && !wait_warp(bar_o_done + t, (j - 1) & 1)) { leave_vote(j + 1); ok = false; break; }
           tc_fence_before();
           mbar_arrive(bar_s_free + t);  // S_t read (for the maximum)
           if (r == 0) sPvKeep[t * 2 + (j & 1)] = 0;
           mbar_arrive(bar_p_lo + t);
           mbar_arrive(bar_p_hi + t);
-        } else if (!(diag ? exp_pass_masked() : exp_pass())) { ok = false; break; }
+        } else if (!(diag ? exp_pass_masked() : exp_pass())) { leave_vote(j + 1); ok = false; break; }
         if constexpr (PER_TOKEN) {  // key scales of tile j+1 into the other buffer
           if (j + 1 < n_iter[t]) {
             sks_t[((j + 1) & 1) * 128 + r] = sk_next;

@@ -108,9 +108,9 @@ int check_scale(float sm_scale) {
 
 int check_gran(int g) { return (g == SAGE_PER_TOKEN || g == SAGE_PER_BLOCK) ? SAGE_OK : SAGE_ERR_INVALID; }
 
-// The block-sparse variant: head dimension 128 and at most 512 key tiles (N <= 65536).
-int check_sparse(int N, int d) {
-  return (d == 128 && (N + 127) / 128 <= sage::kSparseMaxKeyBlocks) ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
+// The block-sparse variant: at most 512 key tiles (N <= 65536), either head dimension.
+int check_sparse(int N) {
+  return (N + 127) / 128 <= sage::kSparseMaxKeyBlocks ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
@@ -383,7 +383,7 @@ int sage_sparse_predict(const void* q, const void* k, int B, int H, int N, int d
   if (!q || !k || !kv_count || !kv_index) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_sparse(N))) return rc;
   if ((rc = check_scale(sm_scale))) return rc;
   if (!(tau > 0.f && tau <= 1.f) || !std::isfinite(theta)) return SAGE_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k)) return SAGE_ERR_INVALID;
@@ -407,7 +407,7 @@ int sage_attn_fwd_sparse_quantized(const int8_t* q8, const int8_t* k8, const flo
   if (!q8 || !k8 || !sq || !sk || !v || !o || !kv_count || !kv_index) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_sparse(N))) return rc;
   if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
   if (!(skip_lambda > 0.f)) return SAGE_ERR_INVALID;  // +inf: no second stage; NaN rejected
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(sk)) return SAGE_ERR_INVALID;
@@ -421,7 +421,7 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
   if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if ((rc = check_sparse(N, d))) return rc;
+  if ((rc = check_sparse(N))) return rc;
   if ((rc = check_scale(sm_scale)) || (rc = check_gran(granularity))) return rc;
   if (!(tau > 0.f && tau <= 1.f) || !std::isfinite(theta) || !(skip_lambda > 0.f)) return SAGE_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;

@@ -107,6 +107,11 @@ SMALL = [
     W.Workload("sp_small_win_causal", 1, 2, 2048, 128, True, True, window=512, align=12.0),
     W.Workload("sp_small_ragged_tok", 1, 2, 1500, 128, False, False, window=384, align=10.0),
     W.Workload("sp_small_ragged_causal_tok", 1, 2, 1100, 128, True, False, window=256, align=10.0),
+    # head dimension 64 (the video-DiT kernel)
+    W.Workload("sp_small_win_d64", 1, 2, 2048, 64, False, True, window=512, align=9.0, bias_std=4.0),
+    W.Workload("sp_small_win_causal_d64", 1, 2, 2048, 64, True, True, window=512, align=9.0),
+    W.Workload("sp_small_ragged_tok_d64", 1, 2, 1500, 64, False, False, window=384, align=8.0),
+    W.Workload("sp_small_ragged_causal_tok_d64", 1, 2, 1100, 64, True, False, window=256, align=8.0),
 ]
 
 
@@ -138,10 +143,11 @@ def test_sparse_fused_kernel_matches_the_oracle(sa, w, lam):
     assert torch.equal(o2, o)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1024, 1000])
-def test_all_blocks_without_stage_two_equal_the_dense_kernel(sa, causal, N):
-    w = W.Workload("sp_dense", 1, 3, N, 128, causal, True, n_out=4, out_mag=20.0)
+def test_all_blocks_without_stage_two_equal_the_dense_kernel(sa, causal, N, d):
+    w = W.Workload("sp_dense", 1, 3, N, d, causal, True, n_out=4, out_mag=20.0)
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     km, q8, k8, sq, sk = sa.empty_quantized(q, 1)
     sa.sage_smooth_k(k, km)
@@ -160,10 +166,11 @@ def test_all_blocks_without_stage_two_equal_the_dense_kernel(sa, causal, N):
     assert torch.equal(o_dense, o_sparse)
 
 
-def test_random_block_lists(sa):
+@pytest.mark.parametrize("d", [64, 128])
+def test_random_block_lists(sa, d):
     # any ascending lists work (stage 1 bypassed), causal lists holding each query's own blocks
     N, causal = 1536, True
-    w = W.Workload("sp_lists", 1, 2, N, 128, causal, True, n_out=4, out_mag=20.0)
+    w = W.Workload("sp_lists", 1, 2, N, d, causal, True, n_out=4, out_mag=20.0)
     q, k, v = W.make_qkv(w)
     nqb, nkb = sa.sparse_blocks(N)
     rng = np.random.default_rng(5)
@@ -184,7 +191,7 @@ def test_random_block_lists(sa):
     assert_close(o.float().cpu().numpy(), o64, float(v.abs().max()), "random lists")
 
 
-BIG = [W.SPARSE, W.SPARSE_CAUSAL]
+BIG = [W.SPARSE, W.SPARSE_CAUSAL, W.SPARSE_DIT]
 
 
 @pytest.mark.parametrize("w", BIG, ids=lambda w: w.name)
@@ -225,7 +232,8 @@ def test_sparse_full_size(sa, w):
 
 
 def test_sparse_rejects_what_it_does_not_support(sa):
-    q = torch.zeros((1, 1, 256, 64), dtype=torch.float16, device="cuda")
+    # more than 512 key tiles (N > 65536): the kernels' lists hold at most 512
+    q = torch.zeros((1, 1, 65536 + 256, 64), dtype=torch.float16, device="cuda")
     with pytest.raises(sa.SageError) as e:
         sa.sage_attn_fwd_sparse(q, q, q, torch.empty_like(q), False, 0.125, 1, TAU, THETA, LAM)
     assert e.value.status == sa.SAGE_ERR_UNSUPPORTED

@@ -104,12 +104,17 @@ TOKEN64 = Workload("token_n16384_d64_full", 1, 64, 16384, 64, False, False, n_ou
 SPARSE = Workload("sparse_n16384_d128_win2048", 1, 64, 16384, 128, False, True, window=2048, align=14.0)
 SPARSE_CAUSAL = Workload("sparse_n16384_d128_win2048_causal", 1, 64, 16384, 128, True, True, window=2048, align=14.0)
 
+# the video-DiT shape (d = 64) with the same window structure: direction length 12 gives
+# in-window scores about 18 above the rest at d^-1/2 = 0.125
+SPARSE_DIT = Workload("sparse_dit_b2h48_n16384_d64_win2048", 2, 48, 16384, 64, False, True, bias_std=4.0,
+                      window=2048, align=12.0)
+
 # a quarter of the block-sparse workload's heads, for profiler captures
 SPARSE_PROFILE = Workload("sparse_profile_b1h16_n16384_d128_win2048", 1, 16, 16384, 128, False, True, window=2048,
                           align=14.0)
 
 ALL = {w.name: w for w in (TINY, SMALL, LLM, DIT, PROFILE, PROFILE64, TOKEN128, TOKEN64, SPARSE, SPARSE_CAUSAL,
-                           SPARSE_PROFILE)}
+                           SPARSE_DIT, SPARSE_PROFILE)}
 for _n in SWEEP_N:
     for _d in SWEEP_D:
         for _c in (False, True):
