@@ -34,6 +34,13 @@ Parity status (which functions are pinned by checks other than themselves):
                     block is kept; textbook attention over the kept keys; a numpy re-
                     derivation of the predicted map; closed forms of the self-similarity;
                     hand-built second-stage cases; limits of tau and theta)
+  e2m1_encode/decode, fp4_microscale, quant_fp4, quant_v_fp4, attn_fp4 (microscaling FP4
+                    variant, SageAttention3 abstract; sage_oracle_sa3.c) ... pinned (the
+                    E2M1 type of ml_dtypes and PyTorch's E4M3; brute-force nearest search;
+                    worked groups; the tile and channel scales' extremes; hand-derived rows
+                    in tests/golden (the online frames, a subnormal group scale); the FP4
+                    error bound against textbook attention on dequantized inputs; the
+                    envelope of a key on an E2M1 midpoint)
 Every pin is itself checked by tests/test_oracle_mutations.py: planted slips
 (dropped or re-routed roundings, signs, indices, group sizes, operands), each of which
 makes the pins fail.
@@ -50,7 +57,8 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c")]
+_SRCS = [os.path.join(_HERE, f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c",
+                                           "sage_oracle_sa3.c")]
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "libsage_oracle.so")
 _lock = threading.Lock()
@@ -111,6 +119,20 @@ def _load():
             lib.oracle_attn_sparse_tiles.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, f64, i64, i64, vp, f64, vp,
                                                      i64, vp, vp]
             lib.oracle_attn_sparse_tiles.restype = i32
+            lib.oracle_e2m1_encode_n.argtypes = [vp, i64, vp]
+            lib.oracle_e2m1_encode_n.restype = None
+            lib.oracle_e2m1_decode_n.argtypes = [vp, i64, vp]
+            lib.oracle_e2m1_decode_n.restype = None
+            lib.oracle_fp4_microscale.argtypes = [vp, i32, vp]
+            lib.oracle_fp4_microscale.restype = ctypes.c_uint8
+            lib.oracle_quant_fp4.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp]
+            lib.oracle_quant_v_fp4.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp]
+            lib.oracle_attn_fp4.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f64, vp, vp,
+                                            vp, vp]
+            lib.oracle_attn_fp4_rows.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f64,
+                                                 vp, i64, vp, vp, vp]
+            for name in ("oracle_quant_fp4", "oracle_quant_v_fp4", "oracle_attn_fp4", "oracle_attn_fp4_rows"):
+                getattr(lib, name).restype = i32
             for name in ("oracle_smooth_k", "oracle_quant", "oracle_qk_int", "oracle_qk_int_rows", "oracle_attn",
                          "oracle_attn_rows", "oracle_attn_probs", "oracle_attn_fp64"):
                 getattr(lib, name).restype = i32
@@ -377,6 +399,118 @@ def sage_attn_fp8pv(q, k, v, causal: bool, sm_scale: float, per_block: bool, smo
     v8, sv, vm = quant_v_fp8(v, smooth_v)
     o64, o16 = attn_fp8pv(q8, k8, sq, sk, v8, sv, vm, causal, sm_scale, (gq, gk))
     return dict(km=km, q8=q8, sq=sq, k8=k8, sk=sk, v8=v8, sv=sv, vm=vm, o64=o64, o16=o16)
+
+
+# ------------------------------------------------------------------ microscaling FP4 variant
+# (SageAttention3 abstract: attention on FP4 tensor cores with microscaling; readings in
+# sage_oracle_sa3.c)
+FP4_TILE, FP4_GROUP = 128, 16
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Round to the nearest E2M1 value (ties to the even mantissa bit, saturating at +-6):
+    4-bit codes, one per uint8 (bit 3 the sign)."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e2m1_encode_n(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e2m1_decode(c) -> np.ndarray:
+    """Value of E2M1 codes (fp64)."""
+    c = np.ascontiguousarray(c, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e2m1_decode_n(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def fp4_microscale(z):
+    """One group of at most 16 fp32 values: (UE4M3 scale byte, E2M1 codes)."""
+    z = np.ascontiguousarray(z, np.float32)
+    if z.ndim != 1 or z.size > FP4_GROUP:
+        raise ValueError("a group holds at most 16 values")
+    codes = np.zeros(z.size, np.uint8)
+    s8 = _load().oracle_fp4_microscale(_ptr(z), z.size, _ptr(codes))
+    return int(s8), codes
+
+
+def quant_fp4(x, km=None):
+    """Q (km None) or smoothed K to FP4: (codes uint8 [*lead, N, d] one per byte, UE4M3 scales
+    uint8 [*lead, N, d/16], fp32 tile scales [*lead, ceil(N/128)])."""
+    xb = _as_fp16_bits(x)
+    BH, N, d = _bhnd(xb)
+    codes = np.empty(xb.shape, np.uint8)
+    s8 = np.empty(xb.shape[:-1] + (d // FP4_GROUP,), np.uint8)
+    g = np.empty(xb.shape[:-2] + (-(-N // FP4_TILE),), np.float32)
+    kmv = None if km is None else np.ascontiguousarray(km, np.float32)
+    _check(_load().oracle_quant_fp4(_ptr(xb), _ptr(kmv) if kmv is not None else None, BH, N, d, _ptr(codes),
+                                    _ptr(s8), _ptr(g)), "oracle_quant_fp4")
+    return codes, s8, g
+
+
+def quant_v_fp4(v, smooth: bool = True):
+    """V to FP4 along the tokens: (codes uint8 [*lead, N, d], UE4M3 scales uint8
+    [*lead, ceil(N/16), d], channel scales gv fp32 [*lead, d], channel means vm or None)."""
+    vb = _as_fp16_bits(v)
+    BH, N, d = _bhnd(vb)
+    codes = np.empty(vb.shape, np.uint8)
+    s8 = np.empty(vb.shape[:-2] + (-(-N // FP4_GROUP), d), np.uint8)
+    gv = np.empty(vb.shape[:-2] + (d,), np.float32)
+    vm = np.empty(vb.shape[:-2] + (d,), np.float32) if smooth else None
+    _check(_load().oracle_quant_v_fp4(_ptr(vb), BH, N, d, int(bool(smooth)), _ptr(vm) if smooth else None,
+                                      _ptr(gv), _ptr(codes), _ptr(s8)), "oracle_quant_v_fp4")
+    return codes, s8, gv, vm
+
+
+def _fp4_args(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm):
+    u8 = lambda a: np.ascontiguousarray(a, np.uint8)  # noqa: E731
+    f32 = lambda a: np.ascontiguousarray(a, np.float32)  # noqa: E731
+    return (u8(q4), u8(qs), f32(gq), u8(k4), u8(ks), f32(gk), u8(v4), u8(vs), f32(gv),
+            None if vm is None else f32(vm))
+
+
+def attn_fp4(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm, causal: bool, sm_scale: float):
+    """Microscaling FP4 attention (readings in sage_oracle_sa3.c).  Returns (O fp64, O fp16,
+    envelope fp64 [*lead, N, d], unsure uint8 [*lead, N])."""
+    a = _fp4_args(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm)
+    BH, N, d = _bhnd(a[6])
+    o64 = np.empty(a[6].shape, np.float64)
+    o16 = np.empty(a[6].shape, np.uint16)
+    env = np.empty(a[6].shape, np.float64)
+    unsure = np.empty(a[6].shape[:-1], np.uint8)
+    ptrs = [_ptr(x) if x is not None else None for x in a]
+    _check(_load().oracle_attn_fp4(*ptrs, BH, N, d, int(bool(causal)), float(sm_scale), _ptr(o64), _ptr(o16),
+                                   _ptr(env), _ptr(unsure)), "oracle_attn_fp4")
+    return o64, o16.view(np.float16), env, unsure
+
+
+def attn_fp4_rows(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm, bh: int, rows, causal: bool, sm_scale: float):
+    """attn_fp4() for the listed query rows of head bh only (arrays flattened to [BH, ...]).
+    Returns (O fp64 [rows, d], envelope [rows, d], unsure [rows])."""
+    a = _fp4_args(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm)
+    BH, N, d = _bhnd(a[6])
+    if not 0 <= bh < BH:
+        raise ValueError("head index out of range")
+    rows = np.ascontiguousarray(rows, np.int64)
+    o64 = np.empty((rows.size, d), np.float64)
+    env = np.empty((rows.size, d), np.float64)
+    unsure = np.empty(rows.size, np.uint8)
+    ptrs = [_ptr(x) if x is not None else None for x in a]
+    _check(_load().oracle_attn_fp4_rows(*ptrs, bh, N, d, int(bool(causal)), float(sm_scale), _ptr(rows),
+                                        rows.size, _ptr(o64), _ptr(env), _ptr(unsure)), "oracle_attn_fp4_rows")
+    return o64, env, unsure
+
+
+def sage_attn_fp4(q, k, v, causal: bool, sm_scale: float, smooth_v: bool = True):
+    """The FP4 variant in order: smooth K, Q and K to FP4, V to FP4 (smoothed), attention with
+    microscaled FP4 P~.  Returns every intermediate."""
+    km = smooth_k(k)
+    q4, qs, gq = quant_fp4(q)
+    k4, ks, gk = quant_fp4(k, km)
+    v4, vs, gv, vm = quant_v_fp4(v, smooth_v)
+    o64, o16, env, unsure = attn_fp4(q4, qs, gq, k4, ks, gk, v4, vs, gv, vm, causal, sm_scale)
+    return dict(km=km, q4=q4, qs=qs, gq=gq, k4=k4, ks=ks, gk=gk, v4=v4, vs=vs, gv=gv, vm=vm, o64=o64, o16=o16,
+                env=env, unsure=unsure)
 
 
 # ------------------------------------------------------------------ block-sparse variant

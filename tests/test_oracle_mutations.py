@@ -12,7 +12,8 @@ cannot tell a slip from the reading it pins shows up here.
 The readings pinned are those of the SageAttention summary page (Summary bullets
 1-2: INT8 Q.K^T after smoothing K, P.V in fp16; idea I1: the K shift) and of the
 SageAttention2 abstract for the FP8 P.V variant (E4M3 P~ and V, V smoothing) and of
-the SpargeAttn abstract for the block-sparse variant (predicted map, softmax-aware skip).
+the SpargeAttn abstract for the block-sparse variant (predicted map, softmax-aware skip) and
+of the SageAttention3 abstract for the microscaling FP4 variant (E2M1 codes, UE4M3 scales).
 """
 import concurrent.futures
 import os
@@ -22,9 +23,10 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRCS = {f: os.path.join(ROOT, "oracle", f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c")}
+SRCS = {f: os.path.join(ROOT, "oracle", f) for f in ("sage_oracle.c", "sage_oracle_sa2.c", "sage_oracle_sparse.c",
+                                                        "sage_oracle_sa3.c")}
 PINS = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py", "test_oracle_pins_fp8.py",
-                                                 "test_oracle_pins_sparse.py")]
+                                                 "test_oracle_pins_sparse.py", "test_oracle_pins_fp4.py")]
 
 # (name, text in sage_oracle.c, replacement, expected number of occurrences)
 BASE_MUTATIONS = [
@@ -91,8 +93,29 @@ SPARSE_MUTATIONS = [
      "        }\n        used[b] = 1;", 1),
 ]
 
+# (name, text in sage_oracle_sa3.c, replacement, expected number of occurrences)
+FP4_MUTATIONS = [
+    ("fp4_ties_to_odd", "(dk == db && (k & 1) == 0)", "(dk == db && (k & 1) == 1)", 1),
+    ("fp4_negative_zero_unsigned", "const uint8_t sign = signbit(x) ? 8 : 0;", "const uint8_t sign = x < 0 ? 8 : 0;", 1),
+    ("fp4_group_scale_over_4", "const float t = gm / 6.0f;", "const float t = gm / 4.0f;", 1),
+    ("fp4_group_max_signed", "if (fabsf(z[i]) > gm) gm = fabsf(z[i]);", "if (z[i] > gm) gm = z[i];", 1),
+    ("fp4_range_448", "#define FP4_RANGE 2688.0f", "#define FP4_RANGE 448.0f", 1),
+    ("fp4_k_not_smoothed", "(km ? km[bh * d + c] : 0.0f)", "0.0f", 2),
+    ("fp4_v_mean_added", "- mean) * r;", "+ mean) * r;", 1),
+    ("fp4_p_shift_12", "#define P_SHIFT 10.0", "#define P_SHIFT 12.0", 1),
+    ("fp4_frame_frozen", "if (mt > m) {", "if (m == -INFINITY) {", 1),
+    ("fp4_row_sum_fp16_terms", "l += p[k];", "l += (double)(_Float16)p[k];", 1),
+    ("fp4_channel_scale_dropped", "const double o = acc[c] * gvc / l", "const double o = acc[c] / l", 1),
+    ("fp4_mean_not_added", "+ (h->vm ? (double)h->vm[c] : 0.0);", "+ 0.0;", 1),
+    ("fp4_key_tile_scale_of_query", "(double)h->gk[j / FP4_TILE]", "(double)h->gk[i / FP4_TILE]", 1),
+    ("fp4_causal_off_by_one", "const int64_t jend = h->causal ? i + 1 : N;", "const int64_t jend = h->causal ? i : N;", 1),
+    ("fp4_envelope_dropped", "b = 2.0 * sd;  /* at most", "b = 0.0;  /* at most", 1),
+    ("fp4_unsure_never", "if (fabs(tmax - nearbyint(tmax)) <= 1e-4) unsure = 1;", ";", 1),
+]
+
 MUTATIONS = ([("sage_oracle.c",) + m for m in BASE_MUTATIONS] + [("sage_oracle_sa2.c",) + m for m in FP8_MUTATIONS]
-             + [("sage_oracle_sparse.c",) + m for m in SPARSE_MUTATIONS])
+             + [("sage_oracle_sparse.c",) + m for m in SPARSE_MUTATIONS]
+             + [("sage_oracle_sa3.c",) + m for m in FP4_MUTATIONS])
 
 CFLAGS = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
 
