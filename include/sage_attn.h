@@ -179,6 +179,49 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
                          int causal, float sm_scale, int granularity, float tau, float theta, float skip_lambda,
                          void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Microscaling FP4 variant, following the SageAttention3 abstract (author pages of Jia Wei and
+ * Haofeng Huang; arXiv 2505.11594): both products of the attention run on Blackwell's FP4 tensor
+ * cores (tcgen05 kind::mxf4nvf4, block16) with microscaling.  Head dimension 128 only
+ * (SAGE_ERR_UNSUPPORTED otherwise).  Formats: E2M1 codes (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their
+ * negatives), two per byte with the even element in the low nibble; one UE4M3 scale per 16
+ * elements along the contraction dimension, e4m3(fl32(max|z| / 6)), codes
+ * e2m1(fl32(z * fl32(1 / scale))); scales stored as the tensor cores' scale atoms: for every 128
+ * rows and 64 elements of the contraction, 512 bytes with row r's four scales at byte
+ * (r % 32) * 16 + (r / 32) * 4.  A second, fp32 scale lifts the range: per 128-token tile of Q
+ * and of smoothed K, g = fl32(a / 2688) with a = the tile's largest |x|, z = fl32(x * fl32(2688 /
+ * a)); per channel of smoothed V the same over all tokens.  P~ = 2^(u - m + 10) in the online
+ * softmax's integer frame m (the ceil of the running row maximum, log2 units), microscaled along
+ * the keys; the row sum uses P~ before rounding.  tiles = ceil(N/128). */
+
+/* Q and K (minus km, the channel means of sage_smooth_k, when km is not null) to FP4.
+ * q, k: fp16 [B,H,N,128] (in); q4, k4: uint8 [B,H,N,64] (out, codes); sfq, sfk: uint8
+ * [B,H,tiles,2,512] (out, scale atoms; rows past N get zero scales); gq, gk: fp32 [B,H,tiles]
+ * (out, tile scales).  No workspace. */
+int sage_quant_qk_fp4(const void* q, const void* k, const float* km, uint8_t* q4, uint8_t* sfq, float* gq,
+                      uint8_t* k4, uint8_t* sfk, float* gk, int B, int H, int N, int d, void* stream);
+
+/* V to FP4 along the tokens (the P.V contraction), smoothed by its exact channel mean when vm is
+ * not null.  v: fp16 [B,H,N,128] (in); v4t: uint8 [B,H,128,tiles*64] (out, codes transposed:
+ * row c holds channel c's codes of keys 0 .. tiles*128-1, keys past N zero); sfv: uint8
+ * [B,H,tiles,2,512] (out, scale atoms with the channels as rows); gv: fp32 [B,H,128] (out, channel
+ * scales); vm: fp32 [B,H,128] (out, channel means) or null.  Allocates a small stream-ordered
+ * workspace (the inverse channel scales). */
+int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, int B, int H, int N, int d,
+                     void* stream);
+
+/* The fused FP4 kernel on quantized inputs (layouts above; vm may be null).  o: fp16
+ * [B,H,N,128] (out).  All pointers 16-byte aligned.  No workspace. */
+int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const float* gq, const uint8_t* k4,
+                                const uint8_t* sfk, const float* gk, const uint8_t* v4t, const uint8_t* sfv,
+                                const float* gv, const float* vm, void* o, int B, int H, int N, int d, int causal,
+                                float sm_scale, void* stream);
+
+/* The whole FP4 variant as a user calls it: smooth K, Q and K to FP4, V to FP4 (smoothed), the
+ * fused kernel.  Allocates its workspace stream-ordered. */
+int sage_attn_fwd_fp4(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                      float sm_scale, void* stream);
+
 /* Debug: the full integer product s[b,h,i,j] = sum_c q8[b,h,i,c] * k8[b,h,j,c] as int32
  * (exact: |s| <= 128*127*127 < 2^31), computed with the same tensor-core path as the fused
  * kernel.  s: int32 [B,H,N,N] (out); needs B*H*N*N < 2^31. */

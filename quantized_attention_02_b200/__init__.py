@@ -57,6 +57,11 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_prep_qk.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
         lib.sage_attn_fwd_fp8pv_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
         lib.sage_attn_fwd_fp8pv.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p]
+        lib.sage_quant_qk_fp4.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_quant_v_fp4.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p]
+        lib.sage_attn_fwd_fp4_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i,
+                                                    _f, _p]
+        lib.sage_attn_fwd_fp4.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _p]
         lib.sage_sparse_predict.argtypes = [_p, _p, _i, _i, _i, _i, _i, _f, _f, _f, _p, _p, _p]
         lib.sage_attn_fwd_sparse_quantized.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _p, _f,
                                                        _p]
@@ -183,6 +188,60 @@ def sage_attn_fwd_fp8pv(q, k, v, o, causal: bool, sm_scale: float, granularity: 
     B, H, N, d = _shape(q)
     _check(get_lib().sage_attn_fwd_fp8pv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
                                          float(sm_scale), int(granularity), _stream(stream)), "sage_attn_fwd_fp8pv")
+
+
+def fp4_tiles(N: int) -> int:
+    """Tiles of 128 tokens of the microscaling FP4 variant: ceil(N/128)."""
+    return (N + 127) // 128
+
+
+def empty_fp4(q, smooth_v: bool = True) -> dict:
+    """Device buffers of the FP4 variant's quantized operands for q-shaped [B,H,N,128] inputs:
+    q4/k4 uint8 [B,H,N,64], sfq/sfk/sfv uint8 [B,H,tiles,2,512], gq/gk fp32 [B,H,tiles],
+    v4t uint8 [B,H,128,tiles*64], gv/vm fp32 [B,H,128] (vm None when not smoothed), km fp32
+    [B,H,128]."""
+    B, H, N, d = _shape(q)
+    t = fp4_tiles(N)
+    u8 = dict(dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    return dict(q4=torch.empty((B, H, N, d // 2), **u8), k4=torch.empty((B, H, N, d // 2), **u8),
+                sfq=torch.empty((B, H, t, 2, 512), **u8), sfk=torch.empty((B, H, t, 2, 512), **u8),
+                sfv=torch.empty((B, H, t, 2, 512), **u8), gq=torch.empty((B, H, t), **f32),
+                gk=torch.empty((B, H, t), **f32), v4t=torch.empty((B, H, d, t * 64), **u8),
+                gv=torch.empty((B, H, d), **f32), vm=torch.empty((B, H, d), **f32) if smooth_v else None,
+                km=torch.empty((B, H, d), **f32))
+
+
+def sage_quant_qk_fp4(q, k, km, q4, sfq, gq, k4, sfk, gk, stream=None) -> None:
+    """Q and K (minus km unless None) to E2M1 codes with UE4M3 scale atoms and fp32 tile scales
+    (microscaling FP4 variant, SageAttention3 abstract)."""
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_quant_qk_fp4(_ptr(q), _ptr(k), _ptr(km), _ptr(q4), _ptr(sfq), _ptr(gq), _ptr(k4), _ptr(sfk),
+                                       _ptr(gk), B, H, N, d, _stream(stream)), "sage_quant_qk_fp4")
+
+
+def sage_quant_v_fp4(v, v4t, sfv, gv, vm=None, stream=None) -> None:
+    """V to E2M1 codes along the tokens (transposed), UE4M3 scale atoms, fp32 channel scales;
+    channel means into vm (V smoothed) unless vm is None."""
+    B, H, N, d = _shape(v)
+    _check(get_lib().sage_quant_v_fp4(_ptr(v), _ptr(v4t), _ptr(sfv), _ptr(gv), _ptr(vm), B, H, N, d, _stream(stream)),
+           "sage_quant_v_fp4")
+
+
+def sage_attn_fwd_fp4_quantized(q4, sfq, gq, k4, sfk, gk, v4t, sfv, gv, vm, o, causal: bool, sm_scale: float,
+                                stream=None) -> None:
+    B, H, N, d = _shape(o)
+    _check(get_lib().sage_attn_fwd_fp4_quantized(_ptr(q4), _ptr(sfq), _ptr(gq), _ptr(k4), _ptr(sfk), _ptr(gk),
+                                                 _ptr(v4t), _ptr(sfv), _ptr(gv), _ptr(vm), _ptr(o), B, H, N, d,
+                                                 int(bool(causal)), float(sm_scale), _stream(stream)),
+           "sage_attn_fwd_fp4_quantized")
+
+
+def sage_attn_fwd_fp4(q, k, v, o, causal: bool, sm_scale: float, stream=None) -> None:
+    """The whole microscaling FP4 variant (smooth K, FP4 Q, K and V, the fused FP4 kernel)."""
+    B, H, N, d = _shape(q)
+    _check(get_lib().sage_attn_fwd_fp4(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, int(bool(causal)),
+                                       float(sm_scale), _stream(stream)), "sage_attn_fwd_fp4")
 
 
 def sparse_blocks(N: int) -> tuple[int, int]:

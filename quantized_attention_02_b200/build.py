@@ -34,7 +34,7 @@ SOURCES = {
     "sparse_kernels.cu": [],
 }
 HEADERS = ["sm100_ptx.cuh", "attn_kernels.cuh", "attn_v3.cuh", "prep_kernels.cuh", "workspace.cuh",
-           "sparse_kernels.cuh"]
+           "sparse_kernels.cuh", "fp4_codes.cuh", "attn_fp4.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

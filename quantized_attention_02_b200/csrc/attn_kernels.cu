@@ -28,6 +28,7 @@
 #include <type_traits>
 
 #include "attn_kernels.cuh"
+#include "fp4_codes.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sage {
@@ -683,6 +684,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 #include "attn_v3.cuh"
+#include "attn_fp4.cuh"
 
 // ---------------------------------------------------------------- debug: INT32 S = q8 k8^T
 // One CTA per (128-row query tile, head), all along grid x.  Thread 0 issues the TMA loads and the same
@@ -862,6 +864,27 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   }
   if (a.D == 128) return ragged ? launch_attn_128<true>(a, st) : launch_attn_128<false>(a, st);
   return ragged ? launch_attn_d<64, true>(a, st) : launch_attn_d<64, false>(a, st);
+}
+
+template <bool CAUSAL, bool RAGGED>
+static cudaError_t launch_attn_fp4_t(const Fp4Args& a, cudaStream_t st) {
+  auto kern = sage_attn_fp4_kernel<CAUSAL, RAGGED>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4Layout::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const unsigned grid = static_cast<unsigned>((a.N + 127) / 128) * static_cast<unsigned>(a.BH);
+  kern<<<grid, Fp4Layout::THREADS, Fp4Layout::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sfq, a.sfk, a.sfv, a.gq, a.gk,
+                                                          a.gv, a.vm, a.o, a.N, a.sm_scale_log2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fp4(const Fp4Args& a, cudaStream_t st) {
+  const bool ragged = a.N % 128 != 0;
+  if (a.causal) return ragged ? launch_attn_fp4_t<true, true>(a, st) : launch_attn_fp4_t<true, false>(a, st);
+  return ragged ? launch_attn_fp4_t<false, true>(a, st) : launch_attn_fp4_t<false, false>(a, st);
 }
 
 template <int D>

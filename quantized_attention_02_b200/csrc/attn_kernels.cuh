@@ -34,6 +34,26 @@ struct AttnArgs {
 };
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+
+// Microscaling FP4 variant (head dimension 128): E2M1 codes, UE4M3 scale atoms and fp32 tile /
+// channel scales as written by launch_quant_qk_fp4 / launch_quant_v_fp4.
+struct Fp4Args {
+  const CUtensorMap* tm_q;  // uint8 [BH][N][64] (3-D), box {64, 128, 1}, 64 B swizzle
+  const CUtensorMap* tm_k;  // the same for K
+  const CUtensorMap* tm_v;  // uint8 [BH][128][ceil(N/128) * 64] (V transposed), box {64, 128, 1}, 64 B swizzle
+  const uint8_t* sfq;       // [BH][ceil(N/128)][2][512] scale atoms of Q, K and V
+  const uint8_t* sfk;
+  const uint8_t* sfv;
+  const float* gq;          // [BH][ceil(N/128)] tile scales of Q and K
+  const float* gk;
+  const float* gv;          // [BH][128] channel scales of V
+  const float* vm;          // [BH][128] channel means of V, or null
+  __half* o;                // fp16 [BH][N][128]
+  int BH, N;
+  bool causal;
+  float sm_scale_log2;      // sm_scale * log2(e)
+};
+cudaError_t launch_attn_fp4(const Fp4Args& a, cudaStream_t st);
 cudaError_t launch_qk_debug(const CUtensorMap& tq, const CUtensorMap& tk, int32_t* s, int BH, int N, int D,
                             cudaStream_t st);
 // One warp waits on an mbarrier that nothing arrives on, with the pipelines' bounded wait.

@@ -86,6 +86,12 @@ bool make_o_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
   return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// FP4 codes: [BH][rows][cols] bytes (Q and K: rows = N tokens, cols = 64; V transposed: rows =
+// 128 channels, cols = tiles * 64), boxes of 64 bytes x 128 rows, 64-byte swizzle.
+bool make_fp4_map3(CUtensorMap* map, const void* base, int rows, int BH, int cols) {
+  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, BH, cols, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 bool make_qk_map(CUtensorMap* map, const int8_t* base, long long rows, int D) {
   return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, D, D,
                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
@@ -504,6 +510,133 @@ int sage_last_device_error(void* stream) {
   cudaError_t e;
   const int code = sage::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);
   return code < 0 ? SAGE_ERR_CUDA : code;
+}
+
+
+// ---------------------------------------------------------------- microscaling FP4 variant
+int sage_quant_qk_fp4(const void* q, const void* k, const float* km, uint8_t* q4, uint8_t* sfq, float* gq,
+                      uint8_t* k4, uint8_t* sfk, float* gk, int B, int H, int N, int d, void* stream) {
+  if (!q || !k || !q4 || !sfq || !gq || !k4 || !sfk || !gk) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q4) || !aligned16(k4) || !aligned16(sfq) || !aligned16(sfk))
+    return SAGE_ERR_INVALID;
+  return cuda_status(sage::launch_quant_qk_fp4(static_cast<const __half*>(q), static_cast<const __half*>(k), km, q4,
+                                               sfq, gq, k4, sfk, gk, B * H, N, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, int B, int H, int N, int d,
+                     void* stream) {
+  if (!v || !v4t || !sfv || !gv) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (!aligned16(v) || !aligned16(v4t) || !aligned16(sfv)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  void* ws = nullptr;
+  if (sage::workspace_alloc(&ws, static_cast<size_t>(BH) * d * 4, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  rc = cuda_status(sage::launch_quant_v_fp4(static_cast<const __half*>(v), v4t, sfv, gv, vm, static_cast<float*>(ws),
+                                            BH, N, st));
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
+}
+
+int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const float* gq, const uint8_t* k4,
+                                const uint8_t* sfk, const float* gk, const uint8_t* v4t, const uint8_t* sfv,
+                                const float* gv, const float* vm, void* o, int B, int H, int N, int d, int causal,
+                                float sm_scale, void* stream) {
+  if (!q4 || !sfq || !gq || !k4 || !sfk || !gk || !v4t || !sfv || !gv || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_scale(sm_scale))) return rc;
+  if (!aligned16(q4) || !aligned16(k4) || !aligned16(v4t) || !aligned16(sfq) || !aligned16(sfk) || !aligned16(sfv) ||
+      !aligned16(o))
+    return SAGE_ERR_INVALID;
+  const int BH = B * H, tiles = (N + 127) / 128;
+  CUtensorMap tq, tk, tv;
+  if (!make_fp4_map3(&tq, q4, N, BH, 64) || !make_fp4_map3(&tk, k4, N, BH, 64) ||
+      !make_fp4_map3(&tv, v4t, 128, BH, tiles * 64))
+    return SAGE_ERR_CUDA;
+  sage::Fp4Args a{};
+  a.tm_q = &tq;
+  a.tm_k = &tk;
+  a.tm_v = &tv;
+  a.sfq = sfq;
+  a.sfk = sfk;
+  a.sfv = sfv;
+  a.gq = gq;
+  a.gk = gk;
+  a.gv = gv;
+  a.vm = vm;
+  a.o = static_cast<__half*>(o);
+  a.BH = BH;
+  a.N = N;
+  a.causal = causal != 0;
+  a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  return cuda_status(sage::launch_attn_fp4(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sage_attn_fwd_fp4(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                      float sm_scale, void* stream) {
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
+  int rc = check_shape(B, H, N, d);
+  if (rc) return rc;
+  if (d != 128) return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_scale(sm_scale))) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const size_t tiles = static_cast<size_t>((N + 127) / 128);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t codes = up(static_cast<size_t>(BH) * N * 64), atoms = up(static_cast<size_t>(BH) * tiles * 1024);
+  const size_t tscales = up(static_cast<size_t>(BH) * tiles * 4), chan = up(static_cast<size_t>(BH) * d * 4);
+  const size_t off_k4 = codes;
+  const size_t off_v4 = off_k4 + codes;
+  const size_t off_sfq = off_v4 + up(static_cast<size_t>(BH) * 128 * tiles * 64);
+  const size_t off_sfk = off_sfq + atoms;
+  const size_t off_sfv = off_sfk + atoms;
+  const size_t off_gq = off_sfv + atoms;
+  const size_t off_gk = off_gq + tscales;
+  const size_t off_km = off_gk + tscales;
+  const size_t off_gv = off_km + chan;
+  const size_t off_vm = off_gv + chan;
+  const size_t off_rv = off_vm + chan;
+  const size_t total = off_rv + chan;
+  void* ws = nullptr;
+  if (sage::workspace_alloc(&ws, total, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SAGE_ERR_NOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* km = reinterpret_cast<float*>(w + off_km);
+  float* gv = reinterpret_cast<float*>(w + off_gv);
+  float* vm = reinterpret_cast<float*>(w + off_vm);
+  nvtxRangePushA("sage_fp4_prep");
+  rc = cuda_status(sage::launch_smooth_k(static_cast<const __half*>(k), km, BH, N, d, st));
+  if (!rc)
+    rc = cuda_status(sage::launch_quant_qk_fp4(static_cast<const __half*>(q), static_cast<const __half*>(k), km, w,
+                                               w + off_sfq, reinterpret_cast<float*>(w + off_gq), w + off_k4,
+                                               w + off_sfk, reinterpret_cast<float*>(w + off_gk), BH, N, st));
+  if (!rc)
+    rc = cuda_status(sage::launch_quant_v_fp4(static_cast<const __half*>(v), w + off_v4, w + off_sfv, gv, vm,
+                                              reinterpret_cast<float*>(w + off_rv), BH, N, st));
+  nvtxRangePop();
+  nvtxRangePushA("sage_fp4_fused");
+  if (!rc)
+    rc = sage_attn_fwd_fp4_quantized(w, w + off_sfq, reinterpret_cast<float*>(w + off_gq), w + off_k4, w + off_sfk,
+                                     reinterpret_cast<float*>(w + off_gk), w + off_v4, w + off_sfv, gv, vm, o, B, H, N,
+                                     d, causal, sm_scale, stream);
+  nvtxRangePop();
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
+  return rc;
 }
 
 }  // extern "C"

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <type_traits>
 
+#include "fp4_codes.cuh"
 #include "prep_kernels.cuh"
 
 namespace sage {
@@ -464,10 +465,14 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-template <int D, bool SMOOTH>
+// FP4 = true: the statistics of the microscaling FP4 variant's V instead of FP8 codes: the same
+// exact channel mean (vm), the channel scale sv = fl32(a / 2688) and its inverse rv =
+// fl32(2688 / a) (2688 = 6 * 448: the largest E2M1 code times the largest E4M3 scale); no codes.
+template <int D, bool SMOOTH, bool FP4 = false>
 __global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __half* __restrict__ v,
                                                                      uint8_t* __restrict__ v8, float* __restrict__ sv,
-                                                                     float* __restrict__ vm, int N) {
+                                                                     float* __restrict__ vm, int N,
+                                                                     float* __restrict__ rv = nullptr) {
   constexpr int T = D / 8;                 // threads per token row (one 16-byte piece each)
   constexpr int R = kSmoothThreads / T;    // rows per pass
   constexpr int U = 4;                     // passes in flight
@@ -584,46 +589,50 @@ __global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __hal
     float mean = 0.f;
     if constexpr (SMOOTH) mean = __fmul_rn(__fdiv_rn(__ll2float_rn(s), static_cast<float>(N)), 5.9604644775390625e-08f);
     const float a = fmaxf(0.f, fmaxf(__fsub_rn(hi, mean), __fsub_rn(mean, lo)));
+    constexpr float kRange = FP4 ? 2688.0f : 448.0f;
     float scale = 0.f, inv = 0.f;
     if (a > 0.f) {
-      scale = __fdiv_rn(a, 448.0f);
-      inv = __fdiv_rn(448.0f, a);
+      scale = __fdiv_rn(a, kRange);
+      inv = __fdiv_rn(kRange, a);
     }
     s_vm[c] = mean;
     s_inv[c] = inv;
     if (rank == 0) {
       sv[static_cast<size_t>(bh) * D + c] = scale;
       if constexpr (SMOOTH) vm[static_cast<size_t>(bh) * D + c] = mean;
+      if constexpr (FP4) rv[static_cast<size_t>(bh) * D + c] = inv;
     }
   }
   cluster.sync();  // every CTA keeps its partials in place until all have read them
+  if constexpr (!FP4) {
 
-  // ---- pass 2: codes of this CTA's token slice
-  float m8[8], i8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    m8[i] = s_vm[piece * 8 + i];
-    i8[i] = s_inv[piece * 8 + i];
-  }
-  uint8_t* out = v8 + (static_cast<size_t>(bh) * N) * D + piece * 8;
-  for (int t = t0 + row; t < t1; t += U * R) {
-    uint4 w[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      w[u] = (t + u * R < t1) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D))
-                              : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (t + u * R >= t1) continue;
-      float x[8];
-      unpack8(w[u], x);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if constexpr (SMOOTH) x[i] = __fsub_rn(x[i], m8[i]);
-        x[i] = __fmul_rn(x[i], i8[i]);
+    // ---- pass 2: codes of this CTA's token slice
+    float m8[8], i8[8];
+  #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      m8[i] = s_vm[piece * 8 + i];
+      i8[i] = s_inv[piece * 8 + i];
+    }
+    uint8_t* out = v8 + (static_cast<size_t>(bh) * N) * D + piece * 8;
+    for (int t = t0 + row; t < t1; t += U * R) {
+      uint4 w[U];
+  #pragma unroll
+      for (int u = 0; u < U; ++u)
+        w[u] = (t + u * R < t1) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t + u * R) * D))
+                                : make_uint4(0u, 0u, 0u, 0u);
+  #pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (t + u * R >= t1) continue;
+        float x[8];
+        unpack8(w[u], x);
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if constexpr (SMOOTH) x[i] = __fsub_rn(x[i], m8[i]);
+          x[i] = __fmul_rn(x[i], i8[i]);
+        }
+        *reinterpret_cast<uint2*>(out + static_cast<size_t>(t + u * R) * D) =
+            make_uint2(e4m3x4(x[0], x[1], x[2], x[3]), e4m3x4(x[4], x[5], x[6], x[7]));
       }
-      *reinterpret_cast<uint2*>(out + static_cast<size_t>(t + u * R) * D) =
-          make_uint2(e4m3x4(x[0], x[1], x[2], x[3]), e4m3x4(x[4], x[5], x[6], x[7]));
     }
   }
 }
@@ -648,9 +657,9 @@ static cudaError_t launch_smooth_d(const __half* k, float* km, int BH, int N, cu
   return cudaLaunchKernelEx(&cfg, smooth_k_kernel<D>, k, km, N);
 }
 
-template <int D>
+template <int D, bool FP4 = false>
 static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N,
-                                        cudaStream_t st) {
+                                        cudaStream_t st, float* rv = nullptr) {
   int ctas = 1;  // the cluster size of smooth_k: >= kSmoothTokensPerCta tokens per CTA, at most 8
   while (ctas < kSmoothMaxCtas && N / (2 * ctas) >= kSmoothTokensPerCta) ctas *= 2;
   cudaLaunchConfig_t cfg{};
@@ -665,8 +674,8 @@ static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8, float* sv,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (vm) return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, true>, v, v8, sv, vm, N);
-  return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, false>, v, v8, sv, vm, N);
+  if (vm) return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, true, FP4>, v, v8, sv, vm, N, rv);
+  return cudaLaunchKernelEx(&cfg, quant_v_fp8_kernel<D, false, FP4>, v, v8, sv, vm, N, rv);
 }
 
 cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* vm, int BH, int N, int D,
@@ -741,6 +750,130 @@ cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, i
                             float* sk, int BH, int N, int D, bool per_token, cudaStream_t st) {
   return D == 128 ? launch_quant_qk_d<128>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st)
                   : launch_quant_qk_d<64>(q, k, km, q8, k8, sq, sk, BH, N, per_token, st);
+}
+
+// ---------------------------------------------------------------- microscaling FP4 variant
+// (SageAttention3 abstract: attention on FP4 tensor cores with microscaling).  Formats: E2M1
+// codes, two per byte (the even element in the low nibble), one UE4M3 scale per 16 elements
+// along the contraction dimension, chosen as e4m3(fl32(max|z| / 6)), codes
+// e2m1(fl32(z * fl32(1 / scale))).  Scales are stored in the tensor cores' scale atoms: 512 bytes
+// per 128 rows x 4 scales (64 elements of the contraction), row r's four scales at byte
+// (r % 32) * 16 + (r / 32) * 4.
+
+// Q (SMOOTH = false) or K minus its channel mean km: one CTA per (head, 128-token tile), one
+// thread per token.  g[bh, tile] = fl32(a / 2688) with a the tile's largest |x|; z = fl32(x *
+// fl32(2688 / a)); codes [BH][N][64 bytes]; scale atoms sf [BH][tiles][2][512].
+template <bool SMOOTH>
+__global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict__ x, const float* __restrict__ km,
+                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                        float* __restrict__ g, int N) {
+  constexpr int D = 128;
+  const int nt = (N + 127) / 128;
+  const int bh = static_cast<int>(blockIdx.x) / nt, tile = static_cast<int>(blockIdx.x) % nt;
+  const int r = threadIdx.x, row = tile * 128 + r;
+  const bool live = row < N;
+  __shared__ float s_km[D];
+  __shared__ float s_max[4];
+  s_km[r] = SMOOTH ? km[static_cast<size_t>(bh) * D + r] : 0.f;
+  __syncthreads();
+  float v[D];
+  const uint4* src = reinterpret_cast<const uint4*>(x + (static_cast<size_t>(bh) * N + (live ? row : 0)) * D);
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    float f[8];
+    unpack8(live ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u), f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[8 * i + k] = (SMOOTH && live) ? __fsub_rn(f[k], s_km[8 * i + k]) : f[k];
+      a = fmaxf(a, fabsf(v[8 * i + k]));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  if ((r & 31) == 0) s_max[r >> 5] = a;
+  __syncthreads();
+  a = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+  const float rr = a > 0.f ? __fdiv_rn(2688.0f, a) : 0.f;
+  if (r == 0) g[static_cast<size_t>(bh) * nt + tile] = __fdiv_rn(a, 2688.0f);
+  uint32_t w[16];
+  uint32_t sfw[2] = {0u, 0u};
+#pragma unroll
+  for (int gi = 0; gi < D / 16; ++gi) {
+    float z[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) z[k] = __fmul_rn(v[16 * gi + k], rr);
+    const uint32_t s8 = microscale16(z, w[2 * gi], w[2 * gi + 1]);
+    sfw[gi >> 2] |= (live ? s8 : 0u) << (8 * (gi & 3));
+  }
+  if (live) {
+    uint4* dst = reinterpret_cast<uint4*>(codes + (static_cast<size_t>(bh) * N + row) * (D / 2));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
+  uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (r & 31) * 16 + (r >> 5) * 4;
+  *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
+  *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+}
+
+// V codes along the tokens: one CTA per (head, 128-key tile), one thread per channel.
+// z = fl32(fl32(v - vm) * rv), groups of 16 keys; codes transposed [BH][128][n_tiles * 64 bytes]
+// (keys past N: zero codes, outside every group's maximum); scale atoms [BH][tiles][2][512] with
+// the channels as rows.
+template <bool SMOOTH>
+__global__ void __launch_bounds__(128) quant_v_fp4_kernel(const __half* __restrict__ v, const float* __restrict__ vm,
+                                                          const float* __restrict__ rv, uint8_t* __restrict__ codes_t,
+                                                          uint8_t* __restrict__ sf, int N) {
+  constexpr int D = 128;
+  const int nt = (N + 127) / 128;
+  const int bh = static_cast<int>(blockIdx.x) / nt, tile = static_cast<int>(blockIdx.x) % nt;
+  const int c = threadIdx.x;
+  const float mean = SMOOTH ? vm[static_cast<size_t>(bh) * D + c] : 0.f;
+  const float rr = rv[static_cast<size_t>(bh) * D + c];
+  const __half* src = v + (static_cast<size_t>(bh) * N + tile * 128) * D + c;
+  const int n_live = min(128, N - tile * 128);
+  uint32_t w[16];
+  uint32_t sfw[2] = {0u, 0u};
+#pragma unroll
+  for (int gi = 0; gi < 8; ++gi) {
+    float z[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int t = 16 * gi + k;
+      const float xv = t < n_live ? __half2float(src[static_cast<size_t>(t) * D]) : 0.f;
+      z[k] = t < n_live ? __fmul_rn(SMOOTH ? __fsub_rn(xv, mean) : xv, rr) : 0.f;
+    }
+    const uint32_t s8 = microscale16(z, w[2 * gi], w[2 * gi + 1]);
+    sfw[gi >> 2] |= s8 << (8 * (gi & 3));
+  }
+  uint4* dst = reinterpret_cast<uint4*>(codes_t + (static_cast<size_t>(bh) * D + c) * (static_cast<size_t>(nt) * 64) +
+                                        tile * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (c & 31) * 16 + (c >> 5) * 4;
+  *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
+  *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+}
+
+cudaError_t launch_quant_qk_fp4(const __half* q, const __half* k, const float* km, uint8_t* q4, uint8_t* sfq,
+                                float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
+  quant_fp4_kernel<false><<<blocks, 128, 0, st>>>(q, nullptr, q4, sfq, gq, N);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (km) quant_fp4_kernel<true><<<blocks, 128, 0, st>>>(k, km, k4, sfk, gk, N);
+  else quant_fp4_kernel<false><<<blocks, 128, 0, st>>>(k, nullptr, k4, sfk, gk, N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v_fp4(const __half* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, float* rv, int BH,
+                               int N, cudaStream_t st) {
+  cudaError_t e = launch_quant_v_fp8_d<128, true>(v, nullptr, gv, vm, BH, N, st, rv);
+  if (e != cudaSuccess) return e;
+  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
+  if (vm) quant_v_fp4_kernel<true><<<blocks, 128, 0, st>>>(v, vm, rv, v4t, sfv, N);
+  else quant_v_fp4_kernel<false><<<blocks, 128, 0, st>>>(v, nullptr, rv, v4t, sfv, N);
+  return cudaGetLastError();
 }
 
 }  // namespace sage

@@ -239,6 +239,31 @@ __device__ __forceinline__ void mma_f8_ss_warp(uint32_t d_tmem, uint64_t a_desc,
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Block-scaled FP4 product: A and B E2M1 (two per byte) from shared memory, one UE4M3 scale per
+// 16 elements of K read from tensor memory at sfa / sfb (K = 64 per instruction: four scales per
+// row, one tensor-memory column per lane quadrant after tcgen05.cp 32x128b.warpx4).
+__device__ __forceinline__ void mma_fp4_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 ln;\n\t"
+      "elect.sync ln|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Shared memory -> tensor memory: 32 rows of 128 bits (a 512-byte scale atom, rows 16 bytes
+// apart), copied to all four lane quadrants (lane q*32 + m gets row m in 4 columns).  Issued by
+// the same elected lane as the products that read it, so they run after it.
+__device__ __forceinline__ void tmem_cp_32x128b_warp(uint32_t taddr, uint64_t s_desc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 ln;\n\t"
+      "elect.sync ln|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(s_desc)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 ln;\n\t"
@@ -352,6 +377,14 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 // Instruction descriptor fields (32-bit): D format bits 4-5 (0 f16, 1 f32, 2 s32),
 // A format bits 7-9 and B format bits 10-12 (f16 = 0; s8 = 1), A major bit 15 and
 // B major bit 16 (0 = K-major, 1 = MN-major), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+// Instruction descriptor of the block-scaled kinds: A format bits 7-9 and B format bits 10-12
+// (E2M1 = 1 for kind::mxf4nvf4), K-major A and B (bits 15, 16 zero), N >> 3 in bits 17-22, the
+// scale format in bit 23 (0 = UE4M3), M >> 4 in bits 24-28; the scale-factor ids (bits 4-5,
+// 29-30) are zero for scale addresses on a column boundary.
+__host__ __device__ constexpr uint32_t make_idesc_fp4(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t d_fmt, uint32_t a_fmt, uint32_t b_fmt,
                                                   uint32_t a_mn_major, uint32_t b_mn_major, uint32_t M,
                                                   uint32_t N) {
