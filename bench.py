@@ -282,6 +282,9 @@ def run_ours(args, w: W.Workload):
 
     fp8 = args.variant == "fp8pv"
     sparse = args.variant == "sparse"
+    fp4 = args.variant == "fp4"
+    if fp4:  # the FP4 variant's quantized operands for its kernel-only timing
+        b4 = sa.empty_fp4(q)
     if sparse:  # the block lists of stage 1 for the sparse variant's kernel-only timing
         nqb, nkb = sa.sparse_blocks(w.N)
         kv_cnt = torch.zeros((w.B, w.H, nqb), dtype=torch.int32, device=dev)
@@ -292,7 +295,9 @@ def run_ours(args, w: W.Workload):
         vm = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
 
     def step():
-        if fp8:
+        if fp4:
+            sa.sage_attn_fwd_fp4(q, k, v, o, w.causal, w.sm_scale, stream)
+        elif fp8:
             sa.sage_attn_fwd_fp8pv(q, k, v, o, w.causal, w.sm_scale, gran, stream)
         elif sparse:
             sa.sage_attn_fwd_sparse(q, k, v, o, w.causal, w.sm_scale, gran, args.tau, args.theta, args.skip_lambda,
@@ -301,7 +306,10 @@ def run_ours(args, w: W.Workload):
             sa.sage_attn_fwd(q, k, v, o, w.causal, w.sm_scale, gran, stream)
 
     def fused():
-        if fp8:
+        if fp4:
+            sa.sage_attn_fwd_fp4_quantized(b4["q4"], b4["sfq"], b4["gq"], b4["k4"], b4["sfk"], b4["gk"], b4["v4t"],
+                                           b4["sfv"], b4["gv"], b4["vm"], o, w.causal, w.sm_scale, stream)
+        elif fp8:
             sa.sage_attn_fwd_fp8pv_quantized(q8, k8, sq, sk, v8, sv, vm, o, w.causal, w.sm_scale, gran, stream)
         elif sparse:
             sa.sage_attn_fwd_sparse_quantized(q8, k8, sq, sk, v, o, w.causal, w.sm_scale, gran, kv_cnt, kv_idx,
@@ -351,6 +359,9 @@ def run_ours(args, w: W.Workload):
     sa.sage_quant_qk(q, k, km, q8, k8, sq, sk, gran, stream)
     if fp8:
         sa.sage_quant_v_fp8(v, v8, sv, vm, stream)
+    if fp4:
+        sa.sage_quant_qk_fp4(q, k, km, b4["q4"], b4["sfq"], b4["gq"], b4["k4"], b4["sfk"], b4["gk"], stream)
+        sa.sage_quant_v_fp4(v, b4["v4t"], b4["sfv"], b4["gv"], b4["vm"], stream)
     if sparse:
         sa.sage_sparse_predict(q, k, w.causal, w.sm_scale, args.tau, args.theta, kv_cnt, kv_idx, stream)
     for _ in range(3):
@@ -386,6 +397,11 @@ def run_ours(args, w: W.Workload):
     }
     if fp8:
         breakdown["quant_v_fp8_ms"] = timed(lambda: sa.sage_quant_v_fp8(v, v8, sv, vm, stream), nb)
+    if fp4:
+        breakdown["quant_qk_fp4_ms"] = timed(lambda: sa.sage_quant_qk_fp4(q, k, km, b4["q4"], b4["sfq"], b4["gq"], b4["k4"],
+                                                                          b4["sfk"], b4["gk"], stream), nb)
+        breakdown["quant_v_fp4_ms"] = timed(lambda: sa.sage_quant_v_fp4(v, b4["v4t"], b4["sfv"], b4["gv"], b4["vm"], stream),
+                                            nb)
     density = None
     if sparse:
         breakdown["sparse_predict_ms"] = timed(
@@ -402,7 +418,7 @@ def run_ours(args, w: W.Workload):
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
-        if fp8 or sparse:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
+        if fp8 or sparse or fp4:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
             q.copy_(qp, non_blocking=True)
             k.copy_(kp, non_blocking=True)
             v.copy_(vp, non_blocking=True)
@@ -435,15 +451,16 @@ def run_ours(args, w: W.Workload):
         p_burst = float(peaks["bf16_tflops"])
         # the kernel-only loop is short (steps x kernel_ms, well under a second), so the burst
         # peak is its denominator; the sustained figure is kept in the note.  The FP8 P.V variant's
-        # P.V runs at the FP8 rate (2 x FP16, as INT8): its roofline is the INT8 one.
-        peak_of = (lambda p: 2.0 * p) if fp8 else mixed_peak_tops
+        # P.V runs at the FP8 rate (2 x FP16, as INT8): its roofline is the INT8 one.  The FP4
+        # variant runs both products at the dense FP4 rate, 4 x FP16 (the datasheet ratio).
+        peak_of = (lambda p: 2.0 * p) if fp8 else ((lambda p: 4.0 * p) if fp4 else mixed_peak_tops)
         peak = peak_of(p_burst)
         # executed work: the sparse variant runs the kept share of the blocks (value stays the
         # dense-equivalent rate, the way block-sparse attention speedups are quoted)
         achieved = ops * (density if sparse else 1.0) / (kernel_ms * 1e-3) / 1e12
         traffic = _traffic_from_profiles(w)
         accuracy = None
-        if args.no_cpu_baseline or world > 1 or fp8 or sparse:  # the CPU baseline belongs to the N=1 headline line only
+        if args.no_cpu_baseline or world > 1 or fp8 or sparse or fp4:  # the CPU baseline belongs to the N=1 headline line only
             cpu_tops, cores, desc = None, None, ("skipped" if world == 1 else "rank 0 at N=1 only")
         else:
             cpu_tops, cores, desc, sample = oracle_sample(w, keep=True)
@@ -452,20 +469,25 @@ def run_ours(args, w: W.Workload):
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3" if fp8 else "int8+f16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e2m1+ue4m3" if fp4 else ("int8+e4m3" if fp8 else "int8+f16"), "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "granularity": "per-block 128Q/64K" if w.per_block else "per-token",
-                       "variant": ("fp8 P.V (E4M3 P~ and V, V smoothed)" if fp8 else
+                       "variant": ("microscaling FP4 (E2M1 Q, K, P~, V with UE4M3 scales per 16; K and V smoothed)"
+                                   if fp4 else "fp8 P.V (E4M3 P~ and V, V smoothed)" if fp8 else
                                    (f"block-sparse (tau {args.tau}, theta {args.theta}, lambda {args.skip_lambda}); "
                                     f"stage-1 kept share {density:.4f}; value = dense-equivalent TOPS" if sparse
                                     else "fp16 P.V")),
                        "inputs": w.describe(), "l2": "inputs larger than L2 (268 MB each at the default); no flush needed",
                        "parallelism": (f"heads sharded over {world} ranks ({w.BH} per rank, "
                                        f"global B*H = {world * w.BH}); no data-path collective")},
-            "roofline": {"bound": "tensor", "kernel": ("sage_attn_v3_kernel" if w.d == 128 else "sage_attn_kernel"), "achieved": round(achieved, 2),
+            "roofline": {"bound": "tensor",
+                         "kernel": ("sage_attn_fp4_kernel" if fp4 else
+                                    "sage_attn_v3_kernel" if w.d == 128 else "sage_attn_kernel"),
+                         "achieved": round(achieved, 2),
                          "peak": round(peak, 2), "unit": "TOPS", "frac": round(achieved / peak, 4),
                          "traffic": traffic,
-                         "peak_note": (f"{'INT8+FP8 roofline 4/(2/P_i8 + 2/P_f8), P_f8 = P_i8' if fp8 else 'mixed INT8+FP16 roofline 4/(2/P_i8 + 2/P_f16)'}"
+                         "peak_note": (f"{'FP4 roofline P_fp4 = 4 x P_f16' if fp4 else 'INT8+FP8 roofline 4/(2/P_i8 + 2/P_f8), P_f8 = P_i8' if fp8 else 'mixed INT8+FP16 roofline 4/(2/P_i8 + 2/P_f16)'}"
                                        f" of {src} peaks: P_f16 = "
                                        f"burst bf16 {p_burst} TFLOP/s (the kernel loop lasts "
                                        f"{kernel_ms * args.steps / 1e3:.2f} s), P_i8 = 2 x P_f16 (dense datasheet "
@@ -479,7 +501,7 @@ def run_ours(args, w: W.Workload):
                     "ms_per_step": round(e2e_ms, 4)},
             "breakdown": {k_: round(v_, 4) for k_, v_ in breakdown.items()},
             "accuracy": accuracy,
-            "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0) + (2 if sparse else 0)) * args.steps,
+            "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0) + (2 if sparse else 0) + (2 if fp4 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
     if world > 1:
@@ -527,9 +549,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=sorted(W.ALL))
-    ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv", "sparse"],
+    ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv", "sparse", "fp4"],
                     help="fp16pv: the SageAttention method (P.V in fp16); fp8pv: its FP8 P.V variant (d=128); "
-                         "sparse: the block-sparse variant (use a sparse_* workload)")
+                         "sparse: the block-sparse variant (use a sparse_* workload); fp4: the microscaling FP4 "
+                         "variant (d=128)")
     ap.add_argument("--tau", type=float, default=0.99, help="sparse: cumulative probability kept by stage 1")
     ap.add_argument("--theta", type=float, default=0.3, help="sparse: self-similarity below which a block is kept")
     ap.add_argument("--skip-lambda", type=float, default=20.0, help="sparse: stage-2 threshold (log2 units)")

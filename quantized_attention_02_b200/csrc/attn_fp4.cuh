@@ -13,9 +13,10 @@
 //   O  += P~ . V4                V4: E2M1 codes of (V - vm) / gv along the keys, 16 keys per scale
 //   O   = O * gv / l + vm        stored as fp16
 //
-// CTA: one 128-row query tile of one head; 6 warps: warp 0 TMA producer (Q once, K and V tiles
+// CTA: one 128-row query tile of one head; 10 warps: warp 0 TMA producer (Q once, K and V tiles
 // and their scale atoms through a 3-stage ring), warp 1 MMA issuer (also allocates tensor
-// memory), warps 2-5 softmax (thread = query row = tensor-memory lane).  Tensor memory:
+// memory), warps 2-9 softmax (two threads per query row = tensor-memory lane, each with half of
+// the row's keys and output columns).  Tensor memory:
 // S [0, 128), O [128, 256), then the scale factors copied from shared memory by tcgen05.cp
 // (4 columns per 512-byte atom): Q 256, K stage s 264 + 8s, P~ 288, V stage s 296 + 8s.
 // Per key tile j the MMA warp issues Q.K^T(j+1) as soon as the softmax holds S(j) in registers,
@@ -35,17 +36,18 @@ struct Fp4Layout {
   static constexpr int OFF_SFP = OFF_SFV + STAGES * SF;
   static constexpr int OFF_GV = OFF_SFP + SF;  // [128] channel scales
   static constexpr int OFF_VM = OFF_GV + 512;  // [128] channel means
-  static constexpr int OFF_BAR = OFF_VM + 512;
+  static constexpr int OFF_XCH = OFF_VM + 512;  // row-maximum exchange [3][2][128], fail flags, row sums [2][128]
+  static constexpr int OFF_BAR = OFF_XCH + 3 * 1024 + 16 + 1024;
   static constexpr int NUM_BARS = 1 + 3 * STAGES + 5;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
   static constexpr uint32_t COL_S = 0, COL_O = 128, COL_SFQ = 256, COL_SFK = 264, COL_SFP = 288, COL_SFV = 296;
   static_assert(COL_SFK + 8 * STAGES <= COL_SFP && COL_SFV + 8 * STAGES <= 512, "tensor-memory columns");
 };
 
 template <bool CAUSAL, bool RAGGED>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     sage_attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const uint8_t* __restrict__ sfq,
                          const uint8_t* __restrict__ sfk, const uint8_t* __restrict__ sfv,
@@ -63,8 +65,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bar_v_full = bar_k_full + S;
   uint64_t* bar_kv_empty = bar_v_full + S;
   uint64_t* bar_s_full = bar_kv_empty + S;  // Q.K^T(j) complete
-  uint64_t* bar_s_free = bar_s_full + 1;    // the softmax holds S(j) in registers (128 arrivals)
-  uint64_t* bar_p_full = bar_s_free + 1;    // P~(j) and its scales in shared memory (128 arrivals)
+  uint64_t* bar_s_free = bar_s_full + 1;    // the softmax holds S(j) in registers (256 arrivals)
+  uint64_t* bar_p_full = bar_s_free + 1;    // P~(j) and its scales in shared memory (256 arrivals)
   uint64_t* bar_o_done = bar_p_full + 1;    // P~.V(j) complete
   uint64_t* bar_drain = bar_o_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -85,8 +87,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar_kv_empty + s, 1);
     }
     mbar_init(bar_s_full, 1);
-    mbar_init(bar_s_free, 128);
-    mbar_init(bar_p_full, 128);
+    mbar_init(bar_s_free, 256);
+    mbar_init(bar_p_full, 256);
     mbar_init(bar_o_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -99,11 +101,12 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp >= 2) {  // the channel scales and means of this head for the epilogue
+  if (warp >= 2 && warp < 6) {  // the channel scales and means of this head for the epilogue
     const int c = threadIdx.x - 64;
     sGV[c] = __ldg(gv + static_cast<size_t>(bh) * L::D + c);
     sVM[c] = vm ? __ldg(vm + static_cast<size_t>(bh) * L::D + c) : 0.f;
   }
+  if (threadIdx.x < 3) reinterpret_cast<int*>(smem + L::OFF_XCH + 3 * 1024)[threadIdx.x] = 0;  // exchange fail flags
   tc_fence_before();
   cta_sync();
   tc_fence_after();
@@ -192,39 +195,65 @@ __global__ void __launch_bounds__(192, 1)
     mma_commit_warp(bar_drain);
     mbar_drain(bar_drain, 0);
   } else {
-    // ============================================================ softmax (thread = query row)
+    // ============================================================ softmax
+    // Two threads per query row (tensor-memory lane): half h of the row's 128 keys and of its
+    // 128 output columns.  They agree on the row maximum through shared memory and a named
+    // barrier of the 256 softmax threads, once per key tile.
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const int q_row = q_tile * L::BM + r;
+    const int c0 = 64 * half;  // this thread's first key of a tile and first output column
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + L::COL_S, tO = tmem + lane_addr + L::COL_O;
+    const uint32_t tS = tmem + lane_addr + L::COL_S + c0, tO = tmem + lane_addr + L::COL_O + c0;
     const uint32_t p_row = smem_u32(smem + L::OFF_P) + r * 64;  // 64-byte swizzle: chunk c at c ^ ((r >> 1) & 3)
-    uint32_t* sfp_word = reinterpret_cast<uint32_t*>(smem + L::OFF_SFP + (r & 31) * 16 + (r >> 5) * 4);
+    // this half's four group scales: atom `half`, row r
+    uint32_t* sfp_word = reinterpret_cast<uint32_t*>(smem + L::OFF_SFP + 512 * half + (r & 31) * 16 + (r >> 5) * 4);
+    float* sMax = reinterpret_cast<float*>(smem + L::OFF_XCH);        // [3 slots][2 halves][128 rows]
+    int* sFail = reinterpret_cast<int*>(smem + L::OFF_XCH + 3 * 1024);  // [3 slots]
     const float c_r = __fmul_rn(__ldg(gq + static_cast<size_t>(bh) * n_qt + q_tile), sm_scale_log2);
     const float* gk_head = gk + static_cast<size_t>(bh) * n_kt;
     float m_use = 0.f;
     float lsum[4] = {0.f, 0.f, 0.f, 0.f};
     bool ok = true;
+    // Exchange of step j: slot j % 3 (last read at step j-3); the flag slot of step j+1 is cleared
+    // here, its last reads (step j-2) being done before every thread reached step j-1's barrier.
+    // A thread whose bounded wait gave up still takes the barrier of the step it leaves in, with
+    // its fail flag set, so that all 256 threads leave at the same barrier.
+    auto exchange = [&](int j, float hm, bool failed) -> float {
+      const int slot = j % 3;
+      if (threadIdx.x == 64) sFail[(j + 1) % 3] = 0;
+      sMax[(slot * 2 + half) * 128 + r] = hm;
+      if (failed) sFail[slot] = 1;
+      asm volatile("barrier.sync 1, 256;" ::: "memory");
+      if (*reinterpret_cast<volatile int*>(sFail + slot)) return NAN;
+      return fmaxf(hm, sMax[(slot * 2 + (half ^ 1)) * 128 + r]);
+    };
     for (int j = 0; j < n_kv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full, j & 1, abort_flag))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full, j & 1, abort_flag))) {
+        exchange(j, 0.f, true);
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      uint32_t x[128];
-      tmem_ld64_sync(tS, *reinterpret_cast<uint32_t(*)[64]>(x));
-      tmem_ld64_sync(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(x + 64));
+      uint32_t x[64];
+      tmem_ld64_sync(tS, x);
       tc_fence_before();
       mbar_arrive(bar_s_free);
       const float cb = __fmul_rn(c_r, __ldg(gk_head + j));
       // masked keys: past the diagonal (causal) and past N (a partial last key tile)
       const bool diag = (CAUSAL && j == q_tile) || (RAGGED && (j + 1) * L::BN > N);
-      const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, N - j * L::BN - 1);
-      float mx = -INFINITY;
+      const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, N - j * L::BN - 1) - c0;
+      float hm = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < 64; ++c) {
         float u = __fmul_rn(__uint_as_float(x[c]), cb);
         if (diag && c > cmax) u = -INFINITY;
         x[c] = __float_as_uint(u);
-        mx = fmaxf(mx, u);
+        hm = fmaxf(hm, u);
       }
+      const float mx = exchange(j, hm, false);
+      if (mx != mx) { ok = false; break; }  // a thread of the softmax gave up waiting
       // integer offset: set by the first tile, moved up when a tile's maximum passes it
       const float m_new = ceilf(mx);
       float alpha = 1.f;
@@ -238,14 +267,18 @@ __global__ void __launch_bounds__(192, 1)
       }
       // P~.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1)
       if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (j - 1) & 1, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (j - 1) & 1, abort_flag))) {
+          if (j + 1 < n_kv) exchange(j + 1, 0.f, true);
+          ok = false;
+          break;
+        }
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) lsum[i] *= alpha;
 #pragma unroll
-        for (int cb2 = 0; cb2 < 128; cb2 += 32) {
+        for (int cb2 = 0; cb2 < 64; cb2 += 32) {
           uint32_t ov[32];
           tmem_ld32_sync(tO + cb2, ov);
 #pragma unroll
@@ -255,40 +288,44 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_st();
       }
       const float m_e = m_use - 10.f;  // p = 2^(u - m + 10); exact: m is an integer
-      uint32_t w[16];
-      uint32_t sfw[2] = {0u, 0u};
+      uint32_t w[8];
+      uint32_t sfw = 0u;
 #pragma unroll
-      for (int gi = 0; gi < 8; ++gi) {
+      for (int gi = 0; gi < 4; ++gi) {
         float z[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           z[k] = fast_exp2(__fsub_rn(__uint_as_float(x[16 * gi + k]), m_e));  // masked: exp2(-inf) = 0
           lsum[k & 3] += z[k];
         }
-        sfw[gi >> 2] |= microscale16(z, w[2 * gi], w[2 * gi + 1]) << (8 * (gi & 3));
+        sfw |= microscale16(z, w[2 * gi], w[2 * gi + 1]) << (8 * gi);
       }
-      // P~ row r: keys 32c .. 32c+31 are the 16-byte chunk c of the row's 64 bytes
+      // P~ row r: keys 32c .. 32c+31 are the 16-byte chunk c of the row's 64 bytes (c = 2 half, 2 half + 1)
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        st_shared_v4(p_row + ((c ^ ((r >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-      sfp_word[0] = sfw[0];
-      sfp_word[128] = sfw[1];  // the second atom, 512 bytes on
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;
+        st_shared_v4(p_row + ((c ^ ((r >> 1) & 3)) << 4), w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+      }
+      *sfp_word = sfw;
       fence_proxy_async_shared();
       mbar_arrive(bar_p_full);
     }
-    // ---- epilogue: O * gv / l + vm -> fp16 -> global
+    // ---- epilogue: O * gv / l + vm -> fp16 -> global (l: the two halves' sums)
+    float* sL = reinterpret_cast<float*>(smem + L::OFF_XCH + 3 * 1024 + 16);  // [2 halves][128 rows]
+    sL[half * 128 + r] = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+    asm volatile("barrier.sync 1, 256;" ::: "memory");
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag))) {
       tc_fence_after();
-      const float inv_l = 1.f / ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3]));
-      __half* orow = o + (static_cast<size_t>(bh) * N + q_row) * L::D;
+      const float inv_l = 1.f / (sL[r] + sL[128 + r]);
+      __half* orow = o + (static_cast<size_t>(bh) * N + q_row) * L::D + c0;
 #pragma unroll
-      for (int cb2 = 0; cb2 < 128; cb2 += 32) {
+      for (int cb2 = 0; cb2 < 64; cb2 += 32) {
         uint32_t ov[32];
         tmem_ld32_sync(tO + cb2, ov);
         uint32_t hv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int c = cb2 + 2 * i;
+          const int c = c0 + cb2 + 2 * i;
           const float a0 = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(ov[2 * i]), inv_l), sGV[c]), sVM[c]);
           const float a1 = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(ov[2 * i + 1]), inv_l), sGV[c + 1]), sVM[c + 1]);
           hv[i] = pack_half2(a0, a1);
