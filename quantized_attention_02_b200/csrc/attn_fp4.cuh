@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(320, 1)
     const float c_r = __fmul_rn(__ldg(gq + static_cast<size_t>(bh) * n_qt + q_tile), sm_scale_log2);
     const float* gk_head = gk + static_cast<size_t>(bh) * n_kt;
     float m_use = 0.f;
-    float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 lsum[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
     bool ok = true;
     // Exchange of step j: slot j % 3 (last read at step j-3); the flag slot of step j+1 is cleared
     // here, its last reads (step j-2) being done before every thread reached step j-1's barrier.
@@ -240,18 +240,22 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld64_sync(tS, x);
       tc_fence_before();
       mbar_arrive(bar_s_free);
-      const float cb = __fmul_rn(c_r, __ldg(gk_head + j));
+      // u = S * cb with cb > 0 (a zero factor only comes with all-zero codes, S = 0, and is kept
+      // off zero so that masked keys, S = -inf, stay -inf): the maximum of the products is the
+      // product of the maximum (rounding is monotonic)
+      const float cb = fmaxf(__fmul_rn(c_r, __ldg(gk_head + j)), 1.17549435e-38f);
       // masked keys: past the diagonal (causal) and past N (a partial last key tile)
       const bool diag = (CAUSAL && j == q_tile) || (RAGGED && (j + 1) * L::BN > N);
       const int cmax = min((CAUSAL && j == q_tile) ? r : L::BN - 1, N - j * L::BN - 1) - c0;
-      float hm = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float u = __fmul_rn(__uint_as_float(x[c]), cb);
-        if (diag && c > cmax) u = -INFINITY;
-        x[c] = __float_as_uint(u);
-        hm = fmaxf(hm, u);
+        for (int c = 0; c < 64; ++c)
+          if (c > cmax) x[c] = 0xFF800000u;
       }
+      float sm = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) sm = max3f(sm, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+      const float hm = sm == -INFINITY ? -INFINITY : __fmul_rn(sm, cb);
       const float mx = exchange(j, hm, false);
       if (mx != mx) { ok = false; break; }  // a thread of the softmax gave up waiting
       // integer offset: set by the first tile, moved up when a tile's maximum passes it
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) lsum[i] *= alpha;
+        for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
 #pragma unroll
         for (int cb2 = 0; cb2 < 64; cb2 += 32) {
           uint32_t ov[32];
@@ -287,18 +291,21 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_wait_st();
       }
-      const float m_e = m_use - 10.f;  // p = 2^(u - m + 10); exact: m is an integer
+      const float m_e = m_use - 10.f;  // p = 2^(S * cb - m + 10); exact: m is an integer
       uint32_t w[8];
       uint32_t sfw = 0u;
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
-        float z[16];
+        float2 z[8];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          z[k] = fast_exp2(__fsub_rn(__uint_as_float(x[16 * gi + k]), m_e));  // masked: exp2(-inf) = 0
-          lsum[k & 3] += z[k];
+        for (int k = 0; k < 8; ++k) {
+          const int c = 16 * gi + 2 * k;
+          const float2 tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
+                                       make_float2(cb, cb), make_float2(-m_e, -m_e));
+          z[k] = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));  // masked: exp2(-inf) = 0
+          lsum[k & 3] = __fadd2_rn(lsum[k & 3], z[k]);
         }
-        sfw |= microscale16(z, w[2 * gi], w[2 * gi + 1]) << (8 * gi);
+        sfw |= microscale16_pos(z, w[2 * gi], w[2 * gi + 1]) << (8 * gi);
       }
       // P~ row r: keys 32c .. 32c+31 are the 16-byte chunk c of the row's 64 bytes (c = 2 half, 2 half + 1)
 #pragma unroll
@@ -312,7 +319,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     // ---- epilogue: O * gv / l + vm -> fp16 -> global (l: the two halves' sums)
     float* sL = reinterpret_cast<float*>(smem + L::OFF_XCH + 3 * 1024 + 16);  // [2 halves][128 rows]
-    sL[half * 128 + r] = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+    const float2 l2 = __fadd2_rn(__fadd2_rn(lsum[0], lsum[1]), __fadd2_rn(lsum[2], lsum[3]));
+    sL[half * 128 + r] = l2.x + l2.y;
     asm volatile("barrier.sync 1, 256;" ::: "memory");
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag))) {
       tc_fence_after();

@@ -57,4 +57,28 @@ __device__ __forceinline__ uint32_t microscale16(const float (&z)[16], uint32_t&
   return s8;
 }
 
+// The same for 16 non-negative values held as 8 pairs (P~): packed maxima and products.
+__device__ __forceinline__ uint32_t microscale16_pos(const float2 (&z)[8], uint32_t& w0, uint32_t& w1) {
+  float gm = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(gm), "f"(z[k].x), "f"(z[k].y));
+    gm = m;
+  }
+  const uint32_t s8 = e4m3_code(__fdiv_rn(gm, 6.0f));
+  const float sd = e4m3_value(s8);
+  const float inv = sd > 0.f ? __frcp_rn(sd) : 0.f;
+  float y[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float2 t = __fmul2_rn(z[k], make_float2(inv, inv));
+    y[2 * k] = t.x;
+    y[2 * k + 1] = t.y;
+  }
+  w0 = e2m1x8(y);
+  w1 = e2m1x8(y + 8);
+  return s8;
+}
+
 }  // namespace sage
