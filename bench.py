@@ -458,7 +458,7 @@ def run_ours(args, w: W.Workload):
         # executed work: the sparse variant runs the kept share of the blocks (value stays the
         # dense-equivalent rate, the way block-sparse attention speedups are quoted)
         achieved = ops * (density if sparse else 1.0) / (kernel_ms * 1e-3) / 1e12
-        traffic = _traffic_from_profiles(w)
+        traffic = _traffic_from_profiles(w, args.variant)
         accuracy = None
         if args.no_cpu_baseline or world > 1 or fp8 or sparse or fp4:  # the CPU baseline belongs to the N=1 headline line only
             cpu_tops, cores, desc = None, None, ("skipped" if world == 1 else "rank 0 at N=1 only")
@@ -510,14 +510,16 @@ def run_ours(args, w: W.Workload):
     return result
 
 
-def _traffic_from_profiles(w):
+def _traffic_from_profiles(w, variant: str = "fp16pv"):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary, if it was
-    taken on this workload with the current kernel; else None."""
+    taken on this workload with the current kernel of this variant; else None.  Entries of the
+    FP4 and FP8 variants' kernels are keyed "fp4:<workload>" / "fp8:<workload>"."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
+    key = f"{variant[:3]}:{w.name}" if variant in ("fp4", "fp8pv") else w.name
     try:
         with open(path) as f:
             t = json.load(f)
-        return t.get(w.name)
+        return t.get(key)
     except (OSError, ValueError):
         return None
 
