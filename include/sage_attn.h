@@ -195,9 +195,11 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
  * the keys; the row sum uses P~ before rounding.  tiles = ceil(N/128). */
 
 /* Q and K (minus km, the channel means of sage_smooth_k, when km is not null) to FP4.
- * q, k: fp16 [B,H,N,128] (in); q4, k4: uint8 [B,H,N,64] (out, codes); sfq, sfk: uint8
- * [B,H,tiles,2,512] (out, scale atoms; rows past N get zero scales); gq, gk: fp32 [B,H,tiles]
- * (out, tile scales).  No workspace. */
+ * q, k: fp16 [B,H,N,128] (in); q4, k4: uint8 [B,H,N,64] (out, codes); sfq: uint8
+ * [B,H,tiles,2,512] (out, scale atoms of Q, the 128 tokens of a tile as rows); sfk: uint8
+ * [B,H,ceil(N/64),2,512] (out, scale atoms of K, the 64 tokens of each half tile as the first 64
+ * rows, the other rows zero); rows past N get zero scales; gq, gk: fp32 [B,H,tiles] (out, tile
+ * scales).  No workspace. */
 int sage_quant_qk_fp4(const void* q, const void* k, const float* km, uint8_t* q4, uint8_t* sfq, float* gq,
                       uint8_t* k4, uint8_t* sfk, float* gk, int B, int H, int N, int d, void* stream);
 

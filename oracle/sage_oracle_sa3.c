@@ -31,7 +31,7 @@
  *                   token 0 of the head.
  *   scores          S_ij = sum_c (q code * scale)(k code * scale) exactly, s = S * gq * gk *
  *                   sm_scale, u = s * log2(e).
- *   P~              per key tile of 128 keys, in the online softmax's order: the row offset m is
+ *   P~              per key tile of 64 keys, in the online softmax's order: the row offset m is
  *                   the integer ceil(max u) over the key tiles seen so far (it only grows; when it
  *                   grows, the running sum and output are scaled by 2^(m_old - m_new), exactly);
  *                   p_j = 2^(u_j - m + 10) (so every p lies in (0, 1024]); the row sum takes the
@@ -56,7 +56,8 @@
 #define ORACLE_ERR_ARG -1
 #define ORACLE_ERR_NOMEM -5
 
-#define FP4_TILE 128    /* tokens per fp32 scale of Q and K; keys per online-softmax tile */
+#define FP4_TILE 128    /* tokens per fp32 scale of Q and K */
+#define FP4_KTILE 64    /* keys per online-softmax tile */
 #define FP4_GROUP 16    /* elements per UE4M3 scale */
 #define FP4_RANGE 2688.0f
 #define P_SHIFT 10.0
@@ -257,7 +258,7 @@ typedef struct {
 static int attn_fp4_row(const fp4_head* h, int64_t i, double* u, double* acc, double* eacc, double* o64,
                         uint16_t* o16, double* env) {
     const int64_t N = h->N, d = h->d, ng = d / FP4_GROUP, ngt = (N + FP4_GROUP - 1) / FP4_GROUP;
-    const int64_t nt = (N + FP4_TILE - 1) / FP4_TILE;
+    const int64_t nt = (N + FP4_KTILE - 1) / FP4_KTILE;
     const int64_t jend = h->causal ? i + 1 : N;
     const double gqi = (double)h->gq[i / FP4_TILE];
     int unsure = 0;
@@ -273,8 +274,8 @@ static int attn_fp4_row(const fp4_head* h, int64_t i, double* u, double* acc, do
     }
     double m = -INFINITY, l = 0.0;
     for (int64_t c = 0; c < d; ++c) acc[c] = eacc[c] = 0.0;
-    for (int64_t t = 0; t < nt && t * FP4_TILE < jend; ++t) {
-        const int64_t j0 = t * FP4_TILE, j1 = (j0 + FP4_TILE < jend) ? j0 + FP4_TILE : jend;
+    for (int64_t t = 0; t < nt && t * FP4_KTILE < jend; ++t) {
+        const int64_t j0 = t * FP4_KTILE, j1 = (j0 + FP4_KTILE < jend) ? j0 + FP4_KTILE : jend;
         double tmax = -INFINITY;
         for (int64_t j = j0; j < j1; ++j)
             if (u[j] > tmax) tmax = u[j];

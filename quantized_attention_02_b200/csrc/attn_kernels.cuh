@@ -39,8 +39,8 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 // channel scales as written by launch_quant_qk_fp4 / launch_quant_v_fp4.
 struct Fp4Args {
   const CUtensorMap* tm_q;  // uint8 [BH][N][64] (3-D), box {64, 128, 1}, 64 B swizzle
-  const CUtensorMap* tm_k;  // the same for K
-  const CUtensorMap* tm_v;  // uint8 [BH][128][ceil(N/128) * 64] (V transposed), box {64, 128, 1}, 64 B swizzle
+  const CUtensorMap* tm_k;  // uint8 [BH][N][64], box {64, 64, 1} (64 keys), 64 B swizzle
+  const CUtensorMap* tm_v;  // uint8 [BH][128][ceil(N/128) * 64] (V transposed), box {32, 128, 1}, 32 B swizzle
   const uint8_t* sfq;       // [BH][ceil(N/128)][2][512] scale atoms of Q, K and V
   const uint8_t* sfk;
   const uint8_t* sfv;

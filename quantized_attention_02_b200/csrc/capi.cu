@@ -87,9 +87,18 @@ bool make_o_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
 }
 
 // FP4 codes: [BH][rows][cols] bytes (Q and K: rows = N tokens, cols = 64; V transposed: rows =
-// 128 channels, cols = tiles * 64), boxes of 64 bytes x 128 rows, 64-byte swizzle.
-bool make_fp4_map3(CUtensorMap* map, const void* base, int rows, int BH, int cols) {
-  return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, BH, cols, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+// 128 channels, cols = tiles * 64), boxes of box_cols bytes x box_rows rows (a box never reaches
+// into the next head), swizzle matching the box width (64 bytes: 64-byte, 32 bytes: 32-byte).
+bool make_fp4_map3(CUtensorMap* map, const void* base, int rows, int BH, int cols, int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows) * cols};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_qk_map(CUtensorMap* map, const int8_t* base, long long rows, int D) {
@@ -561,8 +570,9 @@ int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const flo
     return SAGE_ERR_INVALID;
   const int BH = B * H, tiles = (N + 127) / 128;
   CUtensorMap tq, tk, tv;
-  if (!make_fp4_map3(&tq, q4, N, BH, 64) || !make_fp4_map3(&tk, k4, N, BH, 64) ||
-      !make_fp4_map3(&tv, v4t, 128, BH, tiles * 64))
+  // Q: 128-token boxes; K: 64-key boxes; V^T: 64 keys (32 bytes) of all 128 channels
+  if (!make_fp4_map3(&tq, q4, N, BH, 64, 64, 128) || !make_fp4_map3(&tk, k4, N, BH, 64, 64, 64) ||
+      !make_fp4_map3(&tv, v4t, 128, BH, tiles * 64, 32, 128))
     return SAGE_ERR_CUDA;
   sage::Fp4Args a{};
   a.tm_q = &tq;
@@ -595,7 +605,7 @@ int sage_attn_fwd_fp4(const void* q, const void* k, const void* v, void* o, int 
   const int BH = B * H;
   const size_t tiles = static_cast<size_t>((N + 127) / 128);
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t codes = up(static_cast<size_t>(BH) * N * 64), atoms = up(static_cast<size_t>(BH) * tiles * 1024);
+  const size_t codes = up(static_cast<size_t>(BH) * N * 64), atoms = up(static_cast<size_t>(BH) * tiles * 2 * 1024);
   const size_t tscales = up(static_cast<size_t>(BH) * tiles * 4), chan = up(static_cast<size_t>(BH) * d * 4);
   const size_t off_k4 = codes;
   const size_t off_v4 = off_k4 + codes;

@@ -762,8 +762,11 @@ cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, i
 
 // Q (SMOOTH = false) or K minus its channel mean km: one CTA per (head, 128-token tile), one
 // thread per token.  g[bh, tile] = fl32(a / 2688) with a the tile's largest |x|; z = fl32(x *
-// fl32(2688 / a)); codes [BH][N][64 bytes]; scale atoms sf [BH][tiles][2][512].
-template <bool SMOOTH>
+// fl32(2688 / a)); codes [BH][N][64 bytes].  Scale atoms: Q (ROWS64 = false) [BH][tiles][2][512],
+// the tile's 128 tokens as rows; K (ROWS64 = true) [BH][ceil(N/64)][2][512], each 64-token half
+// in the first 64 rows of its own atoms (the attention kernel's key tiles are 64 tokens), the
+// other rows zero.
+template <bool SMOOTH, bool ROWS64 = false>
 __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict__ x, const float* __restrict__ km,
                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                         float* __restrict__ g, int N) {
@@ -811,9 +814,22 @@ __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict
 #pragma unroll
     for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
   }
-  uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (r & 31) * 16 + (r >> 5) * 4;
-  *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
-  *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+  if constexpr (ROWS64) {
+    const int n64 = (N + 63) / 64, half = tile * 2 + (r >> 6), lr = r & 63;
+    if (half < n64) {
+      uint8_t* atoms = sf + (static_cast<size_t>(bh) * n64 + half) * 1024 + (lr & 31) * 16 + (lr >> 5) * 4;
+      *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
+      *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+      if (lr < 32) {  // rows 64..127 of the atoms (bytes 8..15 of each 16-byte line): zero
+        *reinterpret_cast<uint2*>(atoms + 8) = make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(atoms + 512 + 8) = make_uint2(0u, 0u);
+      }
+    }
+  } else {
+    uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (r & 31) * 16 + (r >> 5) * 4;
+    *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
+    *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+  }
 }
 
 // V codes along the tokens: one CTA per (head, 128-key tile), one thread per channel.
@@ -861,8 +877,8 @@ cudaError_t launch_quant_qk_fp4(const __half* q, const __half* k, const float* k
   quant_fp4_kernel<false><<<blocks, 128, 0, st>>>(q, nullptr, q4, sfq, gq, N);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (km) quant_fp4_kernel<true><<<blocks, 128, 0, st>>>(k, km, k4, sfk, gk, N);
-  else quant_fp4_kernel<false><<<blocks, 128, 0, st>>>(k, nullptr, k4, sfk, gk, N);
+  if (km) quant_fp4_kernel<true, true><<<blocks, 128, 0, st>>>(k, km, k4, sfk, gk, N);
+  else quant_fp4_kernel<false, true><<<blocks, 128, 0, st>>>(k, nullptr, k4, sfk, gk, N);
   return cudaGetLastError();
 }
 

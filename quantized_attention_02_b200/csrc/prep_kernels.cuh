@@ -23,8 +23,8 @@ cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, i
                             float* sk, int BH, int N, int D, bool per_token, cudaStream_t st);
 
 // Microscaling FP4 variant (head dimension 128).  Q and K (minus km when not null) to E2M1
-// codes [BH][N][64 bytes] with scale atoms [BH][ceil(N/128)][2][512] and tile scales
-// [BH][ceil(N/128)].
+// codes [BH][N][64 bytes] and tile scales [BH][ceil(N/128)]; scale atoms of Q [BH][ceil(N/128)]
+// [2][512], of K [BH][ceil(N/64)][2][512] (64 tokens per atom pair).
 cudaError_t launch_quant_qk_fp4(const __half* q, const __half* k, const float* km, uint8_t* q4, uint8_t* sfq,
                                 float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, cudaStream_t st);
 // V to E2M1 along the tokens: transposed codes [BH][128][ceil(N/128) * 64 bytes], scale atoms

@@ -55,6 +55,20 @@ def atoms_to_scales(atoms: np.ndarray) -> np.ndarray:
     return out.reshape(lead + (t * 128, 8))
 
 
+def atoms64_to_scales(atoms: np.ndarray) -> np.ndarray:
+    """K's [..., halves, 2, 512] scale atoms (64 tokens as each atom pair's first rows) ->
+    [..., halves * 64, 8]; also checks that the atoms' other rows are zero."""
+    lead = atoms.shape[:-3]
+    t = atoms.shape[-3]
+    r = np.arange(64)
+    out = np.empty(lead + (t, 64, 8), np.uint8)
+    for g in range(8):
+        out[..., g] = atoms[..., g // 4, :][..., (r % 32) * 16 + (r // 32) * 4 + g % 4]
+    lines = atoms.reshape(lead + (t, 2, 32, 16))
+    assert not lines[..., 8:].any(), "rows 64..127 of K's scale atoms must be zero"
+    return out.reshape(lead + (t * 64, 8))
+
+
 def gpu_quant(sa, q, k, v, smooth_v=True):
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     b = sa.empty_fp4(qd, smooth_v)
@@ -73,7 +87,7 @@ def check_codes(b, ref, N):
         diff = codes != want
         assert not diff.any(), f"{name}: {diff.sum()} codes differ (first at {np.argwhere(diff)[0]})"
         np.testing.assert_array_equal(cpu[gname], ref[gname], err_msg=gname)
-        sc = atoms_to_scales(cpu[sname])
+        sc = atoms_to_scales(cpu[sname]) if name == "q4" else atoms64_to_scales(cpu[sname])
         np.testing.assert_array_equal(sc[..., :N, :], ref["qs" if name == "q4" else "ks"], err_msg=sname)
         assert not sc[..., N:, :].any(), f"{sname}: rows past N must carry zero scales"
     np.testing.assert_array_equal(cpu["gv"], ref["gv"], err_msg="gv")
