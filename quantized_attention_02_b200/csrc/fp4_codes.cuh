@@ -57,7 +57,10 @@ __device__ __forceinline__ uint32_t microscale16(const float (&z)[16], uint32_t&
   return s8;
 }
 
-// The same for 16 non-negative values held as 8 pairs (P~): packed maxima and products.
+// The same for 16 non-negative values held as 8 pairs (P~, whose values the kernel computes in
+// fp32 with exp2 approximations anyway): packed maxima and products, and max/6 and 1/scale
+// within an ulp (a product with fl32(1/6), the hardware reciprocal) instead of correctly
+// rounded: a decision that these change lies within a relative 1e-6 of a rounding midpoint.
 __device__ __forceinline__ uint32_t microscale16_pos(const float2 (&z)[8], uint32_t& w0, uint32_t& w1) {
   float gm = 0.f;
 #pragma unroll
@@ -66,9 +69,10 @@ __device__ __forceinline__ uint32_t microscale16_pos(const float2 (&z)[8], uint3
     asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(gm), "f"(z[k].x), "f"(z[k].y));
     gm = m;
   }
-  const uint32_t s8 = e4m3_code(__fdiv_rn(gm, 6.0f));
+  const uint32_t s8 = e4m3_code(__fmul_rn(gm, 0.16666667163372040f));
   const float sd = e4m3_value(s8);
-  const float inv = sd > 0.f ? __frcp_rn(sd) : 0.f;
+  float inv = 0.f;
+  if (sd > 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(sd));
   float y[16];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
