@@ -280,7 +280,9 @@ __global__ void __launch_bounds__(192, 2)
           const int c = 16 * gi + 2 * k;
           const float2 tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
                                        make_float2(cb, cb), make_float2(-m_e, -m_e));
-          z[k] = make_float2(fast_exp2(tt.x), fast_exp2(tt.y));  // masked: exp2(-inf) = 0
+          // one pair in four on the FMA pipe (exp2_poly2, relative error <= 7.5e-5), the rest on
+          // the MUFU unit; masked keys: exp2(-inf) = 0 (the polynomial gives 2^-126)
+          z[k] = (k & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
           lsum[k & 3] = __fadd2_rn(lsum[k & 3], z[k]);
         }
         sfw |= microscale16_pos(z, w[2 * gi], w[2 * gi + 1]) << (8 * gi);
