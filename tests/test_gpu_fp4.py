@@ -157,6 +157,29 @@ def test_fp4_codes_and_output_match_the_oracle(sa, w):
     assert torch.equal(o2, o)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 129, 200])
+def test_fp4_edge_sizes(sa, N, causal):
+    # a single token, partial 64-key tiles, a partial 128-token scale tile, one key tile plus one key
+    w = W.Workload(f"fp4_edge_{N}", 1, 2, N, 128, causal, True, n_out=2, out_mag=10.0)
+    q, k, v = W.make_qkv(w)
+    b = gpu_quant(sa, q, k, v)
+    ref = oracle.sage_attn_fp4(q, k, v, causal, w.sm_scale)
+    check_codes(b, ref, N)
+    o = torch.empty_like(q, device="cuda")
+    sa.sage_attn_fwd_fp4_quantized(b["q4"], b["sfq"], b["gq"], b["k4"], b["sfk"], b["gk"], b["v4t"], b["sfv"],
+                                   b["gv"], b["vm"], o, causal, w.sm_scale)
+    torch.cuda.synchronize()
+    assert sa.sage_last_device_error() == 0
+    o_gpu = o.float().cpu().numpy().astype(np.float64)
+    err = np.abs(o_gpu - ref["o64"])
+    bar = BASE_FRAC * vhat_max(ref) + ref["env"]
+    sure = ref["unsure"] == 0
+    assert np.all((err <= bar) | ~sure[..., None]), f"N={N}: max excess {(err - bar).max():.3e}"
+    if causal:  # row 0 sees only key 0: O[0] = v^0 (one P~ code times its own scale, over p itself)
+        assert np.isfinite(o_gpu).all()
+
+
 def test_fp4_without_v_smoothing(sa):
     w = W.Workload("fp4_nosmooth", 1, 2, 512, 128, False, True, n_out=2, out_mag=10.0)
     q, k, v = W.make_qkv(w)
