@@ -94,6 +94,38 @@ def test_null_pointers_and_bad_scalars(sa):
     assert L.sage_debug_wait_timeout(None, s) == -1
 
 
+def test_variant_entries_validate_before_any_cuda_call(sa):
+    # FP8 P.V, block-sparse and FP4 entry points: null pointers, unsupported head dimensions and
+    # sizes, bad scalars and misaligned buffers are rejected before anything is enqueued
+    L = sa.get_lib()
+    s = ctypes.c_void_p(0)
+    mis = ctypes.c_void_p(0x1008)
+    inv, uns = sa.SAGE_ERR_INVALID, sa.SAGE_ERR_UNSUPPORTED
+    # microscaling FP4: head dimension 128 only
+    assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 0, 0.1, s) == uns
+    assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 0, 0.1, s) == inv
+    assert L.sage_attn_fwd_fp4(mis, FAKE, FAKE, FAKE, 1, 1, 256, 128, 0, 0.1, s) == inv
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 128, 0, bad, s) == inv
+        assert L.sage_attn_fwd_fp4_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                             1, 1, 256, 128, 0, bad, s) == inv
+    assert L.sage_quant_qk_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 256, 128, s) == inv
+    assert L.sage_quant_qk_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, s) == uns
+    assert L.sage_quant_qk_fp4(FAKE, FAKE, None, mis, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 128, s) == inv
+    assert L.sage_quant_v_fp4(FAKE, None, FAKE, FAKE, None, 1, 1, 256, 128, s) == inv
+    assert L.sage_quant_v_fp4(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 256, 64, s) == uns
+    assert L.sage_attn_fwd_fp4_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, mis, FAKE, None, FAKE,
+                                         1, 1, 256, 128, 0, 0.1, s) == inv
+    # FP8 P.V: head dimension 128 only
+    assert L.sage_attn_fwd_fp8pv(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 0, 0.1, 1, s) == uns
+    # block-sparse: at most 512 key blocks; tau in (0, 1]; lambda > 0
+    assert L.sage_attn_fwd_sparse(FAKE, FAKE, FAKE, FAKE, 1, 1, 65536 + 256, 64, 0, 0.1, 1, 0.9, 0.3, 20.0, s) == uns
+    for tau in (0.0, -0.5, 1.5, float("nan")):
+        assert L.sage_attn_fwd_sparse(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 0, 0.1, 1, tau, 0.3, 20.0, s) == inv
+    for lam in (0.0, -1.0, float("nan")):
+        assert L.sage_attn_fwd_sparse(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 128, 0, 0.1, 1, 0.9, 0.3, lam, s) == inv
+
+
 def test_host_pipeline_validation(sa):
     # every failure below is found before any CUDA call (no GPU is needed)
     L = sa.get_lib()
