@@ -554,7 +554,7 @@ def main(argv=None):
     ap.add_argument("--variant", default="fp16pv", choices=["fp16pv", "fp8pv", "sparse", "fp4"],
                     help="fp16pv: the SageAttention method (P.V in fp16); fp8pv: its FP8 P.V variant (d=128); "
                          "sparse: the block-sparse variant (use a sparse_* workload); fp4: the microscaling FP4 "
-                         "variant (d=128)")
+                         "variant (d=64 or 128)")
     ap.add_argument("--tau", type=float, default=0.99, help="sparse: cumulative probability kept by stage 1")
     ap.add_argument("--theta", type=float, default=0.3, help="sparse: self-similarity below which a block is kept")
     ap.add_argument("--skip-lambda", type=float, default=20.0, help="sparse: stage-2 threshold (log2 units)")

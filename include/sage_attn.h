@@ -182,8 +182,8 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
 /* ---------------------------------------------------------------------------------------
  * Microscaling FP4 variant, following the SageAttention3 abstract (author pages of Jia Wei and
  * Haofeng Huang; arXiv 2505.11594): both products of the attention run on Blackwell's FP4 tensor
- * cores (tcgen05 kind::mxf4nvf4, block16) with microscaling.  Head dimension 128 only
- * (SAGE_ERR_UNSUPPORTED otherwise).  Formats: E2M1 codes (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their
+ * cores (tcgen05 kind::mxf4nvf4, block16) with microscaling.  Head dimension d = 64 or 128.
+ * Formats: E2M1 codes (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their
  * negatives), two per byte with the even element in the low nibble; one UE4M3 scale per 16
  * elements along the contraction dimension, e4m3(fl32(max|z| / 6)), codes
  * e2m1(fl32(z * fl32(1 / scale))); scales stored as the tensor cores' scale atoms: for every 128
@@ -192,28 +192,30 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
  * and of smoothed K, g = fl32(a / 2688) with a = the tile's largest |x|, z = fl32(x * fl32(2688 /
  * a)); per channel of smoothed V the same over all tokens.  P~ = 2^(u - m + 10) in the online
  * softmax's integer frame m (the ceil of the running row maximum, log2 units), microscaled along
- * the keys; the row sum uses P~ before rounding.  tiles = ceil(N/128). */
+ * the keys; the row sum uses P~ before rounding.  tiles = ceil(N/128); A = d / 64, the scale
+ * atoms per row group of Q and K (one per 64 channels). */
 
 /* Q and K (minus km, the channel means of sage_smooth_k, when km is not null) to FP4.
- * q, k: fp16 [B,H,N,128] (in); q4, k4: uint8 [B,H,N,64] (out, codes); sfq: uint8
- * [B,H,tiles,2,512] (out, scale atoms of Q, the 128 tokens of a tile as rows); sfk: uint8
- * [B,H,ceil(N/64),2,512] (out, scale atoms of K, the 64 tokens of each half tile as the first 64
+ * q, k: fp16 [B,H,N,d] (in); q4, k4: uint8 [B,H,N,d/2] (out, codes); sfq: uint8
+ * [B,H,tiles,A,512] (out, scale atoms of Q, the 128 tokens of a tile as rows); sfk: uint8
+ * [B,H,ceil(N/64),A,512] (out, scale atoms of K, the 64 tokens of each half tile as the first 64
  * rows, the other rows zero); rows past N get zero scales; gq, gk: fp32 [B,H,tiles] (out, tile
  * scales).  No workspace. */
 int sage_quant_qk_fp4(const void* q, const void* k, const float* km, uint8_t* q4, uint8_t* sfq, float* gq,
                       uint8_t* k4, uint8_t* sfk, float* gk, int B, int H, int N, int d, void* stream);
 
 /* V to FP4 along the tokens (the P.V contraction), smoothed by its exact channel mean when vm is
- * not null.  v: fp16 [B,H,N,128] (in); v4t: uint8 [B,H,128,tiles*64] (out, codes transposed:
+ * not null.  v: fp16 [B,H,N,d] (in); v4t: uint8 [B,H,d,tiles*64] (out, codes transposed:
  * row c holds channel c's codes of keys 0 .. tiles*128-1, keys past N zero); sfv: uint8
- * [B,H,tiles,2,512] (out, scale atoms with the channels as rows); gv: fp32 [B,H,128] (out, channel
- * scales); vm: fp32 [B,H,128] (out, channel means) or null.  Allocates a small stream-ordered
+ * [B,H,tiles,2,512] (out, scale atoms of keys 0-63 and 64-127 of a tile with the channels as
+ * rows; d = 64: rows 64-127 zero); gv: fp32 [B,H,d] (out, channel scales); vm: fp32 [B,H,d] (out,
+ * channel means) or null.  Allocates a small stream-ordered
  * workspace (the inverse channel scales). */
 int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, int B, int H, int N, int d,
                      void* stream);
 
 /* The fused FP4 kernel on quantized inputs (layouts above; vm may be null).  o: fp16
- * [B,H,N,128] (out).  All pointers 16-byte aligned.  No workspace. */
+ * [B,H,N,d] (out).  All pointers 16-byte aligned.  No workspace. */
 int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const float* gq, const uint8_t* k4,
                                 const uint8_t* sfk, const float* gk, const uint8_t* v4t, const uint8_t* sfv,
                                 const float* gv, const float* vm, void* o, int B, int H, int N, int d, int causal,

@@ -196,17 +196,18 @@ def fp4_tiles(N: int) -> int:
 
 
 def empty_fp4(q, smooth_v: bool = True) -> dict:
-    """Device buffers of the FP4 variant's quantized operands for q-shaped [B,H,N,128] inputs:
-    q4/k4 uint8 [B,H,N,64], sfq/sfv uint8 [B,H,tiles,2,512], sfk uint8 [B,H,ceil(N/64),2,512],
-    gq/gk fp32 [B,H,tiles],
-    v4t uint8 [B,H,128,tiles*64], gv/vm fp32 [B,H,128] (vm None when not smoothed), km fp32
-    [B,H,128]."""
+    """Device buffers of the FP4 variant's quantized operands for q-shaped [B,H,N,d] inputs
+    (d = 64 or 128, A = d/64 scale atoms per row group): q4/k4 uint8 [B,H,N,d/2], sfq uint8
+    [B,H,tiles,A,512], sfk uint8 [B,H,ceil(N/64),A,512], sfv uint8 [B,H,tiles,2,512], gq/gk fp32
+    [B,H,tiles], v4t uint8 [B,H,d,tiles*64], gv/vm fp32 [B,H,d] (vm None when not smoothed), km
+    fp32 [B,H,d]."""
     B, H, N, d = _shape(q)
     t = fp4_tiles(N)
+    a = d // 64
     u8 = dict(dtype=torch.uint8, device=q.device)
     f32 = dict(dtype=torch.float32, device=q.device)
     return dict(q4=torch.empty((B, H, N, d // 2), **u8), k4=torch.empty((B, H, N, d // 2), **u8),
-                sfq=torch.empty((B, H, t, 2, 512), **u8), sfk=torch.empty((B, H, (N + 63) // 64, 2, 512), **u8),
+                sfq=torch.empty((B, H, t, a, 512), **u8), sfk=torch.empty((B, H, (N + 63) // 64, a, 512), **u8),
                 sfv=torch.empty((B, H, t, 2, 512), **u8), gq=torch.empty((B, H, t), **f32),
                 gk=torch.empty((B, H, t), **f32), v4t=torch.empty((B, H, d, t * 64), **u8),
                 gv=torch.empty((B, H, d), **f32), vm=torch.empty((B, H, d), **f32) if smooth_v else None,

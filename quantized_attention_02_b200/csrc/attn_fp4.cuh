@@ -13,52 +13,58 @@
 //   O  += P~ . V4                V4: E2M1 codes of (V - vm) / gv along the keys, 16 keys per scale
 //   O   = O * gv / l + vm        stored as fp16
 //
-// CTA: one 128-row query tile of one head, 6 warps: warp 0 TMA producer (Q once, then 64-key
+// Head dimension D = 64 or 128.  CTA: one 128-row query tile of one head, 6 warps: warp 0 TMA producer (Q once, then 64-key
 // tiles of K and V and their scale atoms through a 3-stage ring), warp 1 MMA issuer (also
 // allocates tensor memory), warps 2-5 softmax (thread = query row = tensor-memory lane, 64 keys
 // per tile).  The CTA holds 256 tensor-memory columns, so two CTAs share an SM and each one's
 // hand-offs overlap the other's exp2 work:
-//   S [0, 64), O [64, 192), then the scale factors copied from shared memory by tcgen05.cp
-//   (4 columns per 512-byte atom): Q 192 (two atoms), K stage s 200 + 8s (two atoms, the 64 keys
-//   as their first 64 rows), P~ 224 (one atom), V stage s 232 + 4s (one atom).
+//   S [0, 64), O [64, 64 + D), then the scale factors copied from shared memory by tcgen05.cp
+//   (4 columns per 512-byte atom, one atom per 64 channels of Q and K): Q at 64 + D, K stage s
+//   8 columns further on + 8s (the 64 keys as the atoms' first 64 rows), P~ (one atom), V stage s
+//   (one atom, channels as rows; D = 64 reads its first 64 rows).
 // Per key tile j the MMA warp issues Q.K^T(j+1) as soon as the softmax holds S(j) in registers,
 // then P~.V(j) once P~(j) and its scales are in shared memory.
 
+template <int D_>
 struct Fp4Layout {
-  static constexpr int BM = 128, BN = 64, D = 128, STAGES = 3;
-  static constexpr int Q_TILE = 128 * 64;  // 128 rows of 128 E2M1 codes (64 bytes), 64-byte swizzle
-  static constexpr int K_TILE = 64 * 64;   // 64 keys x 128 channels, 64-byte swizzle
-  static constexpr int V_TILE = 128 * 32;  // 128 channels x 64 keys (32 bytes), 32-byte swizzle
-  static constexpr int P_TILE = 128 * 32;  // 128 queries x 64 keys, 32-byte swizzle
+  static constexpr int BM = 128, BN = 64, D = D_, STAGES = 3;
+  static constexpr int ROW = D / 2;              // bytes of E2M1 codes per Q / K row
+  static constexpr int NA = D / 64;              // scale atoms per Q / K row group (64 channels each)
+  static constexpr int Q_TILE = 128 * ROW;       // 128 rows, 64-byte (D = 128) / 32-byte (D = 64) swizzle
+  static constexpr int K_TILE = 64 * ROW;        // 64 keys, same swizzle
+  static constexpr int V_TILE = D * 32;          // D channels x 64 keys (32 bytes), 32-byte swizzle
+  static constexpr int P_TILE = 128 * 32;        // 128 queries x 64 keys, 32-byte swizzle
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_TILE;
   static constexpr int OFF_V = OFF_K + STAGES * K_TILE;
   static constexpr int OFF_P = OFF_V + STAGES * V_TILE;
-  static constexpr int OFF_SFQ = OFF_P + P_TILE;           // 2 atoms
-  static constexpr int OFF_SFK = OFF_SFQ + 1024;           // 2 atoms per stage
-  static constexpr int OFF_SFV = OFF_SFK + STAGES * 1024;  // 1 atom per stage
-  static constexpr int OFF_SFP = OFF_SFV + STAGES * 512;   // 1 atom
-  static constexpr int OFF_GV = OFF_SFP + 512;  // [128] channel scales
-  static constexpr int OFF_VM = OFF_GV + 512;   // [128] channel means
+  static constexpr int OFF_SFQ = (OFF_P + P_TILE + 1023) & ~1023;  // NA atoms
+  static constexpr int OFF_SFK = OFF_SFQ + 1024;                   // NA atoms per stage (1 KB slots)
+  static constexpr int OFF_SFV = OFF_SFK + STAGES * 1024;          // 1 atom per stage
+  static constexpr int OFF_SFP = OFF_SFV + STAGES * 512;           // 1 atom
+  static constexpr int OFF_GV = OFF_SFP + 512;  // [D] channel scales
+  static constexpr int OFF_VM = OFF_GV + 512;   // [D] channel means
   static constexpr int OFF_BAR = OFF_VM + 512;
   static constexpr int NUM_BARS = 1 + 3 * STAGES + 5;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t COL_S = 0, COL_O = 64, COL_SFQ = 192, COL_SFK = 200, COL_SFP = 224, COL_SFV = 232;
-  static_assert(COL_SFK + 8 * STAGES <= COL_SFP && COL_SFP + 8 <= COL_SFV && COL_SFV + 4 * STAGES <= TMEM_COLS,
-                "tensor-memory columns");
+  static constexpr uint32_t COL_S = 0, COL_O = 64, COL_SFQ = 64 + D, COL_SFK = COL_SFQ + 8,
+                            COL_SFP = COL_SFK + 8 * STAGES, COL_SFV = COL_SFP + 8;
+  static_assert(COL_SFV + 4 * STAGES <= TMEM_COLS, "tensor-memory columns");
+  static constexpr SwizzleMode QK_SWZ = D == 128 ? kSwizzle64B : kSwizzle32B;
+  static constexpr uint32_t QK_SBO = 8 * ROW;    // 8 rows of codes
 };
 
-template <bool CAUSAL, bool RAGGED>
+template <int D, bool CAUSAL, bool RAGGED>
 __global__ void __launch_bounds__(192, 2)
     sage_attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const uint8_t* __restrict__ sfq,
                          const uint8_t* __restrict__ sfk, const uint8_t* __restrict__ sfv,
                          const float* __restrict__ gq, const float* __restrict__ gk, const float* __restrict__ gv,
                          const float* __restrict__ vm, __half* __restrict__ o, int N, float sm_scale_log2) {
-  using L = Fp4Layout;
+  using L = Fp4Layout<D>;
   constexpr int S = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(192, 2)
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp >= 2) {  // the channel scales and means of this head for the epilogue
+  if (warp >= 2 && threadIdx.x - 64 < D) {  // the channel scales and means of this head for the epilogue
     const int c = threadIdx.x - 64;
     sGV[c] = __ldg(gv + static_cast<size_t>(bh) * L::D + c);
     sVM[c] = vm ? __ldg(vm + static_cast<size_t>(bh) * L::D + c) : 0.f;
@@ -121,19 +127,20 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       int issued[S];
       for (int s = 0; s < S; ++s) issued[s] = 0;
-      mbar_arrive_expect_tx(bar_q, L::Q_TILE + 1024);
+      mbar_arrive_expect_tx(bar_q, L::Q_TILE + L::NA * 512);
       tma_load_3d(smem + L::OFF_Q, &tm_q, bar_q, 0, q_tile * L::BM, bh);
-      bulk_load(smem + L::OFF_SFQ, sfq + (static_cast<size_t>(bh) * n_qt + q_tile) * 1024, 1024, bar_q);
+      bulk_load(smem + L::OFF_SFQ, sfq + (static_cast<size_t>(bh) * n_qt + q_tile) * (L::NA * 512), L::NA * 512,
+                bar_q);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % S, it = j / S;
         if (j >= S && !mbar_wait(bar_kv_empty + s, (it - 1) & 1, abort_flag)) break;
         // scale atoms: K's two (channels 0-63, 64-127) of key tile j; V's one of keys 64 (j % 2) ..
         // + 63 of the 128-token tile j / 2
         const size_t tile128 = static_cast<size_t>(bh) * n_qt + (j >> 1);
-        mbar_arrive_expect_tx(bar_k_full + s, L::K_TILE + 1024);
+        mbar_arrive_expect_tx(bar_k_full + s, L::K_TILE + L::NA * 512);
         tma_load_3d(smem + L::OFF_K + s * L::K_TILE, &tm_k, bar_k_full + s, 0, j * L::BN, bh);
-        bulk_load(smem + L::OFF_SFK + s * 1024, sfk + (static_cast<size_t>(bh) * n_kt + j) * 1024, 1024,
-                  bar_k_full + s);
+        bulk_load(smem + L::OFF_SFK + s * 1024, sfk + (static_cast<size_t>(bh) * n_kt + j) * (L::NA * 512),
+                  L::NA * 512, bar_k_full + s);
         mbar_arrive_expect_tx(bar_v_full + s, L::V_TILE + 512);
         tma_load_3d(smem + L::OFF_V + s * L::V_TILE, &tm_v, bar_v_full + s, j * 32, 0, bh);  // keys j*64.. (bytes)
         bulk_load(smem + L::OFF_SFV + s * 512, sfv + tile128 * 1024 + (j & 1) * 512, 512, bar_v_full + s);
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(192, 2)
   } else if (warp == 1) {
     // ============================================================ MMA issuer (whole warp; elect.sync)
     constexpr uint32_t IDESC_QK = make_idesc_fp4(128, 64);
-    constexpr uint32_t IDESC_PV = make_idesc_fp4(128, 128);
+    constexpr uint32_t IDESC_PV = make_idesc_fp4(128, D);
     const uint32_t sbase = smem_u32(smem);
     auto wait = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag)); };
     // n_atoms 512-byte scale atoms at saddr -> columns col, col + 4, ...
@@ -160,14 +167,14 @@ __global__ void __launch_bounds__(192, 2)
       for (int a = 0; a < n_atoms; ++a)
         tmem_cp_32x128b_warp(tmem + col + 4 * a, make_smem_desc(saddr + 512 * a, 16, 128, kSwizzleNone));
     };
-    // S = Q . K^T over the 128 channels (two K steps of 64 elements = 32 bytes of each 64-byte row)
+    // S = Q . K^T over the D channels (K steps of 64 elements = 32 bytes of each row)
     auto qk = [&](int j) {
       const int s = j % S;
-      copy_scales(L::COL_SFK + 8 * s, sbase + L::OFF_SFK + s * 1024, 2);
+      copy_scales(L::COL_SFK + 8 * s, sbase + L::OFF_SFK + s * 1024, L::NA);
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const uint64_t a = make_smem_desc(sbase + L::OFF_Q + kk * 32, 16, 512, kSwizzle64B);
-        const uint64_t b = make_smem_desc(sbase + L::OFF_K + s * L::K_TILE + kk * 32, 16, 512, kSwizzle64B);
+      for (int kk = 0; kk < L::NA; ++kk) {
+        const uint64_t a = make_smem_desc(sbase + L::OFF_Q + kk * 32, 16, L::QK_SBO, L::QK_SWZ);
+        const uint64_t b = make_smem_desc(sbase + L::OFF_K + s * L::K_TILE + kk * 32, 16, L::QK_SBO, L::QK_SWZ);
         mma_fp4_ss_warp(tmem + L::COL_S, a, b, IDESC_QK, tmem + L::COL_SFQ + 4 * kk,
                         tmem + L::COL_SFK + 8 * s + 4 * kk, kk > 0 ? 1u : 0u);
       }
@@ -176,7 +183,7 @@ __global__ void __launch_bounds__(192, 2)
     bool ok = wait(bar_q, 0) && wait(bar_k_full, 0);
     if (ok) {
       tc_fence_after();
-      copy_scales(L::COL_SFQ, sbase + L::OFF_SFQ, 2);
+      copy_scales(L::COL_SFQ, sbase + L::OFF_SFQ, L::NA);
       qk(0);
     }
     for (int j = 0; ok && j < n_kv; ++j) {
@@ -260,7 +267,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
 #pragma unroll
-        for (int cb2 = 0; cb2 < 128; cb2 += 32) {
+        for (int cb2 = 0; cb2 < D; cb2 += 32) {
           uint32_t ov[32];
           tmem_ld32_sync(tO + cb2, ov);
 #pragma unroll
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(192, 2)
       const float inv_l = 1.f / (l2.x + l2.y);
       __half* orow = o + (static_cast<size_t>(bh) * N + q_row) * L::D;
 #pragma unroll
-      for (int cb2 = 0; cb2 < 128; cb2 += 32) {
+      for (int cb2 = 0; cb2 < D; cb2 += 32) {
         uint32_t ov[32];
         tmem_ld32_sync(tO + cb2, ov);
         uint32_t hv[16];

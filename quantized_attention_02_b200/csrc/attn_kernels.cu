@@ -866,25 +866,31 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
   return ragged ? launch_attn_d<64, true>(a, st) : launch_attn_d<64, false>(a, st);
 }
 
-template <bool CAUSAL, bool RAGGED>
+template <int D, bool CAUSAL, bool RAGGED>
 static cudaError_t launch_attn_fp4_t(const Fp4Args& a, cudaStream_t st) {
-  auto kern = sage_attn_fp4_kernel<CAUSAL, RAGGED>;
+  using L = Fp4Layout<D>;
+  auto kern = sage_attn_fp4_kernel<D, CAUSAL, RAGGED>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4Layout::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const unsigned grid = static_cast<unsigned>((a.N + 127) / 128) * static_cast<unsigned>(a.BH);
-  kern<<<grid, Fp4Layout::THREADS, Fp4Layout::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sfq, a.sfk, a.sfv, a.gq, a.gk,
-                                                          a.gv, a.vm, a.o, a.N, a.sm_scale_log2);
+  kern<<<grid, L::THREADS, L::SMEM, st>>>(*a.tm_q, *a.tm_k, *a.tm_v, a.sfq, a.sfk, a.sfv, a.gq, a.gk, a.gv, a.vm, a.o,
+                                          a.N, a.sm_scale_log2);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_fp4(const Fp4Args& a, cudaStream_t st) {
+template <int D>
+static cudaError_t launch_attn_fp4_d(const Fp4Args& a, cudaStream_t st) {
   const bool ragged = a.N % 128 != 0;
-  if (a.causal) return ragged ? launch_attn_fp4_t<true, true>(a, st) : launch_attn_fp4_t<true, false>(a, st);
-  return ragged ? launch_attn_fp4_t<false, true>(a, st) : launch_attn_fp4_t<false, false>(a, st);
+  if (a.causal) return ragged ? launch_attn_fp4_t<D, true, true>(a, st) : launch_attn_fp4_t<D, true, false>(a, st);
+  return ragged ? launch_attn_fp4_t<D, false, true>(a, st) : launch_attn_fp4_t<D, false, false>(a, st);
+}
+
+cudaError_t launch_attn_fp4(const Fp4Args& a, cudaStream_t st) {
+  return a.D == 128 ? launch_attn_fp4_d<128>(a, st) : launch_attn_fp4_d<64>(a, st);
 }
 
 template <int D>

@@ -35,21 +35,21 @@ struct AttnArgs {
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 
-// Microscaling FP4 variant (head dimension 128): E2M1 codes, UE4M3 scale atoms and fp32 tile /
-// channel scales as written by launch_quant_qk_fp4 / launch_quant_v_fp4.
+// Microscaling FP4 variant (head dimension D = 64 or 128): E2M1 codes, UE4M3 scale atoms and fp32
+// tile / channel scales as written by launch_quant_qk_fp4 / launch_quant_v_fp4.
 struct Fp4Args {
-  const CUtensorMap* tm_q;  // uint8 [BH][N][64] (3-D), box {64, 128, 1}, 64 B swizzle
-  const CUtensorMap* tm_k;  // uint8 [BH][N][64], box {64, 64, 1} (64 keys), 64 B swizzle
-  const CUtensorMap* tm_v;  // uint8 [BH][128][ceil(N/128) * 64] (V transposed), box {32, 128, 1}, 32 B swizzle
-  const uint8_t* sfq;       // [BH][ceil(N/128)][2][512] scale atoms of Q, K and V
-  const uint8_t* sfk;
-  const uint8_t* sfv;
+  const CUtensorMap* tm_q;  // uint8 [BH][N][D/2] (3-D), box {D/2, 128, 1}, 64 B (D=128) / 32 B (D=64) swizzle
+  const CUtensorMap* tm_k;  // uint8 [BH][N][D/2], box {D/2, 64, 1} (64 keys), same swizzle
+  const CUtensorMap* tm_v;  // uint8 [BH][D][ceil(N/128) * 64] (V transposed), box {32, D, 1}, 32 B swizzle
+  const uint8_t* sfq;       // [BH][ceil(N/128)][D/64][512] scale atoms of Q
+  const uint8_t* sfk;       // [BH][ceil(N/64)][D/64][512] of K (64 tokens per atom)
+  const uint8_t* sfv;       // [BH][ceil(N/128)][2][512] of V (channels as rows)
   const float* gq;          // [BH][ceil(N/128)] tile scales of Q and K
   const float* gk;
-  const float* gv;          // [BH][128] channel scales of V
-  const float* vm;          // [BH][128] channel means of V, or null
-  __half* o;                // fp16 [BH][N][128]
-  int BH, N;
+  const float* gv;          // [BH][D] channel scales of V
+  const float* vm;          // [BH][D] channel means of V, or null
+  __half* o;                // fp16 [BH][N][D]
+  int BH, N, D;
   bool causal;
   float sm_scale_log2;      // sm_scale * log2(e)
 };

@@ -86,8 +86,8 @@ bool make_o_map3(CUtensorMap* map, const void* base, int N, int BH, int D) {
   return make_map3(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, BH, D, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// FP4 codes: [BH][rows][cols] bytes (Q and K: rows = N tokens, cols = 64; V transposed: rows =
-// 128 channels, cols = tiles * 64), boxes of box_cols bytes x box_rows rows (a box never reaches
+// FP4 codes: [BH][rows][cols] bytes (Q and K: rows = N tokens, cols = d / 2; V transposed: rows =
+// d channels, cols = tiles * 64), boxes of box_cols bytes x box_rows rows (a box never reaches
 // into the next head), swizzle matching the box width (64 bytes: 64-byte, 32 bytes: 32-byte).
 bool make_fp4_map3(CUtensorMap* map, const void* base, int rows, int BH, int cols, int box_cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -528,11 +528,10 @@ int sage_quant_qk_fp4(const void* q, const void* k, const float* km, uint8_t* q4
   if (!q || !k || !q4 || !sfq || !gq || !k4 || !sfk || !gk) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if (d != 128) return SAGE_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q4) || !aligned16(k4) || !aligned16(sfq) || !aligned16(sfk))
     return SAGE_ERR_INVALID;
   return cuda_status(sage::launch_quant_qk_fp4(static_cast<const __half*>(q), static_cast<const __half*>(k), km, q4,
-                                               sfq, gq, k4, sfk, gk, B * H, N, static_cast<cudaStream_t>(stream)));
+                                               sfq, gq, k4, sfk, gk, B * H, N, d, static_cast<cudaStream_t>(stream)));
 }
 
 int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, int B, int H, int N, int d,
@@ -540,7 +539,6 @@ int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float
   if (!v || !v4t || !sfv || !gv) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if (d != 128) return SAGE_ERR_UNSUPPORTED;
   if (!aligned16(v) || !aligned16(v4t) || !aligned16(sfv)) return SAGE_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
@@ -550,7 +548,7 @@ int sage_quant_v_fp4(const void* v, uint8_t* v4t, uint8_t* sfv, float* gv, float
     return SAGE_ERR_NOMEM;
   }
   rc = cuda_status(sage::launch_quant_v_fp4(static_cast<const __half*>(v), v4t, sfv, gv, vm, static_cast<float*>(ws),
-                                            BH, N, st));
+                                            BH, N, d, st));
   const cudaError_t fe = cudaFreeAsync(ws, st);
   if (!rc && fe != cudaSuccess) rc = SAGE_ERR_CUDA;
   return rc;
@@ -563,16 +561,15 @@ int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const flo
   if (!q4 || !sfq || !gq || !k4 || !sfk || !gk || !v4t || !sfv || !gv || !o) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if (d != 128) return SAGE_ERR_UNSUPPORTED;
   if ((rc = check_scale(sm_scale))) return rc;
   if (!aligned16(q4) || !aligned16(k4) || !aligned16(v4t) || !aligned16(sfq) || !aligned16(sfk) || !aligned16(sfv) ||
       !aligned16(o))
     return SAGE_ERR_INVALID;
   const int BH = B * H, tiles = (N + 127) / 128;
   CUtensorMap tq, tk, tv;
-  // Q: 128-token boxes; K: 64-key boxes; V^T: 64 keys (32 bytes) of all 128 channels
-  if (!make_fp4_map3(&tq, q4, N, BH, 64, 64, 128) || !make_fp4_map3(&tk, k4, N, BH, 64, 64, 64) ||
-      !make_fp4_map3(&tv, v4t, 128, BH, tiles * 64, 32, 128))
+  // Q: 128-token boxes; K: 64-key boxes; V^T: 64 keys (32 bytes) of all d channels
+  if (!make_fp4_map3(&tq, q4, N, BH, d / 2, d / 2, 128) || !make_fp4_map3(&tk, k4, N, BH, d / 2, d / 2, 64) ||
+      !make_fp4_map3(&tv, v4t, d, BH, tiles * 64, 32, d))
     return SAGE_ERR_CUDA;
   sage::Fp4Args a{};
   a.tm_q = &tq;
@@ -588,6 +585,7 @@ int sage_attn_fwd_fp4_quantized(const uint8_t* q4, const uint8_t* sfq, const flo
   a.o = static_cast<__half*>(o);
   a.BH = BH;
   a.N = N;
+  a.D = d;
   a.causal = causal != 0;
   a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
   return cuda_status(sage::launch_attn_fp4(a, static_cast<cudaStream_t>(stream)));
@@ -598,18 +596,18 @@ int sage_attn_fwd_fp4(const void* q, const void* k, const void* v, void* o, int 
   if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
   int rc = check_shape(B, H, N, d);
   if (rc) return rc;
-  if (d != 128) return SAGE_ERR_UNSUPPORTED;
   if ((rc = check_scale(sm_scale))) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SAGE_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   const size_t tiles = static_cast<size_t>((N + 127) / 128);
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t codes = up(static_cast<size_t>(BH) * N * 64), atoms = up(static_cast<size_t>(BH) * tiles * 2 * 1024);
+  // atoms: the largest of sfq (tiles x d/64), sfk (2 tiles x d/64) and sfv (tiles x 2) atoms of 512 bytes
+  const size_t codes = up(static_cast<size_t>(BH) * N * (d / 2)), atoms = up(static_cast<size_t>(BH) * tiles * 4 * 512);
   const size_t tscales = up(static_cast<size_t>(BH) * tiles * 4), chan = up(static_cast<size_t>(BH) * d * 4);
   const size_t off_k4 = codes;
   const size_t off_v4 = off_k4 + codes;
-  const size_t off_sfq = off_v4 + up(static_cast<size_t>(BH) * 128 * tiles * 64);
+  const size_t off_sfq = off_v4 + up(static_cast<size_t>(BH) * d * tiles * 64);
   const size_t off_sfk = off_sfq + atoms;
   const size_t off_sfv = off_sfk + atoms;
   const size_t off_gq = off_sfv + atoms;
@@ -633,10 +631,10 @@ int sage_attn_fwd_fp4(const void* q, const void* k, const void* v, void* o, int 
   if (!rc)
     rc = cuda_status(sage::launch_quant_qk_fp4(static_cast<const __half*>(q), static_cast<const __half*>(k), km, w,
                                                w + off_sfq, reinterpret_cast<float*>(w + off_gq), w + off_k4,
-                                               w + off_sfk, reinterpret_cast<float*>(w + off_gk), BH, N, st));
+                                               w + off_sfk, reinterpret_cast<float*>(w + off_gk), BH, N, d, st));
   if (!rc)
     rc = cuda_status(sage::launch_quant_v_fp4(static_cast<const __half*>(v), w + off_v4, w + off_sfv, gv, vm,
-                                              reinterpret_cast<float*>(w + off_rv), BH, N, st));
+                                              reinterpret_cast<float*>(w + off_rv), BH, N, d, st));
   nvtxRangePop();
   nvtxRangePushA("sage_fp4_fused");
   if (!rc)

@@ -762,22 +762,22 @@ cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, i
 
 // Q (SMOOTH = false) or K minus its channel mean km: one CTA per (head, 128-token tile), one
 // thread per token.  g[bh, tile] = fl32(a / 2688) with a the tile's largest |x|; z = fl32(x *
-// fl32(2688 / a)); codes [BH][N][64 bytes].  Scale atoms: Q (ROWS64 = false) [BH][tiles][2][512],
-// the tile's 128 tokens as rows; K (ROWS64 = true) [BH][ceil(N/64)][2][512], each 64-token half
-// in the first 64 rows of its own atoms (the attention kernel's key tiles are 64 tokens), the
-// other rows zero.
-template <bool SMOOTH, bool ROWS64 = false>
+// fl32(2688 / a)); codes [BH][N][D/2 bytes].  Scale atoms (D/64 per row group, one per 64
+// channels): Q (ROWS64 = false) [BH][tiles][D/64][512], the tile's 128 tokens as rows; K
+// (ROWS64 = true) [BH][ceil(N/64)][D/64][512], each 64-token half in the first 64 rows of its own
+// atoms (the attention kernel's key tiles are 64 tokens), the other rows zero.
+template <int D, bool SMOOTH, bool ROWS64 = false>
 __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict__ x, const float* __restrict__ km,
                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                         float* __restrict__ g, int N) {
-  constexpr int D = 128;
+  constexpr int NA = D / 64;  // scale atoms per row group
   const int nt = (N + 127) / 128;
   const int bh = static_cast<int>(blockIdx.x) / nt, tile = static_cast<int>(blockIdx.x) % nt;
   const int r = threadIdx.x, row = tile * 128 + r;
   const bool live = row < N;
   __shared__ float s_km[D];
   __shared__ float s_max[4];
-  s_km[r] = SMOOTH ? km[static_cast<size_t>(bh) * D + r] : 0.f;
+  if (r < D) s_km[r] = SMOOTH ? km[static_cast<size_t>(bh) * D + r] : 0.f;
   __syncthreads();
   float v[D];
   const uint4* src = reinterpret_cast<const uint4*>(x + (static_cast<size_t>(bh) * N + (live ? row : 0)) * D);
@@ -799,8 +799,10 @@ __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict
   a = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
   const float rr = a > 0.f ? __fdiv_rn(2688.0f, a) : 0.f;
   if (r == 0) g[static_cast<size_t>(bh) * nt + tile] = __fdiv_rn(a, 2688.0f);
-  uint32_t w[16];
-  uint32_t sfw[2] = {0u, 0u};
+  uint32_t w[D / 8];
+  uint32_t sfw[NA];
+#pragma unroll
+  for (int a2 = 0; a2 < NA; ++a2) sfw[a2] = 0u;
 #pragma unroll
   for (int gi = 0; gi < D / 16; ++gi) {
     float z[16];
@@ -812,35 +814,34 @@ __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict
   if (live) {
     uint4* dst = reinterpret_cast<uint4*>(codes + (static_cast<size_t>(bh) * N + row) * (D / 2));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    for (int i = 0; i < D / 32; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
   }
   if constexpr (ROWS64) {
     const int n64 = (N + 63) / 64, half = tile * 2 + (r >> 6), lr = r & 63;
     if (half < n64) {
-      uint8_t* atoms = sf + (static_cast<size_t>(bh) * n64 + half) * 1024 + (lr & 31) * 16 + (lr >> 5) * 4;
-      *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
-      *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
-      if (lr < 32) {  // rows 64..127 of the atoms (bytes 8..15 of each 16-byte line): zero
-        *reinterpret_cast<uint2*>(atoms + 8) = make_uint2(0u, 0u);
-        *reinterpret_cast<uint2*>(atoms + 512 + 8) = make_uint2(0u, 0u);
+      uint8_t* atoms = sf + (static_cast<size_t>(bh) * n64 + half) * (NA * 512) + (lr & 31) * 16 + (lr >> 5) * 4;
+#pragma unroll
+      for (int a2 = 0; a2 < NA; ++a2) {
+        *reinterpret_cast<uint32_t*>(atoms + 512 * a2) = sfw[a2];
+        if (lr < 32)  // rows 64..127 of the atom (bytes 8..15 of each 16-byte line): zero
+          *reinterpret_cast<uint2*>(atoms + 512 * a2 + 8) = make_uint2(0u, 0u);
       }
     }
   } else {
-    uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (r & 31) * 16 + (r >> 5) * 4;
-    *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
-    *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+    uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * (NA * 512) + (r & 31) * 16 + (r >> 5) * 4;
+#pragma unroll
+    for (int a2 = 0; a2 < NA; ++a2) *reinterpret_cast<uint32_t*>(atoms + 512 * a2) = sfw[a2];
   }
 }
 
 // V codes along the tokens: one CTA per (head, 128-key tile), one thread per channel.
-// z = fl32(fl32(v - vm) * rv), groups of 16 keys; codes transposed [BH][128][n_tiles * 64 bytes]
-// (keys past N: zero codes, outside every group's maximum); scale atoms [BH][tiles][2][512] with
-// the channels as rows.
-template <bool SMOOTH>
+// z = fl32(fl32(v - vm) * rv), groups of 16 keys; codes transposed [BH][D][n_tiles * 64 bytes]
+// (keys past N: zero codes, outside every group's maximum); scale atoms [BH][tiles][2][512] (keys
+// 0-63, 64-127 of the tile) with the D channels as rows (D = 64: rows 64..127 zero).
+template <int D, bool SMOOTH>
 __global__ void __launch_bounds__(128) quant_v_fp4_kernel(const __half* __restrict__ v, const float* __restrict__ vm,
                                                           const float* __restrict__ rv, uint8_t* __restrict__ codes_t,
                                                           uint8_t* __restrict__ sf, int N) {
-  constexpr int D = 128;
   const int nt = (N + 127) / 128;
   const int bh = static_cast<int>(blockIdx.x) / nt, tile = static_cast<int>(blockIdx.x) % nt;
   const int c = threadIdx.x;
@@ -869,27 +870,47 @@ __global__ void __launch_bounds__(128) quant_v_fp4_kernel(const __half* __restri
   uint8_t* atoms = sf + (static_cast<size_t>(bh) * nt + tile) * 1024 + (c & 31) * 16 + (c >> 5) * 4;
   *reinterpret_cast<uint32_t*>(atoms) = sfw[0];
   *reinterpret_cast<uint32_t*>(atoms + 512) = sfw[1];
+  if (D == 64 && c < 32) {  // rows 64..127 of the atoms: zero
+    *reinterpret_cast<uint2*>(atoms + 8) = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(atoms + 512 + 8) = make_uint2(0u, 0u);
+  }
+}
+
+template <int D>
+static cudaError_t launch_quant_qk_fp4_d(const __half* q, const __half* k, const float* km, uint8_t* q4, uint8_t* sfq,
+                                         float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N,
+                                         cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
+  quant_fp4_kernel<D, false><<<blocks, 128, 0, st>>>(q, nullptr, q4, sfq, gq, N);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (km) quant_fp4_kernel<D, true, true><<<blocks, 128, 0, st>>>(k, km, k4, sfk, gk, N);
+  else quant_fp4_kernel<D, false, true><<<blocks, 128, 0, st>>>(k, nullptr, k4, sfk, gk, N);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_qk_fp4(const __half* q, const __half* k, const float* km, uint8_t* q4, uint8_t* sfq,
-                                float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, cudaStream_t st) {
-  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
-  quant_fp4_kernel<false><<<blocks, 128, 0, st>>>(q, nullptr, q4, sfq, gq, N);
-  cudaError_t e = cudaGetLastError();
+                                float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, int D,
+                                cudaStream_t st) {
+  return D == 128 ? launch_quant_qk_fp4_d<128>(q, k, km, q4, sfq, gq, k4, sfk, gk, BH, N, st)
+                  : launch_quant_qk_fp4_d<64>(q, k, km, q4, sfq, gq, k4, sfk, gk, BH, N, st);
+}
+
+template <int D>
+static cudaError_t launch_quant_v_fp4_d(const __half* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, float* rv,
+                                        int BH, int N, cudaStream_t st) {
+  cudaError_t e = launch_quant_v_fp8_d<D, true>(v, nullptr, gv, vm, BH, N, st, rv);
   if (e != cudaSuccess) return e;
-  if (km) quant_fp4_kernel<true, true><<<blocks, 128, 0, st>>>(k, km, k4, sfk, gk, N);
-  else quant_fp4_kernel<false, true><<<blocks, 128, 0, st>>>(k, nullptr, k4, sfk, gk, N);
+  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
+  if (vm) quant_v_fp4_kernel<D, true><<<blocks, D, 0, st>>>(v, vm, rv, v4t, sfv, N);
+  else quant_v_fp4_kernel<D, false><<<blocks, D, 0, st>>>(v, nullptr, rv, v4t, sfv, N);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant_v_fp4(const __half* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, float* rv, int BH,
-                               int N, cudaStream_t st) {
-  cudaError_t e = launch_quant_v_fp8_d<128, true>(v, nullptr, gv, vm, BH, N, st, rv);
-  if (e != cudaSuccess) return e;
-  const unsigned blocks = static_cast<unsigned>(BH) * static_cast<unsigned>((N + 127) / 128);
-  if (vm) quant_v_fp4_kernel<true><<<blocks, 128, 0, st>>>(v, vm, rv, v4t, sfv, N);
-  else quant_v_fp4_kernel<false><<<blocks, 128, 0, st>>>(v, nullptr, rv, v4t, sfv, N);
-  return cudaGetLastError();
+                               int N, int D, cudaStream_t st) {
+  return D == 128 ? launch_quant_v_fp4_d<128>(v, v4t, sfv, gv, vm, rv, BH, N, st)
+                  : launch_quant_v_fp4_d<64>(v, v4t, sfv, gv, vm, rv, BH, N, st);
 }
 
 }  // namespace sage

@@ -22,15 +22,16 @@ cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8, float* sv, float* v
 cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, int8_t* q8, int8_t* k8, float* sq,
                             float* sk, int BH, int N, int D, bool per_token, cudaStream_t st);
 
-// Microscaling FP4 variant (head dimension 128).  Q and K (minus km when not null) to E2M1
-// codes [BH][N][64 bytes] and tile scales [BH][ceil(N/128)]; scale atoms of Q [BH][ceil(N/128)]
-// [2][512], of K [BH][ceil(N/64)][2][512] (64 tokens per atom pair).
+// Microscaling FP4 variant (head dimension D = 64 or 128).  Q and K (minus km when not null) to
+// E2M1 codes [BH][N][D/2 bytes] and tile scales [BH][ceil(N/128)]; scale atoms of Q
+// [BH][ceil(N/128)][D/64][512], of K [BH][ceil(N/64)][D/64][512] (64 tokens per atom).
 cudaError_t launch_quant_qk_fp4(const __half* q, const __half* k, const float* km, uint8_t* q4, uint8_t* sfq,
-                                float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, cudaStream_t st);
-// V to E2M1 along the tokens: transposed codes [BH][128][ceil(N/128) * 64 bytes], scale atoms
-// [BH][ceil(N/128)][2][512], channel scales gv [BH][128], channel means vm (V smoothed; nullptr:
-// not smoothed), rv [BH][128] scratch (the inverse channel scales).
+                                float* gq, uint8_t* k4, uint8_t* sfk, float* gk, int BH, int N, int D,
+                                cudaStream_t st);
+// V to E2M1 along the tokens: transposed codes [BH][D][ceil(N/128) * 64 bytes], scale atoms
+// [BH][ceil(N/128)][2][512] (the channels as rows), channel scales gv [BH][D], channel means vm
+// (V smoothed; nullptr: not smoothed), rv [BH][D] scratch (the inverse channel scales).
 cudaError_t launch_quant_v_fp4(const __half* v, uint8_t* v4t, uint8_t* sfv, float* gv, float* vm, float* rv, int BH,
-                               int N, cudaStream_t st);
+                               int N, int D, cudaStream_t st);
 
 }  // namespace sage

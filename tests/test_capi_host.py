@@ -101,8 +101,10 @@ def test_variant_entries_validate_before_any_cuda_call(sa):
     s = ctypes.c_void_p(0)
     mis = ctypes.c_void_p(0x1008)
     inv, uns = sa.SAGE_ERR_INVALID, sa.SAGE_ERR_UNSUPPORTED
-    # microscaling FP4: head dimension 128 only
-    assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, 0, 0.1, s) == uns
+    # microscaling FP4: head dimension 64 or 128
+    assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 96, 0, 0.1, s) == uns
+    assert L.sage_attn_fwd_fp4_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                         1, 1, 256, 32, 0, 0.1, s) == uns
     assert L.sage_attn_fwd_fp4(FAKE, FAKE, FAKE, None, 1, 1, 256, 128, 0, 0.1, s) == inv
     assert L.sage_attn_fwd_fp4(mis, FAKE, FAKE, FAKE, 1, 1, 256, 128, 0, 0.1, s) == inv
     for bad in (0.0, -1.0, float("nan"), float("inf")):
@@ -110,10 +112,10 @@ def test_variant_entries_validate_before_any_cuda_call(sa):
         assert L.sage_attn_fwd_fp4_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
                                              1, 1, 256, 128, 0, bad, s) == inv
     assert L.sage_quant_qk_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 256, 128, s) == inv
-    assert L.sage_quant_qk_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 64, s) == uns
+    assert L.sage_quant_qk_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 256, s) == uns
     assert L.sage_quant_qk_fp4(FAKE, FAKE, None, mis, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 128, s) == inv
     assert L.sage_quant_v_fp4(FAKE, None, FAKE, FAKE, None, 1, 1, 256, 128, s) == inv
-    assert L.sage_quant_v_fp4(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 256, 64, s) == uns
+    assert L.sage_quant_v_fp4(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 256, 96, s) == uns
     assert L.sage_attn_fwd_fp4_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, mis, FAKE, None, FAKE,
                                          1, 1, 256, 128, 0, 0.1, s) == inv
     # FP8 P.V: head dimension 128 only

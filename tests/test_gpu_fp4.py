@@ -45,28 +45,28 @@ def unpack_codes(packed: np.ndarray) -> np.ndarray:
 
 
 def atoms_to_scales(atoms: np.ndarray) -> np.ndarray:
-    """[..., tiles, 2, 512] scale atoms -> [..., tiles * 128, 8] scales per (row, group of 16)."""
+    """[..., tiles, A, 512] scale atoms -> [..., tiles * 128, 4A] scales per (row, group of 16)."""
     lead = atoms.shape[:-3]
-    t = atoms.shape[-3]
+    t, a = atoms.shape[-3], atoms.shape[-2]
     r = np.arange(128)
-    out = np.empty(lead + (t, 128, 8), np.uint8)
-    for g in range(8):
+    out = np.empty(lead + (t, 128, 4 * a), np.uint8)
+    for g in range(4 * a):
         out[..., g] = atoms[..., g // 4, :][..., (r % 32) * 16 + (r // 32) * 4 + g % 4]
-    return out.reshape(lead + (t * 128, 8))
+    return out.reshape(lead + (t * 128, 4 * a))
 
 
 def atoms64_to_scales(atoms: np.ndarray) -> np.ndarray:
-    """K's [..., halves, 2, 512] scale atoms (64 tokens as each atom pair's first rows) ->
-    [..., halves * 64, 8]; also checks that the atoms' other rows are zero."""
+    """[..., halves, A, 512] scale atoms with 64 rows each (K's tokens, or V's channels at d = 64)
+    -> [..., halves * 64, 4A]; also checks that the atoms' other rows are zero."""
     lead = atoms.shape[:-3]
-    t = atoms.shape[-3]
+    t, a = atoms.shape[-3], atoms.shape[-2]
     r = np.arange(64)
-    out = np.empty(lead + (t, 64, 8), np.uint8)
-    for g in range(8):
+    out = np.empty(lead + (t, 64, 4 * a), np.uint8)
+    for g in range(4 * a):
         out[..., g] = atoms[..., g // 4, :][..., (r % 32) * 16 + (r // 32) * 4 + g % 4]
-    lines = atoms.reshape(lead + (t, 2, 32, 16))
-    assert not lines[..., 8:].any(), "rows 64..127 of K's scale atoms must be zero"
-    return out.reshape(lead + (t * 64, 8))
+    lines = atoms.reshape(lead + (t, a, 32, 16))
+    assert not lines[..., 8:].any(), "rows 64..127 of 64-row scale atoms must be zero"
+    return out.reshape(lead + (t * 64, 4 * a))
 
 
 def gpu_quant(sa, q, k, v, smooth_v=True):
@@ -93,15 +93,17 @@ def check_codes(b, ref, N):
     np.testing.assert_array_equal(cpu["gv"], ref["gv"], err_msg="gv")
     if ref["vm"] is not None:
         np.testing.assert_array_equal(cpu["vm"], ref["vm"], err_msg="vm")
-    vt = unpack_codes(cpu["v4t"])                   # [B,H,128,tiles*128]
+    vt = unpack_codes(cpu["v4t"])                   # [B,H,d,tiles*128]
     vcodes = np.swapaxes(vt, -1, -2)[..., :N, :]   # token-major
     diff = vcodes != ref["v4"]
     assert not diff.any(), f"v4: {diff.sum()} codes differ (first at {np.argwhere(diff)[0]})"
     assert not vt[..., N:].any(), "V codes past N must be zero"
-    vs = atoms_to_scales(cpu["sfv"])               # [B,H,tiles*128 (channels per tile), 8]
+    d = vt.shape[-2]
+    # [B,H,tiles*d (channels per tile), 8]
+    vs = atoms_to_scales(cpu["sfv"]) if d == 128 else atoms64_to_scales(cpu["sfv"])
     B, H = vs.shape[:2]
     t = cpu["sfv"].shape[2]
-    vs = vs.reshape(B, H, t, 128, 8).transpose(0, 1, 2, 4, 3).reshape(B, H, t * 8, 128)
+    vs = vs.reshape(B, H, t, d, 8).transpose(0, 1, 2, 4, 3).reshape(B, H, t * 8, d)
     ng = -(-N // 16)
     np.testing.assert_array_equal(vs[..., :ng, :], ref["vs"], err_msg="sfv")
 
@@ -134,6 +136,9 @@ SMALL = [
     W.Workload("fp4_ragged_n1000", 2, 1, 1000, 128, False, True, q_std=1.5),
     W.Workload("fp4_ragged_causal_n700", 1, 2, 700, 128, True, True, bias_std=4.0),
     W.Workload("fp4_win_n2048", 1, 2, 2048, 128, False, True, window=256, align=10.0),
+    W.Workload("fp4_d64_n256", 1, 2, 256, 64, False, True, n_out=4, out_mag=20.0),
+    W.Workload("fp4_d64_ragged_causal_n700", 1, 2, 700, 64, True, True, bias_std=4.0),
+    W.Workload("fp4_d64_win_n2048", 2, 1, 2048, 64, False, True, window=256, align=12.0, bias_std=4.0),
 ]
 
 
@@ -157,11 +162,12 @@ def test_fp4_codes_and_output_match_the_oracle(sa, w):
     assert torch.equal(o2, o)
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 129, 200])
-def test_fp4_edge_sizes(sa, N, causal):
+def test_fp4_edge_sizes(sa, N, causal, d):
     # a single token, partial 64-key tiles, a partial 128-token scale tile, one key tile plus one key
-    w = W.Workload(f"fp4_edge_{N}", 1, 2, N, 128, causal, True, n_out=2, out_mag=10.0)
+    w = W.Workload(f"fp4_edge_{N}", 1, 2, N, d, causal, True, n_out=2, out_mag=10.0)
     q, k, v = W.make_qkv(w)
     b = gpu_quant(sa, q, k, v)
     ref = oracle.sage_attn_fp4(q, k, v, causal, w.sm_scale)
@@ -201,7 +207,7 @@ def test_fp4_without_v_smoothing(sa):
     check_o(o.float().cpu().numpy(), o64, env, unsure, vhat_max(ref), "no V smoothing")
 
 
-@pytest.mark.parametrize("w", [W.HEADLINE, W.SPARSE], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [W.HEADLINE, W.SPARSE, W.SPARSE_DIT], ids=lambda w: w.name)
 def test_fp4_full_size_sampled_rows(sa, w):
     q, k, v = W.make_qkv(w)
     o = torch.empty_like(q, device="cuda")
@@ -242,8 +248,8 @@ def test_fp4_close_to_exact_attention(sa):
     assert c_ref >= 0.95, f"the method's cosine to exact attention {c_ref:.4f}"
 
 
-def test_fp4_rejects_head_dimension_64(sa):
-    q = torch.zeros((1, 1, 256, 64), dtype=torch.float16, device="cuda")
+def test_fp4_rejects_other_head_dimensions(sa):
+    q = torch.zeros((1, 1, 256, 96), dtype=torch.float16, device="cuda")
     with pytest.raises(sa.SageError) as e:
         sa.sage_attn_fwd_fp4(q, q, q, torch.empty_like(q), False, 0.125)
     assert e.value.status == sa.SAGE_ERR_UNSUPPORTED
