@@ -9,7 +9,9 @@
 //   online softmax over 64-key tiles with an integer offset m = ceil(max u seen so far); when it
 //   grows, O and the row sum are scaled by 2^(m_old - m_new) (exact)
 //   p   = 2^(u - m + 10)         the row sum takes p unrounded
-//   P~  = microscaled E2M1 of p, one UE4M3 scale per 16 keys
+//   P~  = microscaled E2M1 of p, one UE4M3 scale per 16 keys; the kernel takes a group's
+//         scale from the exp2 of its largest score and the codes of p / scale as
+//         exp2(u - m + 10 - log2 scale), one exponential per key
 //   O  += P~ . V4                V4: E2M1 codes of (V - vm) / gv along the keys, 16 keys per scale
 //   O   = O * gv / l + vm        stored as fp16
 //
@@ -242,9 +244,16 @@ __global__ void __launch_bounds__(192, 2)
         for (int c = 0; c < 64; ++c)
           if (c > cmax) x[c] = 0xFF800000u;
       }
-      float sm = -INFINITY;
+      // the largest score of each group of 16 keys (the group's largest p, below) and of the row
+      float gs[4];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) sm = max3f(sm, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+      for (int gi = 0; gi < 4; ++gi) {
+        float g = fmaxf(__uint_as_float(x[16 * gi]), __uint_as_float(x[16 * gi + 1]));
+#pragma unroll
+        for (int c = 16 * gi + 2; c < 16 * gi + 16; c += 2) g = max3f(g, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+        gs[gi] = g;
+      }
+      const float sm = fmaxf(fmaxf(gs[0], gs[1]), fmaxf(gs[2], gs[3]));
       const float mx = sm == -INFINITY ? -INFINITY : __fmul_rn(sm, cb);
       // integer offset: set by the first tile (every row sees key 0), moved up when a tile's
       // maximum passes it
@@ -281,18 +290,33 @@ __global__ void __launch_bounds__(192, 2)
       uint32_t sfw = 0u;
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
-        float2 z[8];
+        // group scale from the group's largest p, the exp2 of its largest score (fl(S * cb - m + 10)
+        // rounds as in the pass below); then the codes' operand z = p / scale directly as
+        // exp2(S * cb - m + 10 - log2 scale), and p = z * scale for the row sum.  A zero scale (all
+        // p of the group below 6 * 2^-10) keeps z = p, whose codes round to zero.
+        const float gm = fast_exp2(fmaf(gs[gi], cb, -m_e));
+        const uint32_t s8 = e4m3_code(__fmul_rn(gm, 0.16666667163372040f));
+        float nb = -m_e, se = 1.f;
+        if (s8 != 0u) {
+          se = e4m3_value(s8);
+          nb = -__fadd_rn(m_e, fast_log2(se));
+        }
+        float y[16];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int c = 16 * gi + 2 * k;
           const float2 tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
-                                       make_float2(cb, cb), make_float2(-m_e, -m_e));
+                                       make_float2(cb, cb), make_float2(nb, nb));
           // one pair in four on the FMA pipe (exp2_poly2, relative error <= 7.5e-5), the rest on
           // the MUFU unit; masked keys: exp2(-inf) = 0 (the polynomial gives 2^-126)
-          z[k] = (k & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
-          lsum[k & 3] = __fadd2_rn(lsum[k & 3], z[k]);
+          const float2 z = (k & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
+          lsum[k & 3] = __ffma2_rn(z, make_float2(se, se), lsum[k & 3]);
+          y[2 * k] = z.x;
+          y[2 * k + 1] = z.y;
         }
-        sfw |= microscale16_pos(z, w[2 * gi], w[2 * gi + 1]) << (8 * gi);
+        w[2 * gi] = e2m1x8(y);
+        w[2 * gi + 1] = e2m1x8(y + 8);
+        sfw |= s8 << (8 * gi);
       }
       // P~ row r: keys 32c .. 32c+31 are the 16-byte chunk c of the row's 32 bytes
 #pragma unroll

@@ -1,5 +1,5 @@
 // fp4_codes.cuh -- E2M1 / E4M3 conversions and the microscaling of one group of 16 values,
-// shared by the FP4 quantization kernels and the FP4 attention kernel.
+// used by the FP4 quantization kernels (the conversions also by the FP4 attention kernel).
 //
 // Microscaling (SageAttention3 abstract: FP4 attention with microscaling; the format is the
 // one Blackwell's block-scaled FP4 products read): one UE4M3 scale per 16 elements along the
@@ -52,34 +52,6 @@ __device__ __forceinline__ uint32_t microscale16(const float (&z)[16], uint32_t&
   float y[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) y[k] = __fmul_rn(z[k], inv);
-  w0 = e2m1x8(y);
-  w1 = e2m1x8(y + 8);
-  return s8;
-}
-
-// The same for 16 non-negative values held as 8 pairs (P~, whose values the kernel computes in
-// fp32 with exp2 approximations anyway): packed maxima and products, and max/6 and 1/scale
-// within an ulp (a product with fl32(1/6), the hardware reciprocal) instead of correctly
-// rounded: a decision that these change lies within a relative 1e-6 of a rounding midpoint.
-__device__ __forceinline__ uint32_t microscale16_pos(const float2 (&z)[8], uint32_t& w0, uint32_t& w1) {
-  float gm = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float m;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(gm), "f"(z[k].x), "f"(z[k].y));
-    gm = m;
-  }
-  const uint32_t s8 = e4m3_code(__fmul_rn(gm, 0.16666667163372040f));
-  const float sd = e4m3_value(s8);
-  float inv = 0.f;
-  if (sd > 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(sd));
-  float y[16];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float2 t = __fmul2_rn(z[k], make_float2(inv, inv));
-    y[2 * k] = t.x;
-    y[2 * k + 1] = t.y;
-  }
   w0 = e2m1x8(y);
   w1 = e2m1x8(y + 8);
   return s8;
