@@ -267,23 +267,10 @@ __global__ void __launch_bounds__(192, 2)
         m_use = m_new;
         rescale = true;
       }
-      // P~.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1)
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (j - 1) & 1, abort_flag))) { ok = false; break; }
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
+      const bool any_rescale = __any_sync(0xffffffffu, rescale);
+      if (any_rescale) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) lsum[i] = __fmul2_rn(lsum[i], make_float2(alpha, alpha));
-#pragma unroll
-        for (int cb2 = 0; cb2 < D; cb2 += 32) {
-          uint32_t ov[32];
-          tmem_ld32_sync(tO + cb2, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tO + cb2, ov);
-        }
-        tmem_wait_st();
       }
       const float m_e = m_use - 10.f;  // p = 2^(S * cb - m + 10); exact: m is an integer
       uint32_t w[8];
@@ -317,6 +304,23 @@ __global__ void __launch_bounds__(192, 2)
         w[2 * gi] = e2m1x8(y);
         w[2 * gi + 1] = e2m1x8(y + 8);
         sfw |= s8 << (8 * gi);
+      }
+      // P~.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1): the
+      // codes above are computed in registers while it runs
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (j - 1) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (any_rescale) {
+#pragma unroll
+        for (int cb2 = 0; cb2 < D; cb2 += 32) {
+          uint32_t ov[32];
+          tmem_ld32_sync(tO + cb2, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tO + cb2, ov);
+        }
+        tmem_wait_st();
       }
       // P~ row r: keys 32c .. 32c+31 are the 16-byte chunk c of the row's 32 bytes
 #pragma unroll
