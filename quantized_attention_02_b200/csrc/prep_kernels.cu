@@ -469,7 +469,7 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 // exact channel mean (vm), the channel scale sv = fl32(a / 2688) and its inverse rv =
 // fl32(2688 / a) (2688 = 6 * 448: the largest E2M1 code times the largest E4M3 scale); no codes.
 template <int D, bool SMOOTH, bool FP4 = false>
-__global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __half* __restrict__ v,
+__global__ void __launch_bounds__(kSmoothThreads, 2) quant_v_fp8_kernel(const __half* __restrict__ v,
                                                                      uint8_t* __restrict__ v8, float* __restrict__ sv,
                                                                      float* __restrict__ vm, int N,
                                                                      float* __restrict__ rv = nullptr) {
@@ -488,14 +488,16 @@ __global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __hal
   const int t1 = min(N, t0 + slice);
   const __half* base = v + (static_cast<size_t>(bh) * N) * D + piece * 8;
 
-  // ---- pass 1: exact sums, maxima and minima of this thread's 8 channels over its rows
+  // ---- pass 1: exact sums, maxima and minima of this thread's 8 channels over its rows (the
+  // extrema as fp16 pairs: exact, two channels per instruction)
   long long acc[8];
-  float mx[8], mn[8];
+  __half2 hmx[4], hmn[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    acc[i] = 0;
-    mx[i] = -INFINITY;
-    mn[i] = INFINITY;
+  for (int i = 0; i < 8; ++i) acc[i] = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hmx[i] = __halves2half2(__ushort_as_half(0xFC00u), __ushort_as_half(0xFC00u));  // -inf
+    hmn[i] = __halves2half2(__ushort_as_half(0x7C00u), __ushort_as_half(0x7C00u));  // +inf
   }
   constexpr int ITERS = kSplitFlushTokens / U;
   for (int t = t0 + row; t < t1;) {
@@ -521,11 +523,9 @@ __global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __hal
         for (int i = 0; i < 4; ++i) {
           if constexpr (SMOOTH) split_acc(words[i], hs[2 * i], hs[2 * i + 1], ls[i]);
           if (live[u]) {
-            const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&words[i]));
-            mx[2 * i] = fmaxf(mx[2 * i], x.x);
-            mx[2 * i + 1] = fmaxf(mx[2 * i + 1], x.y);
-            mn[2 * i] = fminf(mn[2 * i], x.x);
-            mn[2 * i + 1] = fminf(mn[2 * i + 1], x.y);
+            const __half2 x = *reinterpret_cast<const __half2*>(&words[i]);
+            hmx[i] = __hmax2(hmx[i], x);
+            hmn[i] = __hmin2(hmn[i], x);
           }
         }
       }
@@ -537,6 +537,14 @@ __global__ void __launch_bounds__(kSmoothThreads) quant_v_fp8_kernel(const __hal
         acc[2 * i + 1] += (static_cast<long long>(hs[2 * i + 1]) << 18) + __float2int_rn(__fmul_rn(ls[i].y, 16777216.0f));
       }
     }
+  }
+  float mx[8], mn[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mx[2 * i] = __low2float(hmx[i]);
+    mx[2 * i + 1] = __high2float(hmx[i]);
+    mn[2 * i] = __low2float(hmn[i]);
+    mn[2 * i + 1] = __high2float(hmn[i]);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
