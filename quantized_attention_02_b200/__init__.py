@@ -386,12 +386,25 @@ def empty_quantized(q: torch.Tensor, granularity: int):
     return km, q8, k8, sq, sk
 
 
+VARIANTS = ("fp16pv", "fp8pv", "fp4")
+
+
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
-             sm_scale: float | None = None, granularity: int = SAGE_PER_BLOCK, stream=None) -> torch.Tensor:
-    """O = softmax(Q K^T sm_scale) V with smoothed INT8 Q K^T and FP16 P V.
-    sm_scale defaults to d^-1/2."""
+             sm_scale: float | None = None, granularity: int = SAGE_PER_BLOCK, variant: str = "fp16pv",
+             stream=None) -> torch.Tensor:
+    """O = softmax(Q K^T sm_scale) V on fp16 [B, H, N, d] CUDA tensors; sm_scale defaults to d^-1/2.
+    variant: "fp16pv" the method (smoothed K, INT8 Q K^T with per-token or per-block scales, FP16 P V);
+    "fp8pv" its FP8 P~ V variant (E4M3 P~ and smoothed V; d = 128); "fp4" the microscaling FP4 variant
+    (E2M1 Q, K, P~, V with UE4M3 scales per 16 elements; granularity does not apply)."""
+    if variant not in VARIANTS:
+        raise ValueError(f"variant must be one of {VARIANTS}, not {variant!r}")
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(q.shape[-1])
     o = torch.empty_like(q)
-    sage_attn_fwd(q, k, v, o, causal, sm_scale, granularity, stream)
+    if variant == "fp4":
+        sage_attn_fwd_fp4(q, k, v, o, causal, sm_scale, stream)
+    elif variant == "fp8pv":
+        sage_attn_fwd_fp8pv(q, k, v, o, causal, sm_scale, granularity, stream)
+    else:
+        sage_attn_fwd(q, k, v, o, causal, sm_scale, granularity, stream)
     return o

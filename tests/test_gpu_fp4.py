@@ -253,3 +253,19 @@ def test_fp4_rejects_other_head_dimensions(sa):
     with pytest.raises(sa.SageError) as e:
         sa.sage_attn_fwd_fp4(q, q, q, torch.empty_like(q), False, 0.125)
     assert e.value.status == sa.SAGE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_sageattn_variants_match_their_entry_points(sa, d):
+    w = W.Workload(f"variants_d{d}", 1, 2, 320, d, True, True, n_out=2, out_mag=10.0)
+    q, k, v = (x.cuda() for x in W.make_qkv(w))
+    calls = [("fp16pv", lambda o: sa.sage_attn_fwd(q, k, v, o, True, w.sm_scale, sa.SAGE_PER_BLOCK)),
+             ("fp4", lambda o: sa.sage_attn_fwd_fp4(q, k, v, o, True, w.sm_scale))]
+    if d == 128:
+        calls.append(("fp8pv", lambda o: sa.sage_attn_fwd_fp8pv(q, k, v, o, True, w.sm_scale, sa.SAGE_PER_BLOCK)))
+    for variant, direct in calls:
+        want = torch.empty_like(q)
+        direct(want)
+        got = sa.sageattn(q, k, v, causal=True, sm_scale=w.sm_scale, variant=variant)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), variant
