@@ -847,16 +847,22 @@ __global__ void __launch_bounds__(128) quant_fp4_kernel(const __half* __restrict
 // (keys past N: zero codes, outside every group's maximum); scale atoms [BH][tiles][2][512] (keys
 // 0-63, 64-127 of the tile) with the D channels as rows (D = 64: rows 64..127 zero).
 template <int D, bool SMOOTH>
-__global__ void __launch_bounds__(128) quant_v_fp4_kernel(const __half* __restrict__ v, const float* __restrict__ vm,
-                                                          const float* __restrict__ rv, uint8_t* __restrict__ codes_t,
-                                                          uint8_t* __restrict__ sf, int N) {
+__global__ void __launch_bounds__(D) quant_v_fp4_kernel(const __half* __restrict__ v, const float* __restrict__ vm,
+                                                        const float* __restrict__ rv, uint8_t* __restrict__ codes_t,
+                                                        uint8_t* __restrict__ sf, int N) {
   const int nt = (N + 127) / 128;
   const int bh = static_cast<int>(blockIdx.x) / nt, tile = static_cast<int>(blockIdx.x) % nt;
   const int c = threadIdx.x;
   const float mean = SMOOTH ? vm[static_cast<size_t>(bh) * D + c] : 0.f;
   const float rr = rv[static_cast<size_t>(bh) * D + c];
-  const __half* src = v + (static_cast<size_t>(bh) * N + tile * 128) * D + c;
   const int n_live = min(128, N - tile * 128);
+  // the tile's rows in shared memory (16-byte loads across the CTA), then one channel per thread
+  __shared__ uint4 s_tile[128 * D / 8];
+  const uint4* gsrc = reinterpret_cast<const uint4*>(v + (static_cast<size_t>(bh) * N + tile * 128) * D);
+#pragma unroll 4
+  for (int i = c; i < n_live * (D / 8); i += D) s_tile[i] = __ldg(gsrc + i);
+  __syncthreads();
+  const __half* src = reinterpret_cast<const __half*>(s_tile) + c;
   uint32_t w[16];
   uint32_t sfw[2] = {0u, 0u};
 #pragma unroll
