@@ -418,7 +418,7 @@ def run_ours(args, w: W.Workload):
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
-        if fp8 or sparse or fp4:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
+        if sparse:  # the variant's C-ABI call between a host->device copy of Q, K, V and the copy of O back
             q.copy_(qp, non_blocking=True)
             k.copy_(kp, non_blocking=True)
             v.copy_(vp, non_blocking=True)
@@ -426,8 +426,9 @@ def run_ours(args, w: W.Workload):
             op.copy_(o, non_blocking=True)
             return
         # the C-ABI call with host buffers: copies in, compute and copies out overlap across
-        # chunks of heads inside the call
-        sa.sage_attn_fwd_host(qp, kp, vp, op, w.causal, w.sm_scale, gran, 0, stream)
+        # chunks of heads inside the call (the method, or its FP8 P.V / FP4 variant)
+        sa.sage_attn_fwd_host(qp, kp, vp, op, w.causal, w.sm_scale, gran, 0, stream,
+                              variant="fp4" if fp4 else ("fp8pv" if fp8 else "fp16pv"))
 
     e2e_step()
     torch.cuda.synchronize(dev)

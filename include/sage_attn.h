@@ -327,6 +327,20 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
 int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
                        int causal, float sm_scale, int granularity, int heads_per_chunk, void* stream);
 
+/* Variants for sage_attn_fwd_host_variant. */
+enum { SAGE_VARIANT_FP16PV = 0, SAGE_VARIANT_FP8PV = 1, SAGE_VARIANT_FP4 = 2 };
+
+/* sage_attn_fwd_host for the method or one of its variants: each chunk of heads runs
+ * sage_attn_fwd (SAGE_VARIANT_FP16PV, identical to sage_attn_fwd_host), sage_attn_fwd_fp8pv
+ * (SAGE_VARIANT_FP8PV, d = 128) or sage_attn_fwd_fp4 (SAGE_VARIANT_FP4, d = 64 or 128;
+ * granularity must still be a valid value and is not used) on its device copies.  The output
+ * is bit-identical to that entry point on the whole tensors.  An unknown variant gives
+ * SAGE_ERR_INVALID, SAGE_VARIANT_FP8PV with d = 64 SAGE_ERR_UNSUPPORTED, both before any copy
+ * is enqueued; otherwise as sage_attn_fwd_host. */
+int sage_attn_fwd_host_variant(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                               int causal, float sm_scale, int granularity, int heads_per_chunk, int variant,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

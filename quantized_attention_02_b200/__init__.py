@@ -74,12 +74,14 @@ def get_lib() -> ctypes.CDLL:
         lib.sage_debug_mma_peak.argtypes = [_i, _i, _i, _p, _p, _p]
         lib.sage_debug_wait_timeout.argtypes = [_p, _p]
         lib.sage_attn_fwd_host.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p]
+        lib.sage_attn_fwd_host_variant.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _p]
         for n in ("sage_smooth_k", "sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_quantized",
                   "sage_debug_qk_int32", "sage_last_device_error", "sage_attn_fwd_noalloc",
                   "sage_debug_attn_trace", "sage_debug_mma_peak", "sage_attn_fwd_host",
                   "sage_debug_wait_timeout", "sage_quant_v_fp8", "sage_attn_fwd_fp8pv_quantized", "sage_prep_qk",
                   "sage_attn_fwd_fp8pv", "sage_sparse_predict", "sage_attn_fwd_sparse_quantized",
-                  "sage_attn_fwd_sparse"):
+                  "sage_attn_fwd_sparse", "sage_attn_fwd_host_variant", "sage_quant_qk_fp4", "sage_quant_v_fp4",
+                  "sage_attn_fwd_fp4_quantized", "sage_attn_fwd_fp4"):
             getattr(lib, n).restype = _i
         _lib = lib
     return _lib
@@ -344,19 +346,26 @@ def _host_ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+SAGE_VARIANT_FP16PV, SAGE_VARIANT_FP8PV, SAGE_VARIANT_FP4 = 0, 1, 2
+_VARIANT_CODES = {"fp16pv": SAGE_VARIANT_FP16PV, "fp8pv": SAGE_VARIANT_FP8PV, "fp4": SAGE_VARIANT_FP4}
+
+
 def sage_attn_fwd_host(q, k, v, o, causal: bool, sm_scale: float, granularity: int, heads_per_chunk: int = 0,
-                       stream=None) -> None:
+                       stream=None, variant: str = "fp16pv") -> None:
     """Whole forward pass on HOST tensors [B, H, N, d] (fp16): copies in, compute and copies
-    out overlap across chunks of heads.  Asynchronous on `stream` (the current CUDA stream by
-    default): synchronize it before reading o or changing q, k, v."""
+    out overlap across chunks of heads.  variant: "fp16pv" (the method), "fp8pv" or "fp4".
+    Asynchronous on `stream` (the current CUDA stream by default): synchronize it before reading
+    o or changing q, k, v."""
+    if variant not in _VARIANT_CODES:
+        raise ValueError(f"variant must be one of {tuple(_VARIANT_CODES)}, not {variant!r}")
     B, H, N, d = _shape(q)
     for t in (k, v, o):
         if tuple(t.shape) != (B, H, N, d):
             raise ValueError("q, k, v, o must have the same shape")
-    _check(get_lib().sage_attn_fwd_host(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(o), B, H, N, d,
-                                        int(bool(causal)), float(sm_scale), int(granularity), int(heads_per_chunk),
-                                        _stream(stream)),
-           "sage_attn_fwd_host")
+    _check(get_lib().sage_attn_fwd_host_variant(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(o), B, H, N, d,
+                                                int(bool(causal)), float(sm_scale), int(granularity),
+                                                int(heads_per_chunk), _VARIANT_CODES[variant], _stream(stream)),
+           "sage_attn_fwd_host_variant")
 
 
 def sage_noalloc_scratch_bytes(B: int, H: int, N: int, d: int, granularity: int) -> int:

@@ -1,5 +1,6 @@
-// host_pipeline.cu -- sage_attn_fwd_host: the whole forward pass for Q, K, V and O in host
-// memory, with the host<->device copies overlapped with the compute.
+// host_pipeline.cu -- sage_attn_fwd_host(_variant): the whole forward pass (the method, or its
+// FP8 P.V or FP4 variant) for Q, K, V and O in host memory, with the host<->device copies
+// overlapped with the compute.
 //
 // Heads are independent problems (the K mean, the scales and the attention of a (b,h) use
 // that head's tokens only), so the B*H heads are cut into chunks of consecutive heads, each a
@@ -84,14 +85,18 @@ Slot carve(uint8_t* base, int hc, int N, int d, int granularity) {
 
 extern "C" {
 
-int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
-                       float sm_scale, int granularity, int heads_per_chunk, void* stream) {
+int sage_attn_fwd_host_variant(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d,
+                               int causal, float sm_scale, int granularity, int heads_per_chunk, int variant,
+                               void* stream) {
   if (!q || !k || !v || !o) return SAGE_ERR_INVALID;
+  if (variant != SAGE_VARIANT_FP16PV && variant != SAGE_VARIANT_FP8PV && variant != SAGE_VARIANT_FP4)
+    return SAGE_ERR_INVALID;
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return SAGE_ERR_INVALID;
   if (granularity != SAGE_PER_TOKEN && granularity != SAGE_PER_BLOCK) return SAGE_ERR_INVALID;
   if (!(sm_scale > 0.f) || sm_scale > 3.4e38f) return SAGE_ERR_INVALID;  // also rejects NaN and inf
   if (heads_per_chunk < 0) return SAGE_ERR_INVALID;
   if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (variant == SAGE_VARIANT_FP8PV && d != 128) return SAGE_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N * d >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
   const int BH = B * H;
   // default: sixteen chunks, at least one head each (measured at B*H = 64, N = 16384, d = 128:
@@ -149,9 +154,15 @@ int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int
     }
     // the slot's output buffer must have been copied out before this chunk's kernels write it
     if (c >= n_slots && cudaStreamWaitEvent(st, ev_out[i], 0) != cudaSuccess) { rc = SAGE_ERR_CUDA; break; }
-    rc = sage_smooth_k(s.k, s.km, 1, hn, N, d, st);
-    if (!rc) rc = sage_quant_qk(s.q, s.k, s.km, s.q8, s.k8, s.sq, s.sk, 1, hn, N, d, granularity, st);
-    if (!rc) rc = sage_attn_fwd_quantized(s.q8, s.k8, s.sq, s.sk, s.v, s.o, 1, hn, N, d, causal, sm_scale, granularity, st);
+    if (variant == SAGE_VARIANT_FP4) {
+      rc = sage_attn_fwd_fp4(s.q, s.k, s.v, s.o, 1, hn, N, d, causal, sm_scale, st);
+    } else if (variant == SAGE_VARIANT_FP8PV) {
+      rc = sage_attn_fwd_fp8pv(s.q, s.k, s.v, s.o, 1, hn, N, d, causal, sm_scale, granularity, st);
+    } else {
+      rc = sage_smooth_k(s.k, s.km, 1, hn, N, d, st);
+      if (!rc) rc = sage_quant_qk(s.q, s.k, s.km, s.q8, s.k8, s.sq, s.sk, 1, hn, N, d, granularity, st);
+      if (!rc) rc = sage_attn_fwd_quantized(s.q8, s.k8, s.sq, s.sk, s.v, s.o, 1, hn, N, d, causal, sm_scale, granularity, st);
+    }
     if (rc) break;
     if (cudaEventRecord(ev_done[i], st) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_done[i], 0) != cudaSuccess ||
         cudaMemcpyAsync(ho + off, s.o, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
@@ -184,6 +195,12 @@ int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int
   if (cudaFreeAsync(ws, st) != cudaSuccess && !rc) rc = SAGE_ERR_CUDA;
   if (rc == SAGE_ERR_CUDA) cudaGetLastError();
   return rc;
+}
+
+int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int d, int causal,
+                       float sm_scale, int granularity, int heads_per_chunk, void* stream) {
+  return sage_attn_fwd_host_variant(q, k, v, o, B, H, N, d, causal, sm_scale, granularity, heads_per_chunk,
+                                    SAGE_VARIANT_FP16PV, stream);
 }
 
 }  // extern "C"

@@ -140,6 +140,12 @@ def test_host_pipeline_validation(sa):
     assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 0, 64, 0, 0.1, 1, 0, s) == -1    # N
     assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 64, 0, float("nan"), 1, 0, s) == -1
     assert L.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 64, 0, 0.1, 5, 0, s) == -1  # granularity
+    V = L.sage_attn_fwd_host_variant
+    assert V(FAKE, FAKE, FAKE, FAKE, *ok_args, 0, 3, s) == -1                            # unknown variant
+    assert V(FAKE, FAKE, FAKE, FAKE, *ok_args, 0, -1, s) == -1
+    assert V(FAKE, FAKE, FAKE, FAKE, *ok_args, 0, sa.SAGE_VARIANT_FP8PV, s) == -2       # FP8 P.V: d = 128 only
+    assert V(FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 96, 0, 0.1, 1, 0, sa.SAGE_VARIANT_FP4, s) == -2
+    assert V(FAKE, FAKE, FAKE, None, *ok_args, 0, sa.SAGE_VARIANT_FP4, s) == -1
 
 
 def test_binding_rejects_cpu_tensors(sa):

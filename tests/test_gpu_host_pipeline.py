@@ -1,7 +1,8 @@
-"""sage_attn_fwd_host: host tensors in, host tensor out, copies overlapped with the compute
-across chunks of heads.  Its output must equal sage_attn_fwd on the same tensors bit for bit
-(each head is an independent problem running the same kernels), for any chunking, pinned or
-pageable host memory, ragged N and both head dimensions."""
+"""sage_attn_fwd_host(_variant): host tensors in, host tensor out, copies overlapped with the
+compute across chunks of heads.  Its output must equal the device entry point of the same
+method or variant on the same tensors bit for bit (each head is an independent problem running
+the same kernels), for any chunking, pinned or pageable host memory, ragged N and both head
+dimensions."""
 import numpy as np
 import pytest
 import torch
@@ -59,3 +60,29 @@ def test_host_pipeline_on_a_side_stream_then_reuse(sa):
     assert sa.sage_last_device_error(s) == 0
     np.testing.assert_array_equal(o1.numpy().view(np.uint16), o2.numpy().view(np.uint16))
     assert np.isfinite(o1.float().numpy()).all()
+
+
+VARIANT_CASES = [
+    # variant, workload, heads_per_chunk
+    ("fp4", W.Workload("host_fp4_b1h5_n300_d128", 1, 5, 300, 128, False, True, n_out=4, out_mag=20.0), 2),
+    ("fp4", W.Workload("host_fp4_b2h3_n200_d64_causal", 2, 3, 200, 64, True, True, bias_std=4.0), 0),
+    ("fp8pv", W.Workload("host_fp8_b1h4_n384_d128_causal", 1, 4, 384, 128, True, True, n_out=4, out_mag=20.0), 3),
+]
+
+
+@pytest.mark.parametrize("variant,w,hpc", VARIANT_CASES, ids=lambda x: x if isinstance(x, str) else str(x))
+def test_host_pipeline_variants_match_their_device_entries(sa, variant, w, hpc):
+    q, k, v = W.make_qkv(w)
+    ref = torch.empty_like(v.cuda())
+    if variant == "fp4":
+        sa.sage_attn_fwd_fp4(q.cuda(), k.cuda(), v.cuda(), ref, w.causal, w.sm_scale)
+    else:
+        sa.sage_attn_fwd_fp8pv(q.cuda(), k.cuda(), v.cuda(), ref, w.causal, w.sm_scale, sa.SAGE_PER_BLOCK)
+    q, k, v = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o = torch.full_like(q, float("nan")).pin_memory()
+    st = torch.cuda.current_stream()
+    sa.sage_attn_fwd_host(q, k, v, o, w.causal, w.sm_scale, sa.SAGE_PER_BLOCK, heads_per_chunk=hpc, stream=st,
+                          variant=variant)
+    st.synchronize()
+    assert sa.sage_last_device_error(st) == 0
+    np.testing.assert_array_equal(o.numpy().view(np.uint16), ref.cpu().numpy().view(np.uint16))
