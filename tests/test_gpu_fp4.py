@@ -207,7 +207,8 @@ def test_fp4_without_v_smoothing(sa):
     check_o(o.float().cpu().numpy(), o64, env, unsure, vhat_max(ref), "no V smoothing")
 
 
-@pytest.mark.parametrize("w", [W.HEADLINE, W.SPARSE, W.SPARSE_DIT], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [W.HEADLINE, W.SPARSE, W.SPARSE_DIT, W.LLM, W.DIT, W.SPARSE_CAUSAL],
+                         ids=lambda w: w.name)
 def test_fp4_full_size_sampled_rows(sa, w):
     q, k, v = W.make_qkv(w)
     o = torch.empty_like(q, device="cuda")
@@ -215,7 +216,8 @@ def test_fp4_full_size_sampled_rows(sa, w):
     torch.cuda.synchronize()
     assert sa.sage_last_device_error() == 0
     og = o.view(w.BH, w.N, w.d).float().cpu().numpy()
-    rows = np.array([0, 1, 127, 128, 5000, 8191, 12345, w.N - 1])
+    # first rows, tile edges, the causal diagonal's 64-key halves, a middle row and the last one
+    rows = np.unique(np.clip(np.array([0, 1, 63, 64, 127, 128, 2047, 4095, 5000, 8191, 12345, w.N - 1]), 0, w.N - 1))
     for h in (0, w.BH // 2, w.BH - 1):
         qh, kh, vh = (x.view(w.BH, w.N, w.d)[h:h + 1] for x in (q, k, v))
         km = oracle.smooth_k(kh)
