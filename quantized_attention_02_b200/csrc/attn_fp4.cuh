@@ -275,12 +275,15 @@ __global__ void __launch_bounds__(192, 2)
       const float m_e = m_use - 10.f;  // p = 2^(S * cb - m + 10); exact: m is an integer
       uint32_t w[8];
       uint32_t sfw = 0u;
+      // the tile's codes in three phases over all 64 keys (the four group scales, every exponent
+      // argument and exponential, then the row sums and codes), so that each result is consumed
+      // well after it is produced.  Group scale: the exp2 of the group's largest score (rounded as
+      // in phase 2); the codes' operand p / scale is exp2(S * cb - m + 10 - log2 scale), and the
+      // row sum adds z * scale = p.  A zero scale (all p of the group below 6 * 2^-10) keeps
+      // z = p, whose codes round to zero.  Phase 1:
+      float nbv[4], sev[4];
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) {
-        // group scale from the group's largest p, the exp2 of its largest score (fl(S * cb - m + 10)
-        // rounds as in the pass below); then the codes' operand z = p / scale directly as
-        // exp2(S * cb - m + 10 - log2 scale), and p = z * scale for the row sum.  A zero scale (all
-        // p of the group below 6 * 2^-10) keeps z = p, whose codes round to zero.
         const float gm = fast_exp2(fmaf(gs[gi], cb, -m_e));
         const uint32_t s8 = e4m3_code(__fmul_rn(gm, 0.16666667163372040f));
         float nb = -m_e, se = 1.f;
@@ -288,22 +291,38 @@ __global__ void __launch_bounds__(192, 2)
           se = e4m3_value(s8);
           nb = -__fadd_rn(m_e, fast_log2(se));
         }
-        float y[16];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c = 16 * gi + 2 * k;
-          const float2 tt = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])),
-                                       make_float2(cb, cb), make_float2(nb, nb));
-          // one pair in four on the FMA pipe (exp2_poly2, relative error <= 7.5e-5), the rest on
-          // the MUFU unit; masked keys: exp2(-inf) = 0 (the polynomial gives 2^-126)
-          const float2 z = (k & 3) == 3 ? exp2_poly2(tt) : make_float2(fast_exp2(tt.x), fast_exp2(tt.y));
-          lsum[k & 3] = __ffma2_rn(z, make_float2(se, se), lsum[k & 3]);
-          y[2 * k] = z.x;
-          y[2 * k + 1] = z.y;
-        }
-        w[2 * gi] = e2m1x8(y);
-        w[2 * gi + 1] = e2m1x8(y + 8);
+        nbv[gi] = nb;
+        sev[gi] = se;
         sfw |= s8 << (8 * gi);
+      }
+      // phase 2: every exponent argument, then every exponential (one pair in four on the FMA
+      // pipe, exp2_poly2, relative error <= 7.5e-5; the rest on the MUFU unit; masked keys give
+      // exp2(-inf) = 0, the polynomial 2^-126)
+      float2 zz[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float nb = nbv[i >> 3];
+        zz[i] = __ffma2_rn(make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), make_float2(cb, cb),
+                           make_float2(nb, nb));
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        zz[i] = (i & 3) == 3 ? exp2_poly2(zz[i]) : make_float2(fast_exp2(zz[i].x), fast_exp2(zz[i].y));
+      // phase 3: row sums and codes
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float se = sev[i >> 3];
+        lsum[i & 3] = __ffma2_rn(zz[i], make_float2(se, se), lsum[i & 3]);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          y[2 * k] = zz[4 * q4 + k].x;
+          y[2 * k + 1] = zz[4 * q4 + k].y;
+        }
+        w[q4] = e2m1x8(y);
       }
       // P~.V(j-1) must be complete before O is rescaled and before P~(j) overwrites P~(j-1): the
       // codes above are computed in registers while it runs
