@@ -395,16 +395,19 @@ def empty_quantized(q: torch.Tensor, granularity: int):
     return km, q8, k8, sq, sk
 
 
-VARIANTS = ("fp16pv", "fp8pv", "fp4")
+VARIANTS = ("fp16pv", "fp8pv", "fp4", "sparse")
 
 
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              sm_scale: float | None = None, granularity: int = SAGE_PER_BLOCK, variant: str = "fp16pv",
-             stream=None) -> torch.Tensor:
+             stream=None, tau: float = 0.99, theta: float = 0.3, skip_lambda: float = 20.0) -> torch.Tensor:
     """O = softmax(Q K^T sm_scale) V on fp16 [B, H, N, d] CUDA tensors; sm_scale defaults to d^-1/2.
     variant: "fp16pv" the method (smoothed K, INT8 Q K^T with per-token or per-block scales, FP16 P V);
     "fp8pv" its FP8 P~ V variant (E4M3 P~ and smoothed V; d = 128); "fp4" the microscaling FP4 variant
-    (E2M1 Q, K, P~, V with UE4M3 scales per 16 elements; granularity does not apply)."""
+    (E2M1 Q, K, P~, V with UE4M3 scales per 16 elements; granularity does not apply); "sparse" the
+    block-sparse variant (stage 1 keeps the key blocks reaching cumulative probability tau, theta the
+    self-similarity below which a block is always kept; stage 2 drops a block whose scores all lie
+    skip_lambda log2 units below the running row maximum; N <= 65536)."""
     if variant not in VARIANTS:
         raise ValueError(f"variant must be one of {VARIANTS}, not {variant!r}")
     if sm_scale is None:
@@ -412,6 +415,8 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     o = torch.empty_like(q)
     if variant == "fp4":
         sage_attn_fwd_fp4(q, k, v, o, causal, sm_scale, stream)
+    elif variant == "sparse":
+        sage_attn_fwd_sparse(q, k, v, o, causal, sm_scale, granularity, tau, theta, skip_lambda, stream)
     elif variant == "fp8pv":
         sage_attn_fwd_fp8pv(q, k, v, o, causal, sm_scale, granularity, stream)
     else:

@@ -263,6 +263,8 @@ def test_sageattn_variants_match_their_entry_points(sa, d):
     q, k, v = (x.cuda() for x in W.make_qkv(w))
     calls = [("fp16pv", lambda o: sa.sage_attn_fwd(q, k, v, o, True, w.sm_scale, sa.SAGE_PER_BLOCK)),
              ("fp4", lambda o: sa.sage_attn_fwd_fp4(q, k, v, o, True, w.sm_scale))]
+    calls.append(("sparse", lambda o: sa.sage_attn_fwd_sparse(q, k, v, o, True, w.sm_scale, sa.SAGE_PER_BLOCK,
+                                                              0.99, 0.3, 20.0)))
     if d == 128:
         calls.append(("fp8pv", lambda o: sa.sage_attn_fwd_fp8pv(q, k, v, o, True, w.sm_scale, sa.SAGE_PER_BLOCK)))
     for variant, direct in calls:
