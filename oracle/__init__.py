@@ -402,7 +402,7 @@ def sage_attn_fp8pv(q, k, v, causal: bool, sm_scale: float, per_block: bool, smo
 
 
 # ------------------------------------------------------------------ microscaling FP4 variant
-# (SageAttention3 abstract: attention on FP4 tensor cores with microscaling; readings in
+# (SageAttention3 entry: microscaling FP4 attention on FP4 tensor cores; readings in
 # sage_oracle_sa3.c)
 FP4_TILE, FP4_GROUP = 128, 16
 

@@ -218,7 +218,7 @@ def empty_fp4(q, smooth_v: bool = True) -> dict:
 
 def sage_quant_qk_fp4(q, k, km, q4, sfq, gq, k4, sfk, gk, stream=None) -> None:
     """Q and K (minus km unless None) to E2M1 codes with UE4M3 scale atoms and fp32 tile scales
-    (microscaling FP4 variant, SageAttention3 abstract)."""
+    (microscaling FP4 variant, SageAttention3 entry: title and abstract)."""
     B, H, N, d = _shape(q)
     _check(get_lib().sage_quant_qk_fp4(_ptr(q), _ptr(k), _ptr(km), _ptr(q4), _ptr(sfq), _ptr(gq), _ptr(k4), _ptr(sfk),
                                        _ptr(gk), B, H, N, d, _stream(stream)), "sage_quant_qk_fp4")

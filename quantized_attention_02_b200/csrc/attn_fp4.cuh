@@ -1,7 +1,7 @@
 // attn_fp4.cuh -- the fused attention kernel of the microscaling FP4 variant (included by
 // attn_kernels.cu, after the head-dimension-128 kernel whose helpers it uses).
 //
-// Method (SageAttention3 abstract: attention on Blackwell's FP4 tensor cores with microscaling;
+// Method (SageAttention3 entry: microscaling FP4 attention on Blackwell's FP4 tensor cores;
 // the readings are the oracle's, oracle/sage_oracle_sa3.c):
 //   S   = Q4 . K4^T              E2M1 x E2M1 with one UE4M3 scale per 16 channels
 //                                (tcgen05 kind::mxf4nvf4 block16), fp32 in tensor memory

@@ -1,7 +1,7 @@
 // fp4_codes.cuh -- E2M1 / E4M3 conversions and the microscaling of one group of 16 values,
 // used by the FP4 quantization kernels (the conversions also by the FP4 attention kernel).
 //
-// Microscaling (SageAttention3 abstract: FP4 attention with microscaling; the format is the
+// Microscaling (SageAttention3 entry: microscaling FP4 attention; the format is the
 // one Blackwell's block-scaled FP4 products read): one UE4M3 scale per 16 elements along the
 // contraction dimension, e4m3(fl32(max|z| / 6)); codes e2m1(fl32(z * fl32(1 / scale))), a zero
 // scale giving zero codes.

@@ -761,7 +761,7 @@ cudaError_t launch_quant_qk(const __half* q, const __half* k, const float* km, i
 }
 
 // ---------------------------------------------------------------- microscaling FP4 variant
-// (SageAttention3 abstract: attention on FP4 tensor cores with microscaling).  Formats: E2M1
+// (SageAttention3 entry: microscaling FP4 attention on Blackwell's FP4 tensor cores).  Formats: E2M1
 // codes, two per byte (the even element in the low nibble), one UE4M3 scale per 16 elements
 // along the contraction dimension, chosen as e4m3(fl32(max|z| / 6)), codes
 // e2m1(fl32(z * fl32(1 / scale))).  Scales are stored in the tensor cores' scale atoms: 512 bytes

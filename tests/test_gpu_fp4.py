@@ -1,4 +1,4 @@
-"""GPU parity of the microscaling FP4 variant (SageAttention3 abstract: both products of the
+"""GPU parity of the microscaling FP4 variant (SageAttention3 entry: both products of the
 attention on FP4 tensor cores with microscaling) through the C ABI, against
 oracle/sage_oracle_sa3.c.
 

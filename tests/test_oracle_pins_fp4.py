@@ -4,8 +4,8 @@ brute-force nearest-value search, the format's extremes, hand-derived rows
 (tests/golden/fp4_online_frames.json) and an error bound against textbook attention on the
 dequantized inputs.
 
-The variant follows the SageAttention3 abstract (attention on FP4 tensor cores with
-microscaling); its open points are the readings written at the top of sage_oracle_sa3.c.
+The variant follows the SageAttention3 entry (microscaling FP4 attention on FP4 tensor cores); its
+open points are the readings written at the top of sage_oracle_sa3.c.
 tests/test_oracle_mutations.py plants slips in that file and checks that this file fails on
 each of them.
 """
