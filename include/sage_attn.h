@@ -108,7 +108,7 @@ int sage_attn_fwd_quantized(const int8_t* q8, const int8_t* k8, const float* sq,
 
 /* ---------------------------------------------------------------------------------------
  * FP8 P.V variant, following the SageAttention2 abstract (author pages of Jia Wei and Haofeng
- * Huang; arXiv 2411.10958): the matrices (P~, V) are quantized to FP8, V is smoothed, and P~V is
+ * Huang): the matrices (P~, V) are quantized to FP8, V is smoothed, and P~V is
  * accumulated in an FP32 buffer.  Q.K^T stays the INT8 product above (the abstract's INT4 Q.K^T
  * is not part of this variant).  FP8 is E4M3 (bias 7, largest finite 448), round to nearest
  * even, saturating.  Head dimension 128 only (d = 64 returns SAGE_ERR_UNSUPPORTED).
@@ -140,7 +140,7 @@ int sage_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* o, in
 
 /* ---------------------------------------------------------------------------------------
  * Block-sparse variant, following the SpargeAttn abstract (author pages of Jia Wei and Haofeng
- * Huang; arXiv 2502.18137): a sparse and quantized attention with a two-stage online filter.
+ * Huang): a sparse and quantized attention with a two-stage online filter.
  * Stage 1 predicts the attention map at block level and skips the products of the blocks it
  * drops; stage 2, inside the online softmax, skips the P.V product (and the exp2 work) of a block
  * whose scores all lie far below the running row maximum.  Head dimension 64 or 128 and
@@ -181,7 +181,7 @@ int sage_attn_fwd_sparse(const void* q, const void* k, const void* v, void* o, i
 
 /* ---------------------------------------------------------------------------------------
  * Microscaling FP4 variant, following the SageAttention3 abstract (author pages of Jia Wei and
- * Haofeng Huang; arXiv 2505.11594): both products of the attention run on Blackwell's FP4 tensor
+ * Haofeng Huang): both products of the attention run on Blackwell's FP4 tensor
  * cores (tcgen05 kind::mxf4nvf4, block16) with microscaling.  Head dimension d = 64 or 128.
  * Formats: E2M1 codes (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their
  * negatives), two per byte with the even element in the low nibble; one UE4M3 scale per 16

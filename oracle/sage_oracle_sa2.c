@@ -7,7 +7,7 @@
  *
  * What it computes follows the SageAttention2 abstract ("SageAttention2: Efficient Attention
  * with Thorough Outlier Smoothing and Per-thread INT4 Quantization", author pages of Jia Wei
- * and Haofeng Huang; and its arXiv 2411.10958 abstract): the matrices (P~, V) are quantized to
+ * and Haofeng Huang): the matrices (P~, V) are quantized to
  * FP8, V (and Q) are smoothed, and P~V is accumulated in an FP32 buffer.  Q.K^T stays the
  * INT8 product of sage_oracle.c (smoothed K, absmax INT8 Q and K): the INT4 Q.K^T of that
  * abstract is not part of this variant.  The abstract leaves the formats open; the readings:

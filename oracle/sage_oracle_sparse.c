@@ -7,7 +7,7 @@
  *
  * What it computes follows the SpargeAttn abstract ("SpargeAttention: Accurate and Training-
  * free Sparse Attention Accelerating Any Model Inference", author pages of Jia Wei and Haofeng
- * Huang; arXiv 2502.18137): a sparse and quantized attention with a two-stage online filter --
+ * Huang): a sparse and quantized attention with a two-stage online filter --
  * the first stage predicts the attention map quickly, so that some matrix products are skipped;
  * the second, a softmax-aware filter inside the online softmax, skips further products.  The
  * abstract gives no formulas; the readings:
