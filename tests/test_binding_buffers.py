@@ -42,3 +42,12 @@ def test_sageattn_rejects_an_unknown_variant():
     q = torch.zeros((1, 1, 128, 64), dtype=torch.float16)
     with pytest.raises(ValueError):
         sa.sageattn(q, q, q, variant="int4")
+
+
+def test_binding_constants_match_the_header():
+    import re
+    text = open(sa.HEADER_PATH).read()
+    consts = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(SAGE_[A-Z0-9_]+)\s*=\s*(-?\d+)", text)}
+    for name in ("SAGE_PER_TOKEN", "SAGE_PER_BLOCK", "SAGE_VARIANT_FP16PV", "SAGE_VARIANT_FP8PV", "SAGE_VARIANT_FP4",
+                 "SAGE_OK", "SAGE_ERR_INVALID", "SAGE_ERR_UNSUPPORTED"):
+        assert getattr(sa, name) == consts[name], name
